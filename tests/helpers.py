@@ -52,6 +52,9 @@ def oracle_prefill(q, k, v, g, beta, cu_seqlens, h0, scale=1.0, heads=None, form
 
 def assert_prefill_close(o_gpu, hT_gpu, o_ref, hT_ref, what=""):
     e_o, a_o = rel_frob(o_gpu, o_ref), max_abs(o_gpu, o_ref)
+    if hT_ref is not None:
+        print(f"[parity] {what}: o rel_frob={e_o:.2e} max_abs={a_o:.2e}; hT rel_frob="
+              f"{rel_frob(hT_gpu, hT_ref):.2e} max_abs={max_abs(hT_gpu, hT_ref):.2e}")
     assert e_o <= PREFILL_REL_FROB and a_o <= PREFILL_MAX_ABS, \
         f"{what} o: rel_frob={e_o:.3e} max_abs={a_o:.3e}"
     if hT_ref is not None:
