@@ -152,6 +152,38 @@ int gdn_verify_woa(float* const* h_table, const uint16_t* q, const uint16_t* k, 
                    gdn_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * gdn_verify_woa_static -- gdn_verify_woa without a caller-provided stash.
+ * No counterpart on the source pages: this entry point exists for callers
+ * that cannot allocate device memory themselves -- for example an engine that
+ * reserves all device memory up front in its own pool and forbids further
+ * allocations while serving, or a latency-bound decode loop that must not
+ * call cudaMalloc (which can synchronise the whole device).  Such a caller
+ * still passes every input and output; only the stash (the scratch the verify
+ * leaves for the fold) lives in the library.
+ *
+ * The stash is a static device array of GDN_STATIC_STASH_FLOATS f32 (8 MiB)
+ * that every GPU loading this library holds until the process exits.
+ * Sequence b uses floats [b * S, (b + 1) * S) with
+ * S = gdn_stash_seq_floats(H_v, d_k, d_v); batch * S must not exceed
+ * GDN_STATIC_STASH_FLOATS (GDN_ERR_SHAPE otherwise).  On success
+ * *stash_out receives the array's device address: pass it, with
+ * stash_seq_floats = S, to gdn_fold.  The first call on each device looks that
+ * address up (cudaGetSymbolAddress, with the device current); make that first
+ * call before any stream capture.  Nothing is allocated or freed, by this call
+ * or by anything it calls.  All calls share the one array and it keeps the
+ * last call's contents: a verify whose fold has not yet run must not be
+ * followed by another static verify, and calls that overlap on the GPU (other
+ * streams, other host threads) race on it.  Every other argument, guard and
+ * error is as for gdn_verify_woa; stash_out must not be NULL.
+ * ------------------------------------------------------------------------ */
+#define GDN_STATIC_STASH_FLOATS (2u * 1024u * 1024u)
+int gdn_verify_woa_static(float* const* h_table, const uint16_t* q, const uint16_t* k,
+                          int qk_stride, const uint16_t* v, int v_stride, const float* g,
+                          const float* beta, int gb_stride, uint16_t* o, int batch, int H_k,
+                          int H_v, int d_k, int d_v, float scale, uint32_t* engaged_flag,
+                          const float** stash_out, gdn_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * gdn_fold -- the post-verdict fold.
  * Page "ssm_gdn_woa.rs", gdn_wy4_fold: when the engaged word is set it applies
  * the stashed rows 0..na_tab[b] to H, reading and writing each touched state

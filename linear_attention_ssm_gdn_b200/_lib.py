@@ -41,6 +41,8 @@ SIGNATURES = {
     "gdn_stash_seq_floats": (_I, [_I, _I, _I]),
     "gdn_verify_woa": (_I, [_P, _P, _P, _I, _P, _I, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I,
                             _F, _P, _P]),
+    "gdn_verify_woa_static": (_I, [_P, _P, _P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I,
+                                   _F, _P, _P, _P]),
     "gdn_fold": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     "gdn_flag_clear": (_I, [_P, _P]),
     "gdn_debug_device_errors": (_I, [_P]),

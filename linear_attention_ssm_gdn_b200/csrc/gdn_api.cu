@@ -233,6 +233,41 @@ int gdn_verify_woa(float* const* h_table, const uint16_t* q, const uint16_t* k, 
                      fn);
 }
 
+int gdn_verify_woa_static(float* const* h_table, const uint16_t* q, const uint16_t* k,
+                          int qk_stride, const uint16_t* v, int v_stride, const float* g,
+                          const float* beta, int gb_stride, uint16_t* o, int batch, int H_k,
+                          int H_v, int d_k, int d_v, float scale, uint32_t* engaged_flag,
+                          const float** stash_out, gdn_stream_t stream) {
+  const char* fn = "gdn_verify_woa_static";
+  if (!stash_out) return fail(GDN_ERR_NULL, "gdn_verify_woa_static: null stash_out");
+  if (!h_table || !engaged_flag)
+    return fail(GDN_ERR_NULL, "gdn_verify_woa_static: null table/flag");
+  if (!q || !k || !v || !g || !beta || !o)
+    return fail(GDN_ERR_NULL, "gdn_verify_woa_static: null q/k/v/g/beta/o");
+  int rc = check_heads(fn, H_k, H_v, d_k, d_v);
+  if (rc != GDN_OK) return rc;
+  if (batch < 0) return fail(GDN_ERR_SHAPE, "gdn_verify_woa_static: batch < 0");
+  if (qk_stride < H_k * d_k || v_stride < H_v * d_v || gb_stride < H_v)
+    return fail(GDN_ERR_STRIDE, "gdn_verify_woa_static: a stride is shorter than its row");
+  const int ssf = gdn_stash_seq_floats(H_v, d_k, d_v);
+  if (size_t(batch) * size_t(ssf) > gdn::static_stash_floats())
+    return fail(GDN_ERR_SHAPE,
+                "gdn_verify_woa_static: batch * gdn_stash_seq_floats() exceeds the static stash "
+                "(GDN_STATIC_STASH_FLOATS = 2 Mi floats, 8 MiB)");
+  float* stash = nullptr;
+  cudaError_t e = gdn::static_stash_address(&stash);
+  if (e != cudaSuccess) return cuda_status(e, fn);
+  *stash_out = stash;
+  if (batch == 0) {
+    gdn::clear_error();
+    return GDN_OK;
+  }
+  return cuda_status(gdn::launch_verify(h_table, q, k, qk_stride, v, v_stride, g, beta, gb_stride,
+                                        o, stash, ssf, batch, H_k, H_v, d_k, scale, engaged_flag,
+                                        reinterpret_cast<cudaStream_t>(stream)),
+                     fn);
+}
+
 int gdn_fold(float* const* h_table, const float* stash, const int32_t* na_tab,
              const uint16_t* k, int qk_stride, uint32_t* engaged_flag, int k_rows, int batch,
              int H_k, int H_v, int d_k, int d_v, int stash_seq_floats, gdn_stream_t stream) {

@@ -39,6 +39,11 @@ cudaError_t launch_verify(float* const* h_table, const uint16_t* q, const uint16
                           int stash_seq_floats, int batch, int H_k, int H_v, int D, float scale,
                           uint32_t* flag, cudaStream_t s);
 
+// Device address of the library-owned verify stash on the current device
+// (looked up once per device); nullptr and the error on failure.
+cudaError_t static_stash_address(float** out);
+size_t static_stash_floats();
+
 cudaError_t launch_fold(float* const* h_table, const float* stash, const int32_t* na_tab,
                         const uint16_t* k, int qk_stride, uint32_t* flag, int k_rows,
                         int batch, int H_k, int H_v, int D, int stash_seq_floats,

@@ -22,12 +22,19 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "gdn_device.cuh"
 #include "gdn_internal.h"
 
 namespace gdn {
 
 __device__ uint32_t g_err_verify;
+
+// The verify stash for callers that cannot allocate (gdn_verify_woa_static):
+// 2 Mi floats = 8 MiB, held by every device that loads the library.
+constexpr size_t kStaticStashFloats = size_t(2) * 1024 * 1024;
+static __device__ __align__(256) float g_static_stash[kStaticStashFloats];
 
 constexpr uint32_t kFlagEngaged = 1u;
 constexpr uint32_t kFlagError = 2u;
@@ -244,6 +251,29 @@ cudaError_t launch_fold(float* const* h_table, const float* stash, const int32_t
     fold_kernel<64><<<grid, 128, 0, s>>>(h_table, stash, na_tab, k, qk_stride, flag, H_k, H_v,
                                          stash_seq_floats);
   return cudaGetLastError();
+}
+
+size_t static_stash_floats() { return kStaticStashFloats; }
+
+// In host code g_static_stash names a host-side stand-in, not device memory,
+// so its device address is looked up once per device (with that device
+// current) and cached.
+cudaError_t static_stash_address(float** out) {
+  static std::mutex mu;
+  static float* cache[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == nullptr) {
+    float* ptr = nullptr;
+    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_static_stash);
+    if (e != cudaSuccess) return e;
+    cache[dev] = ptr;
+  }
+  *out = cache[dev];
+  return cudaSuccess;
 }
 
 // Read and clear this file's device error word (host; synchronous).
