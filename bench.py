@@ -137,7 +137,8 @@ class ClockSampler:
 def make_inputs(dev):
     import torch
 
-    from linear_attention_ssm_gdn_b200 import gdn_stash_seq_floats
+    from linear_attention_ssm_gdn_b200 import (gdn_chunk_prefill_workspace_bytes,
+                                               gdn_stash_seq_floats)
     from linear_attention_ssm_gdn_b200 import inputs as I
 
     w2 = I.workload(2)
@@ -158,6 +159,8 @@ def make_inputs(dev):
     d["flag"] = torch.zeros(1, dtype=torch.int32, device=dev)
     d["vo"] = torch.empty(vi.batch * 4, vi.H_v, vi.d_v, dtype=torch.bfloat16, device=dev)
     d["stash"] = torch.empty(vi.batch, gdn_stash_seq_floats(vi.H_v, vi.d_k, vi.d_v), device=dev)
+    ws = gdn_chunk_prefill_workspace_bytes(T, p.num_seqs, p.H_k, H_v, p.d_k, dv)
+    d["ws"] = torch.empty(max(ws, 1), dtype=torch.uint8, device=dev)
     meta = dict(T=T, N=p.num_seqs, H_k=p.H_k, H_v=H_v, d_k=p.d_k, d_v=dv, nv=ba.nv,
                 vpg=ba.vheads_per_group, vbatch=vi.batch)
     return host, d, meta
@@ -174,7 +177,7 @@ def step_calls(d, meta, ev=None):
     if ev:
         ev[1].record()
     gdn_chunk_prefill(d["q"], d["k"], d["v"], d["gates"][:, :nv], d["gates"][:, nv:], d["cu"],
-                      h0=d["h0"], hT=d["hT"], o=d["o"])
+                      h0=d["h0"], hT=d["hT"], o=d["o"], workspace=d["ws"])
     if ev:
         ev[2].record()
     gdn_flag_clear(d["flag"])

@@ -71,8 +71,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for phase `parity` of `bar` to complete.  Gives up (returns false) when
 // *abort becomes nonzero or after kSpinLimitCycles; on a timeout it sets
 // *abort and ORs `err_bit` into *err (a global error word, may be null).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* err, uint32_t err_bit) {
+static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                       uint32_t* err, uint32_t err_bit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
@@ -325,6 +325,11 @@ __device__ __forceinline__ uint32_t cluster_id_x() {
   asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
   return r;
 }
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
 __device__ __forceinline__ uint32_t num_clusters_x() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
@@ -365,9 +370,9 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 }
 
 // Bounded wait with cluster-scope acquire (for barriers other CTAs arrive on).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort, uint32_t* err,
-                                                  uint32_t err_bit) {
+static __device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort, uint32_t* err,
+                                               uint32_t err_bit) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
@@ -390,6 +395,48 @@ __device__ __forceinline__ void fence_proxy_async_cluster() {
 __device__ __forceinline__ void cluster_sync_start() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
+}
+
+}  // namespace gdn
+
+// ---------------------------------------------------------------------------
+// Non-tensor bulk copies (cp.async.bulk), no multicast; and a non-blocking
+// mbarrier probe for threads that poll several barriers.
+// ---------------------------------------------------------------------------
+namespace gdn {
+
+// global -> this CTA's shared memory, completing `bytes` on `bar`.
+__device__ __forceinline__ void bulk_load_g2s(void* dst, const void* src, uint32_t bytes,
+                                              uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// this CTA's shared memory -> global (bulk-group completion).
+__device__ __forceinline__ void bulk_store_s2g(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(dst)),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 
 }  // namespace gdn

@@ -4,23 +4,23 @@
 // "state spine" (chunk_delta_h) that carries the f32 recurrent state across
 // chunks with bf16 tensor-core operands and an f32 accumulator.  Here the whole
 // chunk step is one kernel, and each (sequence, v-head) unit is handled by a
-// cluster of three CTAs on three SMs:
+// cluster of two or three CTAs on as many SMs:
 //
-//   rank 0, the SPINE: holds H (f32, registers) and runs the per-chunk critical
-//     chain  Vn^T = U^T - H^T W^T,  dH^T = (e^{G_C - G_r} Vn)^T K,
-//     H <- e^{G_C} H + dH,  and the outputs  o_r = e^{G_r} scale (Q H)_r +
-//     (Aqk Vn)_r  (tcgen05 MMAs, TMEM accumulators, M = d_v = 128 lanes);
-//   ranks 1 and 2, the PREPS: compute everything that does not depend on H for
-//     alternate chunks (rank 1 even chunks, rank 2 odd ones), two chunks at a
-//     time per CTA (one per 4-warp group):
+//   rank 0, the SPINE, runs the per-chunk critical chain on tcgen05 MMAs with
+//     TMEM accumulators (M = d_v = 128 lanes), keeping H^T in TMEM (f32):
+//       Vn^T = U^T - H^T W^T,   H^T <- e^{G_C} H^T + (e^{G_C - G_r} Vn)^T K,
+//     and the outputs  o_r = e^{G_r} scale (Q H)_r + (Aqk Vn)_r;
+//   ranks 1 (and 2), the PREPS, compute everything that does not depend on H,
+//     each for its share of the chunks, two chunks at a time per CTA:
 //       P1 = [K;Q] K^T                                 (MMA)
 //       A[r][s]   = beta_r e^{G_r-G_s} k_r.k_s, s < r   (f32)
 //       Aqk[r][s] = scale e^{G_r-G_s} q_r.k_s, s <= r
 //       T = (I + A)^{-1}                               (blocked, f32, CUDA cores)
 //       W^T = K^T (T diag(beta e^G))^T,  U^T = V^T (T diag(beta))^T   (MMAs)
-//     and store W^T, U^T, Aqk (bf16) and the gate factors straight into one of
-//     the spine's two shared-memory slots (distributed shared memory stores,
-//     then a remote mbarrier arrive).  The spine frees a slot the same way.
+//     and bulk-store W^T, U^T, Aqk (bf16) and the gate factors into a 4-entry
+//     ring in global memory (the workspace; it stays in L2), from where the
+//     spine's TMA warp bulk-loads them into one of two shared-memory slots.
+//     Hand-offs are mbarrier arrivals across the cluster.
 //
 // This is the WY/UT chunk form: within a chunk of rows r = 0..L-1 with
 // G_r = g_0 + ... + g_r, (I + A) Vn = diag(beta) V - diag(beta e^G) K H, the
@@ -30,8 +30,9 @@
 // d_k = d_v = 64 runs the same code with the upper halves of every tile zero.
 //
 // No TMA multicast: every CTA loads its own K/Q/V tiles (L2 serves re-reads).
-// Every wait is bounded (gdn_device.cuh); a timeout sets g_err_prefill and the
-// kernel returns instead of hanging.
+// Every mbarrier wait is bounded (gdn_device.cuh); a timeout sets
+// g_err_prefill and the kernel returns instead of hanging.  Named barriers are
+// used only among threads that are all guaranteed to arrive.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -47,35 +48,37 @@ namespace pf {
 
 constexpr int C = 64;          // chunk rows
 constexpr int kThreads = 320;  // 10 warps
-constexpr int kCluster = 3;    // spine + 2 preps
 constexpr int kAS = 68;        // f32 row stride of the A / T scratch (16-byte rows)
+
+// ---- global slot-ring entry (workspace): W^T | U^T | Aqk | gate factors
+constexpr uint32_t G_W = 0, G_U = 16384, G_AQK = 32768, G_GATE = 40960;
+constexpr uint32_t G_GATE_BYTES = 528;  // e^{G_r} 64 | e^{G_C-G_r} 64 | e^{G_C} | pad
+constexpr uint32_t SLOT_G = 41984;      // 41 KB, a multiple of 1024
+constexpr uint32_t SLOT_TX = G_GATE + G_GATE_BYTES;
+constexpr int kRing = 4;
 
 // ---- spine shared memory (bytes from a 1024-aligned base)
 constexpr uint32_t S_KQ = 0;            // [2 stages][2 boxes][K 64x128B | Q 64x128B]
 constexpr uint32_t S_HT = 65536;        // H^T bf16, [2 boxes][128 x 128B]
 constexpr uint32_t S_VN = 98304;        // Vn^T bf16 [128 x 128B]
 constexpr uint32_t S_VNS = 114688;      // scaled Vn^T bf16
-constexpr uint32_t S_OST = 131072;      // output staging [64 rows][d_v] bf16, row-major
-constexpr uint32_t S_SLOT = 147456;     // 2 slots of {W^T, U^T, Aqk}
-constexpr uint32_t SL_W = 0;            // W^T bf16 [128 (d_k) x 128B] (MN-major B operand)
-constexpr uint32_t SL_U = 16384;        // U^T bf16 [128 (d_v) x 128B] (swizzled rows)
-constexpr uint32_t SL_AQK = 32768;      // Aqk bf16 [64 x 128B] (K-major B operand)
+constexpr uint32_t S_SLOT = 131072;     // 2 slots of {W^T, U^T, Aqk}, same layout as G_*
 constexpr uint32_t SL_BYTES = 40960;
-constexpr uint32_t S_SGATE = S_SLOT + 2 * SL_BYTES;  // 2 x [e^{G_r} 64 | e^{G_C-G_r} 64 | e^{G_C}]
+constexpr uint32_t S_SGATE = S_SLOT + 2 * SL_BYTES;  // 2 x 528 B of gate factors
 constexpr uint32_t SG_FLOATS = 132;
-constexpr uint32_t S_BARS = S_SGATE + 2 * SG_FLOATS * 4;
+constexpr uint32_t S_BARS = S_SGATE + 2 * G_GATE_BYTES;
 // ---- prep shared memory: two item groups of P_WG bytes
 constexpr uint32_t P_KQ = 0;        // [2 boxes][K | Q]
 constexpr uint32_t P_V = 32768;     // [2 boxes][64 x 128B]
 constexpr uint32_t P_T1B = 49152;   // T diag(beta e^G) bf16 [64 x 128B]
 constexpr uint32_t P_T2B = 57344;   // T diag(beta) bf16
-constexpr uint32_t P_AF = 65536;    // A f32 [64][kAS]
+constexpr uint32_t P_AF = 65536;    // A f32 [64][kAS]; later the W^T | U^T staging
 constexpr uint32_t P_TF = P_AF + 64 * kAS * 4;  // T f32 [64][kAS]
-constexpr uint32_t P_XS = P_TF + 64 * kAS * 4;  // block-product scratch, 3 x 16 x 16 f32
-constexpr uint32_t P_GATE = P_XS + 3 * 256 * 4;
+constexpr uint32_t P_XS = P_T1B;    // inverse scratch (32x32 f32), in the T1/T2 tiles' space
+constexpr uint32_t P_GATE = P_TF + 64 * kAS * 4;
 constexpr int PG_G = 0, PG_BET = 64, PG_E1 = 128, PG_E2 = 192, PG_BEG = 448, PG_EG = 512,
-              PG_ECG = 576, PG_DEC = 640;  // floats
-constexpr uint32_t P_AQK = (P_GATE + 644 * 4 + 1023) / 1024 * 1024;  // Aqk bf16 [64][128B] staging
+              PG_ECG = 576, PG_DEC = 640;  // floats; PG_EG..PG_DEC+3 is the gate block
+constexpr uint32_t P_AQK = (P_GATE + 644 * 4 + 1023) / 1024 * 1024;  // Aqk bf16 staging
 constexpr uint32_t P_WG = P_AQK + 8192;
 constexpr uint32_t P_BARS = 2 * P_WG;
 constexpr uint32_t BAR_BYTES = 24 * 8;
@@ -84,30 +87,27 @@ constexpr uint32_t kSmemBytes =
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 static_assert(S_BARS % 8 == 0 && P_BARS % 8 == 0, "barrier alignment");
+static_assert(P_AF + 32768 <= P_GATE, "W^T | U^T staging fits in the A / T scratch");
 
 // ---- barriers (spine)
 enum {
-  SB_KQF = 0,     // +stage: K/Q tiles landed (TMA)
-  SB_KQE = 2,     // +stage: K/Q tiles free (MMA commit)
-  SB_SLOTF = 4,   // +slot: a prep filled the slot (128 remote arrivals)
-  SB_HREADY = 6,  // H^T bf16 written (128)
-  SB_VNFULL = 7,  // -H^T W^T done (commit)
-  SB_VNREADY = 8, // Vn / scaled Vn written (128)
-  SB_DHFULL = 9,  // H += dH done (commit)
-  SB_OFULL = 10,  // +buf: O1, O2 done (commit)
-  SB_OFREE = 12,  // +buf: O1, O2 read back (128)
-  SB_EPISYNC = 14,
-  SB_DRAIN = 15,
-  SB_EXIT = 16,
-  SB_COUNT = 17
+  SB_KQF = 0,      // +stage: K/Q tiles landed (TMA)
+  SB_KQE = 2,      // +stage: K/Q tiles free (MMA commit)
+  SB_SLOTF = 4,    // +slot: slot data landed (bulk loads)
+  SB_SFREE = 6,    // +slot: slot no longer read (128, epilogue warps)
+  SB_GREADY = 8,   // +ring: a prep stored this ring entry (1 remote arrival)
+  SB_VNFULL = 12,  // -H^T W^T done (commit)
+  SB_DHFULL = 13,  // H += dH done (commit)
+  SB_OFULL = 14,   // +buf: O1, O2 done (commit)
+  SB_OFREE = 16,   // +buf: O1, O2 read back (128)
+  SB_DRAIN = 18,
+  SB_EXIT = 19,
+  SB_COUNT = 20
 };
 // ---- barriers (prep); per group w: base + w
 enum {
-  PB_KQVF = 0, PB_KQVE = 2, PB_P1F = 4, PB_P1FREE = 6, PB_TREADY = 8, PB_WUF = 10, PB_SYNC = 12,
-  // +group: the spine released this CTA's slot for the group that writes it
-  // next (slot item ks is followed by ks + 1, which group (ks + 1) & 1 writes);
-  // 128 remote arrivals each
-  PB_SLOTFREE = 14,
+  PB_KQVF = 0, PB_KQVE = 2, PB_P1F = 4, PB_P1FREE = 6, PB_TREADY = 8, PB_WUF = 10,
+  PB_GFREE = 12,  // +ring: the spine has loaded this ring entry (1 remote arrival)
   PB_DRAIN = 16,
   PB_EXIT = 17,
   PB_COUNT = 18
@@ -116,7 +116,7 @@ enum {
 // ---- TMEM columns
 // spine: Vn, O1 x2, O2 x2, and the state H^T itself (f32, lane j = row j)
 constexpr uint32_t ST_VN = 0, ST_O1 = 64, ST_O2 = 192, ST_H = 320;
-constexpr uint32_t PT_P1 = 0, PT_W = 64, PT_U = 128, PT_WG = 192;    // prep, per group
+constexpr uint32_t PT_P1 = 0, PT_W = 64, PT_U = 128, PT_WG = 192;  // prep, per group
 
 struct Params {
   const float* g;
@@ -125,6 +125,7 @@ struct Params {
   const float* h0;
   float* hT;
   uint16_t* o;
+  uint8_t* ws;  // 4 global slot-ring entries of SLOT_G bytes per cluster
   int gb_stride, num_seqs, total_tokens, H_k, H_v, D;
   float scale;
 };
@@ -174,22 +175,12 @@ __device__ __forceinline__ void it_next(ChunkIter& it, const Params& p, int uste
   it_skip_empty(it, p, ustep);
 }
 
-// Advance to the first chunk at or after the current one with c % 4 == sel.
-__device__ __forceinline__ void it_align(ChunkIter& it, const Params& p, int ustep, int sel) {
-  while (it.ok && (it.c & 3) != sel) it_next(it, p, ustep);
+// Advance to the first chunk at or after the current one that prep rank
+// 1 + par (of P) hands to its group w: c % P == par and (c / P) % 2 == w.
+__device__ __forceinline__ void it_align(ChunkIter& it, const Params& p, int ustep, int P, int par,
+                                         int w) {
+  while (it.ok && (it.c % P != par || ((it.c / P) & 1) != w)) it_next(it, p, ustep);
 }
-
-// Bounded barrier among the 128 threads of one warpgroup (mbarrier based).
-struct WgSync {
-  uint64_t* bar;
-  uint32_t phase;
-  __device__ __forceinline__ bool operator()(volatile int* abort, uint32_t* err) {
-    mbar_arrive(bar);
-    const bool ok = mbar_wait(bar, phase, abort, err, 64u);
-    phase ^= 1u;
-    return ok;
-  }
-};
 
 template <int NCH>
 __device__ __forceinline__ void pack_chunks(const float* x, uint32_t* out) {
@@ -242,121 +233,174 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* x) {
 }
 
 // ---------------------------------------------------------------------------
-// T = (I + A)^{-1} for a strictly lower triangular 64x64 A (f32, row stride
-// kAS), by 16x16 blocks: the diagonal blocks by forward substitution, then the
-// block diagonals L = 1, 2, 3:
-//   X = sum_{l in blocks bj .. bi-1} A_{bi,l} T_{l,bj};   T_{bi,bj} = -T_{bi,bi} X
-// 128 threads; every phase is a set of independent 2-column tasks.
+// Named (hardware) barriers among the threads of one prep group.  Used only
+// where every thread of the group is guaranteed to arrive (no early exits in
+// between); after a bounded wait that may fail, group_all() first agrees on
+// the outcome so that all threads leave together.
 // ---------------------------------------------------------------------------
-template <int LD>
-__device__ __forceinline__ void level_x(const float* Af, const float* Tf, float* Xs, int p) {
-  constexpr int NB = 4 - LD;
-  constexpr int PARTS = (LD == 3) ? 3 : 1;
-  constexpr int KLEN = 16 * LD / PARTS;
-  constexpr int NT = NB * PARTS;  // tasks per thread (128 tasks per block-part)
-  const int i = p >> 3, q = p & 7;
-  float acc[NT][2];
-#pragma unroll
-  for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = 0.f;
-#pragma unroll
-  for (int l = 0; l < KLEN; l += 4) {
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      const int b = t / PARTS, part = t % PARTS;
-      const int bi = b + LD, bj = b, k0 = 16 * bj + part * KLEN;
-      const float4 a = *reinterpret_cast<const float4*>(Af + (16 * bi + i) * kAS + k0 + l);
-      const float* tc = Tf + (k0 + l) * kAS + 16 * bj + 2 * q;
-      const float2 t0 = *reinterpret_cast<const float2*>(tc);
-      const float2 t1 = *reinterpret_cast<const float2*>(tc + kAS);
-      const float2 t2 = *reinterpret_cast<const float2*>(tc + 2 * kAS);
-      const float2 t3 = *reinterpret_cast<const float2*>(tc + 3 * kAS);
-      acc[t][0] = fmaf(a.x, t0.x, acc[t][0]);
-      acc[t][1] = fmaf(a.x, t0.y, acc[t][1]);
-      acc[t][0] = fmaf(a.y, t1.x, acc[t][0]);
-      acc[t][1] = fmaf(a.y, t1.y, acc[t][1]);
-      acc[t][0] = fmaf(a.z, t2.x, acc[t][0]);
-      acc[t][1] = fmaf(a.z, t2.y, acc[t][1]);
-      acc[t][0] = fmaf(a.w, t3.x, acc[t][0]);
-      acc[t][1] = fmaf(a.w, t3.y, acc[t][1]);
-    }
-  }
-#pragma unroll
-  for (int t = 0; t < NT; ++t)
-    *reinterpret_cast<float2*>(Xs + t * 256 + i * 16 + 2 * q) = make_float2(acc[t][0], acc[t][1]);
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-template <int LD>
-__device__ __forceinline__ void level_t(float* Tf, const float* Xs, int p) {
-  constexpr int NB = 4 - LD;
-  constexpr int PARTS = (LD == 3) ? 3 : 1;
-  const int i = p >> 3, q = p & 7;
+__device__ __forceinline__ bool named_all(int id, int nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(v)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+// ---------------------------------------------------------------------------
+// T = (I + A)^{-1} for a strictly lower triangular 64x64 A (f32, row stride
+// kAS), 128 threads (4 warps), with 16x16 blocks D_i = (I + A_ii)^{-1}:
+//   1. warp w: D_w by forward substitution (lane j < 16 owns column j and
+//      pushes each new x_l into the running sums of the rows below it);
+//   2. warp pair p (blocks 2p, 2p+1):  T_{2p+1,2p} = -D_{2p+1} A_{2p+1,2p} D_{2p};
+//   3. X = A[32:64, 0:32] T[0:32, 0:32];
+//   4. T[32:64, 0:32] = -T[32:64, 32:64] X.
+// Each thread of steps 2-4 owns a small output tile (independent accumulators).
+// bar_base: named barrier ids bar_base (128 threads), bar_base+1+p (pairs).
+// X scratch (32x32 f32) at Xs; the pair products use Xs too.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void invert_unit_lower64(const float* Af, float* Tf, float* Xs, int p,
+                                                    int bar_base) {
+  const int w = p >> 5, ln = p & 31;
+  // 1. diagonal blocks
+  if (ln < 16) {
+    const int j = ln;
+    const float* Ab = Af + (16 * w) * kAS + 16 * w;
+    float x[16], acc[16];
 #pragma unroll
-  for (int b = 0; b < NB; ++b) {
-    const int bi = b + LD, bj = b;
-    const float* tr = Tf + (16 * bi + i) * kAS + 16 * bi;
-    float y0 = 0.f, y1 = 0.f;
+    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int l = 0; l < 16; ++l) {
+      x[l] = (l < j) ? 0.f : ((l == j) ? 1.f : -acc[l]);
+#pragma unroll
+      for (int i = l + 1; i < 16; ++i) acc[i] = fmaf(Ab[i * kAS + l], x[l], acc[i]);
+    }
+    float* Tb = Tf + (16 * w) * kAS + 16 * w + j;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) Tb[i * kAS] = x[i];
+  } else if ((w & 1) == 0) {
+    // Steps 3 and 4 read the upper blocks T_{0,1} and T_{2,3} as zeros; the
+    // scratch is reused between items, so clear them here (idle lanes).
+    float* Tz = Tf + (16 * w) * kAS + 16 * (w + 1) + (ln - 16);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) Tz[i * kAS] = 0.f;
+  }
+  // 2. first sub-diagonal blocks, one per warp pair: thread t of the pair owns
+  //    row t>>2, columns 4(t&3)..+3
+  {
+    const int pr = w >> 1, t = p & 63;
+    const int bi = 2 * pr + 1, bj = 2 * pr;
+    const int i = t >> 2, c4 = 4 * (t & 3);
+    float* Y = Xs + pr * 256;
+    named_sync(bar_base + 1 + pr, 64);
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* ar = Af + (16 * bi + i) * kAS + 16 * bj;
 #pragma unroll
     for (int l = 0; l < 16; l += 4) {
-      const float4 a = *reinterpret_cast<const float4*>(tr + l);
+      const float4 a = *reinterpret_cast<const float4*>(ar + l);
       const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-        for (int part = 0; part < PARTS; ++part) {
-          const float2 xv = *reinterpret_cast<const float2*>(Xs + (b * PARTS + part) * 256 +
-                                                             (l + m) * 16 + 2 * q);
-          x0 += xv.x;
-          x1 += xv.y;
-        }
-        y0 = fmaf(av[m], x0, y0);
-        y1 = fmaf(av[m], x1, y1);
+        const float4 d = *reinterpret_cast<const float4*>(Tf + (16 * bj + l + m) * kAS + 16 * bj + c4);
+        y[0] = fmaf(av[m], d.x, y[0]);
+        y[1] = fmaf(av[m], d.y, y[1]);
+        y[2] = fmaf(av[m], d.z, y[2]);
+        y[3] = fmaf(av[m], d.w, y[3]);
       }
     }
-    *reinterpret_cast<float2*>(Tf + (16 * bi + i) * kAS + 16 * bj + 2 * q) = make_float2(-y0, -y1);
-  }
-}
-
-__device__ __forceinline__ bool invert_unit_lower64(const float* Af, float* Tf, float* Xs, int p,
-                                                    WgSync& sync, volatile int* abort,
-                                                    uint32_t* err) {
-  const int lane = p & 31, d = p >> 5;
-  if (lane < 16) {  // diagonal block d, column j
-    const int j = lane;
-    const float* Ab = Af + (16 * d) * kAS + 16 * d;
-    float x[16];
+    *reinterpret_cast<float4*>(Y + i * 16 + c4) = make_float4(y[0], y[1], y[2], y[3]);
+    named_sync(bar_base + 1 + pr, 64);
+    float z[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* dr = Tf + (16 * bi + i) * kAS + 16 * bi;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = (i == j) ? 1.f : 0.f;
+    for (int l = 0; l < 16; l += 4) {
+      const float4 a = *reinterpret_cast<const float4*>(dr + l);
+      const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-    for (int i = 1; i < 16; ++i) {
-      float s = 0.f;
-#pragma unroll
-      for (int l = 0; l < i; ++l) s = fmaf(Ab[i * kAS + l], x[l], s);
-      if (i > j) x[i] = -s;
+      for (int m = 0; m < 4; ++m) {
+        const float4 yv = *reinterpret_cast<const float4*>(Y + (l + m) * 16 + c4);
+        z[0] = fmaf(av[m], yv.x, z[0]);
+        z[1] = fmaf(av[m], yv.y, z[1]);
+        z[2] = fmaf(av[m], yv.z, z[2]);
+        z[3] = fmaf(av[m], yv.w, z[3]);
+      }
     }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) Tf[(16 * d + i) * kAS + 16 * d + j] = x[i];
+    *reinterpret_cast<float4*>(Tf + (16 * bi + i) * kAS + 16 * bj + c4) =
+        make_float4(-z[0], -z[1], -z[2], -z[3]);
   }
-  if (!sync(abort, err)) return false;
-  level_x<1>(Af, Tf, Xs, p);
-  if (!sync(abort, err)) return false;
-  level_t<1>(Tf, Xs, p);
-  if (!sync(abort, err)) return false;
-  level_x<2>(Af, Tf, Xs, p);
-  if (!sync(abort, err)) return false;
-  level_t<2>(Tf, Xs, p);
-  if (!sync(abort, err)) return false;
-  level_x<3>(Af, Tf, Xs, p);
-  if (!sync(abort, err)) return false;
-  level_t<3>(Tf, Xs, p);
-  return sync(abort, err);
+  named_sync(bar_base, 128);
+  // 3. X = A[32:64, 0:32] T[0:32, 0:32]; thread p owns rows 2(p>>3)..+1, cols 4(p&7)..+3
+  const int r0 = 2 * (p >> 3), c0 = 4 * (p & 7);
+  {
+    float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* a0r = Af + (32 + r0) * kAS;
+    const float* a1r = a0r + kAS;
+#pragma unroll 2
+    for (int k = 0; k < 32; k += 4) {
+      const float4 a0 = *reinterpret_cast<const float4*>(a0r + k);
+      const float4 a1 = *reinterpret_cast<const float4*>(a1r + k);
+      const float av0[4] = {a0.x, a0.y, a0.z, a0.w}, av1[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float4 tv = *reinterpret_cast<const float4*>(Tf + (k + m) * kAS + c0);
+        x0[0] = fmaf(av0[m], tv.x, x0[0]);
+        x0[1] = fmaf(av0[m], tv.y, x0[1]);
+        x0[2] = fmaf(av0[m], tv.z, x0[2]);
+        x0[3] = fmaf(av0[m], tv.w, x0[3]);
+        x1[0] = fmaf(av1[m], tv.x, x1[0]);
+        x1[1] = fmaf(av1[m], tv.y, x1[1]);
+        x1[2] = fmaf(av1[m], tv.z, x1[2]);
+        x1[3] = fmaf(av1[m], tv.w, x1[3]);
+      }
+    }
+    *reinterpret_cast<float4*>(Xs + r0 * 32 + c0) = make_float4(x0[0], x0[1], x0[2], x0[3]);
+    *reinterpret_cast<float4*>(Xs + (r0 + 1) * 32 + c0) = make_float4(x1[0], x1[1], x1[2], x1[3]);
+  }
+  named_sync(bar_base, 128);
+  // 4. T[32:64, 0:32] = -T[32:64, 32:64] X  (T[32+r, 32+k] = 0 for k > r)
+  {
+    float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* t0r = Tf + (32 + r0) * kAS + 32;
+    const float* t1r = t0r + kAS;
+#pragma unroll 2
+    for (int k = 0; k < 32; k += 4) {
+      const float4 a0 = *reinterpret_cast<const float4*>(t0r + k);
+      const float4 a1 = *reinterpret_cast<const float4*>(t1r + k);
+      const float av0[4] = {a0.x, a0.y, a0.z, a0.w}, av1[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float4 xv = *reinterpret_cast<const float4*>(Xs + (k + m) * 32 + c0);
+        z0[0] = fmaf(av0[m], xv.x, z0[0]);
+        z0[1] = fmaf(av0[m], xv.y, z0[1]);
+        z0[2] = fmaf(av0[m], xv.z, z0[2]);
+        z0[3] = fmaf(av0[m], xv.w, z0[3]);
+        z1[0] = fmaf(av1[m], xv.x, z1[0]);
+        z1[1] = fmaf(av1[m], xv.y, z1[1]);
+        z1[2] = fmaf(av1[m], xv.z, z1[2]);
+        z1[3] = fmaf(av1[m], xv.w, z1[3]);
+      }
+    }
+    *reinterpret_cast<float4*>(Tf + (32 + r0) * kAS + c0) =
+        make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
+    *reinterpret_cast<float4*>(Tf + (32 + r0 + 1) * kAS + c0) =
+        make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
+  }
+  named_sync(bar_base, 128);
 }
 
 }  // namespace pf
 
 using namespace pf;
 
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -364,6 +408,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t rank = cluster_ctarank();
+  const uint32_t ncta = cluster_nctarank();  // 2 or 3: the spine and P = ncta - 1 preps
+  const int P = int(ncta) - 1;
   const bool spine = rank == 0;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (spine ? S_BARS : P_BARS));
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);  // after 24 barrier slots
@@ -376,6 +422,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   const int nbox = D / 64;
   const int u0 = int(cluster_id_x());
   const int ustep = int(num_clusters_x());
+  uint8_t* ring = p.ws + size_t(cluster_id_x()) * kRing * SLOT_G;
 
   for (uint32_t i = tid * 16; i < kSmemBytes; i += kThreads * 16)
     *reinterpret_cast<uint4*>(smem + i) = make_uint4(0, 0, 0, 0);
@@ -384,19 +431,15 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     if (spine) {
       for (int b = 0; b < SB_COUNT; ++b) {
         uint32_t cnt = 1;
-        if (b == SB_SLOTF || b == SB_SLOTF + 1 || b == SB_HREADY || b == SB_VNREADY ||
-            b == SB_OFREE || b == SB_OFREE + 1 || b == SB_EPISYNC)
-          cnt = 128;
-        if (b == SB_EXIT) cnt = kCluster;
+        if (b == SB_SFREE || b == SB_SFREE + 1 || b == SB_OFREE || b == SB_OFREE + 1) cnt = 128;
+        if (b == SB_EXIT) cnt = ncta;
         mbar_init(&bars[b], cnt);
       }
     } else {
       for (int b = 0; b < PB_COUNT; ++b) {
         uint32_t cnt = 1;
-        if (b == PB_P1FREE || b == PB_P1FREE + 1 || b == PB_TREADY || b == PB_TREADY + 1 ||
-            b == PB_SYNC || b == PB_SYNC + 1 || b == PB_SLOTFREE || b == PB_SLOTFREE + 1)
-          cnt = 128;
-        if (b == PB_EXIT) cnt = kCluster;
+        if (b == PB_P1FREE || b == PB_P1FREE + 1 || b == PB_TREADY || b == PB_TREADY + 1) cnt = 128;
+        if (b == PB_EXIT) cnt = ncta;
         mbar_init(&bars[b], cnt);
       }
     }
@@ -418,7 +461,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
     // SPINE
     // =====================================================================
     if (warp == 8) {
-      // ---------------- TMA: K and Q tiles of every chunk (2 stages)
+      // ---------------- TMA: K and Q tiles (2 stages) and the slot data of
+      // every chunk (2 shared-memory slots fed from the 4-entry global ring)
       if (elect_one()) {
         ChunkIter it;
         it_start(it, p, u0, ustep);
@@ -434,77 +478,42 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
             tma_load_3d(kq + b * 16384, &tm_k, fb, b * 64, hk, it.t0);
             tma_load_3d(kq + b * 16384 + 8192, &tm_q, fb, b * 64, hk, it.t0);
           }
+          // slot st: free once the epilogue is done with chunk c-2; the ring
+          // entry once a prep has stored chunk c there
+          if (!mbar_wait(&bars[SB_SFREE + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 1u)) break;
+          if (!mbar_wait_cluster(&bars[SB_GREADY + (c & 3)], (c >> 2) & 1, abort_flag, err, 1u))
+            break;
+          fence_proxy_async_global();
+          uint64_t* sb = &bars[SB_SLOTF + st];
+          mbar_arrive_expect_tx(sb, SLOT_TX);
+          const uint8_t* src = ring + (c & 3) * SLOT_G;
+          bulk_load_g2s(smem + S_SLOT + st * SL_BYTES, src, G_GATE, sb);
+          bulk_load_g2s(smem + S_SGATE + st * G_GATE_BYTES, src + G_GATE, G_GATE_BYTES, sb);
           issued = c + 1;
           it_next(it, p, ustep);
         }
-        for (int cc = issued - 2; cc < issued; ++cc)
-          if (cc >= 0) mbar_wait(&bars[SB_KQF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
-      }
-      __syncwarp();
-    } else if (warp == 9) {
-      // ---------------- MMA issue (one thread), chunk by chunk
-      if (elect_one()) {
-        const uint32_t id_vn = make_idesc_bf16(128, 64, 0, 1, /*b_neg=*/1);
-        const uint32_t id_o1 = make_idesc_bf16(128, 64, 0, 0);
-        const uint32_t id_dh = make_idesc_bf16(128, 128, 0, 1);
-        const uint32_t id_o2 = make_idesc_bf16(128, 64, 0, 0);
-        ChunkIter it;
-        it_start(it, p, u0, ustep);
-        while (it.ok) {
-          const int c = it.c, st = c & 1, ob = c & 1;
-          const uint32_t kq = sbase + S_KQ + st * 32768;
-          const uint32_t slot = sbase + S_SLOT + st * SL_BYTES;
-          if (!mbar_wait(&bars[SB_KQF + st], (c >> 1) & 1, abort_flag, err, 2u)) break;
-          if (!mbar_wait_cluster(&bars[SB_SLOTF + st], (c >> 1) & 1, abort_flag, err, 2u)) break;
-          if (!mbar_wait(&bars[SB_HREADY], c & 1, abort_flag, err, 2u)) break;
-          fence_proxy_async_smem();
-          tc_fence_after();
-          // Vn^T := -H^T W^T   (U^T is added by the state warps)
-          for (int kk = 0; kk < ksteps_d; ++kk) {
-            const uint32_t a = sbase + S_HT + (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16_ss(tmem + ST_VN, make_sdesc_sw128(a, 16, 1024),
-                        make_sdesc_sw128(slot + SL_W + kk * 2048, 8192, 1024), id_vn, kk > 0);
-          }
-          mma_commit(&bars[SB_VNFULL]);
-          // O1^T = H^T Q^T into buffer ob (free once the epilogue read chunk c-2)
-          if (c >= 2 && !mbar_wait(&bars[SB_OFREE + ob], ((c >> 1) & 1) ^ 1, abort_flag, err, 2u))
-            break;
-          tc_fence_after();
-          for (int kk = 0; kk < ksteps_d; ++kk) {
-            const uint32_t a = sbase + S_HT + (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t b = kq + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32;
-            mma_bf16_ss(tmem + ST_O1 + 64u * ob, make_sdesc_sw128(a, 16, 1024),
-                        make_sdesc_sw128(b, 16, 1024), id_o1, kk > 0);
-          }
-          // H^T += Vns^T K ; O2^T = Vn^T Aqk^T
-          if (!mbar_wait(&bars[SB_VNREADY], c & 1, abort_flag, err, 2u)) break;
-          tc_fence_after();
-          // H^T (already scaled by e^{G_C} in TMEM) += Vns^T K
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem + ST_H, make_sdesc_sw128(sbase + S_VNS + kk * 32, 16, 1024),
-                        make_sdesc_sw128(kq + kk * 2048, 16384, 1024), id_dh, 1);
-          mma_commit(&bars[SB_DHFULL]);
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem + ST_O2 + 64u * ob, make_sdesc_sw128(sbase + S_VN + kk * 32, 16, 1024),
-                        make_sdesc_sw128(slot + SL_AQK + kk * 32, 16, 1024), id_o2, kk > 0);
-          mma_commit(&bars[SB_OFULL + ob]);
-          mma_commit(&bars[SB_KQE + st]);
-          it_next(it, p, ustep);
+        for (int cc = issued - 2; cc < issued; ++cc) {
+          if (cc < 0) continue;
+          mbar_wait(&bars[SB_KQF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
+          mbar_wait(&bars[SB_SLOTF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
         }
-        mma_commit(&bars[SB_DRAIN]);
-        mbar_wait(&bars[SB_DRAIN], 0, nullptr, err, 8u);
       }
       __syncwarp();
     } else if (warp < 4) {
       // ---------------- state warps: thread j owns row j of H^T, kept in TMEM
       // (f32, 128 columns at ST_H).  Per chunk: read H^T, write its bf16 copy
-      // (the A operand of Vn and O1), write back e^{G_C} H^T so that the dH MMA
-      // accumulates H_{c+1} = e^{G_C} H_c + dH in place.
+      // (the A operand of Vn and O1) and write back e^{G_C} H^T, so that the dH
+      // MMA accumulates H_{c+1} = e^{G_C} H_c + dH in place.  Thread 0 also
+      // issues the chunk's MMAs right after the group's named barriers.
       const int j = tid;
+      const bool issuer = j == 0;
       const uint32_t lane_off = uint32_t(warp * 32) << 16;
       const uint32_t th = tmem + lane_off + ST_H;
       const bool jv = j < D;
       const int units = p.num_seqs * p.H_v;
+      const uint32_t id_vn = make_idesc_bf16(128, 64, 0, 1, /*b_neg=*/1);
+      const uint32_t id_o = make_idesc_bf16(128, 64, 0, 0);
+      const uint32_t id_dh = make_idesc_bf16(128, 128, 0, 1);
       int c = 0;
       bool ok = true;
       for (int u = u0; u < units && ok; u += ustep) {
@@ -513,70 +522,98 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
         seq_range(p, n, tb, te);
         const size_t state_off = (size_t(n) * p.H_v + h) * size_t(D) * D;
         const float* h0 = (p.h0 != nullptr && jv) ? p.h0 + state_off + j : nullptr;
+#pragma unroll 1
+        for (int q4 = 0; q4 < 4; ++q4) {  // H^T row j <- h0 (or zeros)
+          float x[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            x[i] = (h0 != nullptr && 32 * q4 + i < D) ? h0[size_t(32 * q4 + i) * D] : 0.f;
+          tmem_st32(th + 32u * q4, x);
+        }
+        tmem_st_wait();
         for (int t0 = tb; t0 < te && ok; t0 += C, ++c) {
           const int st = c & 1;
-          const bool first = t0 == tb;
-          if (!first) {  // H = e^{G_C} H_{c-1} + dH landed
+          const uint32_t kq = sbase + S_KQ + st * 32768;
+          const uint32_t slot = sbase + S_SLOT + st * SL_BYTES;
+          if (t0 > tb) {  // H = e^{G_C} H_{c-1} + dH landed
             ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u);
-            if (!ok) break;
             tc_fence_after();
           }
-          ok = mbar_wait_cluster(&bars[SB_SLOTF + st], (c >> 1) & 1, abort_flag, err, 16u);
-          if (!ok) break;
-          const float* sg = reinterpret_cast<const float*>(smem + S_SGATE) + st * SG_FLOATS;
+          ok = ok && mbar_wait(&bars[SB_SLOTF + st], (c >> 1) & 1, abort_flag, err, 16u);
+          if (ok && issuer)  // ring entry c & 3 has been copied in: the prep may reuse it
+            mbar_arrive_remote(
+                mapa_shared(sbase + P_BARS + (PB_GFREE + (c & 3)) * 8, 1 + uint32_t(c % P)));
+          const float* sg = reinterpret_cast<const float*>(smem + S_SGATE + st * G_GATE_BYTES);
           const float dec = sg[128];
 #pragma unroll 1
-          for (int q4 = 0; q4 < 4; ++q4) {
-            float x[32];
-            if (first) {
+          for (int hh = 0; hh < 2; ++hh) {  // 64 columns = one 128-byte box row at a time
+            float x[64];
+            tmem_ld32(th + 64u * hh, *reinterpret_cast<float(*)[32]>(x));
+            tmem_ld32(th + 64u * hh + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+            tmem_ld_wait();
+            st_row64_bf16(sbase + S_HT + hh * 16384, uint32_t(j), x);
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                x[i] = (h0 != nullptr && 32 * q4 + i < D) ? h0[size_t(32 * q4 + i) * D] : 0.f;
-            } else {
-              tmem_ld32(th + 32u * q4, x);
-              tmem_ld_wait();
-            }
-            const uint32_t ht = sbase + S_HT + (q4 >> 1) * 16384;
-#pragma unroll
-            for (int hc = 0; hc < 4; ++hc) {
-              const int cc = 4 * (q4 & 1) + hc;
-              st_shared_v4(ht + sw128_offset(j, cc * 16), pack_bf16x2(x[8 * hc], x[8 * hc + 1]),
-                           pack_bf16x2(x[8 * hc + 2], x[8 * hc + 3]),
-                           pack_bf16x2(x[8 * hc + 4], x[8 * hc + 5]),
-                           pack_bf16x2(x[8 * hc + 6], x[8 * hc + 7]));
-            }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] *= dec;
-            tmem_st32(th + 32u * q4, x);
+            for (int i = 0; i < 64; ++i) x[i] *= dec;
+            tmem_st32(th + 64u * hh, *reinterpret_cast<float(*)[32]>(x));
+            tmem_st32(th + 64u * hh + 32, *reinterpret_cast<float(*)[32]>(x + 32));
           }
           tmem_st_wait();
           fence_proxy_async_smem();
           tc_fence_before();
-          mbar_arrive(&bars[SB_HREADY]);
+          if (!named_all(1, 128, ok)) {
+            ok = false;
+            break;
+          }
+          if (issuer) {
+            tc_fence_after();
+            ok = mbar_wait(&bars[SB_KQF + st], (c >> 1) & 1, abort_flag, err, 2u);
+            if (ok) {  // Vn^T := -H^T W^T   (U^T is added below)
+              for (int kk = 0; kk < ksteps_d; ++kk) {
+                const uint32_t a = sbase + S_HT + (kk >> 2) * 16384 + (kk & 3) * 32;
+                mma_bf16_ss(tmem + ST_VN, make_sdesc_sw128(a, 16, 1024),
+                            make_sdesc_sw128(slot + G_W + kk * 2048, 8192, 1024), id_vn, kk > 0);
+              }
+              mma_commit(&bars[SB_VNFULL]);
+              // O1^T = H^T Q^T into buffer st (free once the epilogue read chunk c-2)
+              ok = c < 2 ||
+                   mbar_wait(&bars[SB_OFREE + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 2u);
+              if (ok) {
+                tc_fence_after();
+                for (int kk = 0; kk < ksteps_d; ++kk) {
+                  const uint32_t a = sbase + S_HT + (kk >> 2) * 16384 + (kk & 3) * 32;
+                  const uint32_t b = kq + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32;
+                  mma_bf16_ss(tmem + ST_O1 + 64u * st, make_sdesc_sw128(a, 16, 1024),
+                              make_sdesc_sw128(b, 16, 1024), id_o, kk > 0);
+                }
+              }
+            }
+          }
           // Vn = U - (H W)  ->  Vn^T and e^{G_C - G_r} Vn^T rows in bf16
-          ok = mbar_wait(&bars[SB_VNFULL], c & 1, abort_flag, err, 16u);
-          if (!ok) break;
+          ok = ok && mbar_wait(&bars[SB_VNFULL], c & 1, abort_flag, err, 16u);
           tc_fence_after();
-          {
-            const uint8_t* urow = smem + S_SLOT + st * SL_BYTES + SL_U;
+          if (ok) {
+            const uint8_t* urow = smem + S_SLOT + st * SL_BYTES + G_U;
 #pragma unroll 1
-            for (int q4 = 0; q4 < 4; ++q4) {  // 16 columns (two 16-byte chunks) at a time
-              float vn[16];
-              tmem_ld16(tmem + lane_off + ST_VN + 16u * q4, vn);
+            for (int hf = 0; hf < 2; ++hf) {  // 32 columns (four 16-byte chunks) at a time
+              float vn[32];
+              tmem_ld32(tmem + lane_off + ST_VN + 32u * hf, vn);
               tmem_ld_wait();
 #pragma unroll
-              for (int hc = 0; hc < 2; ++hc) {
-                const int cc = 2 * q4 + hc;
+              for (int hc = 0; hc < 4; ++hc) {
+                const int cc = 4 * hf + hc;
                 const uint4 uv = *reinterpret_cast<const uint4*>(urow + sw128_offset(j, cc * 16));
+                const float4 e0 = *reinterpret_cast<const float4*>(sg + 64 + 8 * cc);
+                const float4 e1 = *reinterpret_cast<const float4*>(sg + 64 + 8 * cc + 4);
+                const float ec[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
                 const uint32_t uw[4] = {uv.x, uv.y, uv.z, uv.w};
                 float x[8], y[8];
 #pragma unroll
-                for (int kq = 0; kq < 4; ++kq) {
-                  x[2 * kq] = vn[8 * hc + 2 * kq] + __uint_as_float(uw[kq] << 16);
-                  x[2 * kq + 1] = vn[8 * hc + 2 * kq + 1] + __uint_as_float(uw[kq] & 0xFFFF0000u);
+                for (int kq2 = 0; kq2 < 4; ++kq2) {
+                  x[2 * kq2] = vn[8 * hc + 2 * kq2] + __uint_as_float(uw[kq2] << 16);
+                  x[2 * kq2 + 1] = vn[8 * hc + 2 * kq2 + 1] + __uint_as_float(uw[kq2] & 0xFFFF0000u);
                 }
 #pragma unroll
-                for (int m = 0; m < 8; ++m) y[m] = x[m] * sg[64 + 8 * cc + m];
+                for (int m = 0; m < 8; ++m) y[m] = x[m] * ec[m];
                 st_shared_v4(sbase + S_VN + sw128_offset(j, cc * 16), pack_bf16x2(x[0], x[1]),
                              pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
                              pack_bf16x2(x[6], x[7]));
@@ -588,11 +625,27 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
           tc_fence_before();
-          mbar_arrive(&bars[SB_VNREADY]);
+          if (!named_all(1, 128, ok)) {
+            ok = false;
+            break;
+          }
+          if (issuer) {
+            tc_fence_after();
+            // H^T (already scaled by e^{G_C} in TMEM) += Vns^T K ; O2^T = Vn^T Aqk^T
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(tmem + ST_H, make_sdesc_sw128(sbase + S_VNS + kk * 32, 16, 1024),
+                          make_sdesc_sw128(kq + kk * 2048, 16384, 1024), id_dh, 1);
+            mma_commit(&bars[SB_DHFULL]);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(tmem + ST_O2 + 64u * st,
+                          make_sdesc_sw128(sbase + S_VN + kk * 32, 16, 1024),
+                          make_sdesc_sw128(slot + G_AQK + kk * 32, 16, 1024), id_o, kk > 0);
+            mma_commit(&bars[SB_OFULL + st]);
+            mma_commit(&bars[SB_KQE + st]);
+          }
         }
         if (!ok) break;
-        // final state: H after the last chunk's update (or h0 for an empty sequence)
-        if (te > tb) {
+        if (te > tb) {  // the last chunk's update
           ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u);
           if (!ok) break;
           tc_fence_after();
@@ -602,14 +655,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int q4 = 0; q4 < 4; ++q4) {
             float x[32];
-            if (te > tb) {
-              tmem_ld32(th + 32u * q4, x);
-              tmem_ld_wait();
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                x[i] = (h0 != nullptr && 32 * q4 + i < D) ? h0[size_t(32 * q4 + i) * D] : 0.f;
-            }
+            tmem_ld32(th + 32u * q4, x);
+            tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i)
               if (32 * q4 + i < D) hT[size_t(32 * q4 + i) * D] = x[i];
@@ -617,13 +664,15 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
       }
-    } else {
+      if (issuer) {  // every MMA this thread issued has completed
+        mma_commit(&bars[SB_DRAIN]);
+        mbar_wait(&bars[SB_DRAIN], 0, nullptr, err, 8u);
+      }
+    } else if (warp < 8) {
       // ---------------- epilogue warps: o_r = e^{G_r} scale O1[r] + O2[r]
       const int e = tid - 128;
       const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
-      WgSync sync{&bars[SB_EPISYNC], 0};
-      uint8_t* ost = smem + S_OST;
-      const int row_bytes = D * 2;
+      const bool ev = e < D;
       ChunkIter it;
       it_start(it, p, u0, ustep);
       while (it.ok) {
@@ -631,51 +680,50 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
         const int L = min(C, it.te - it.t0);
         if (!mbar_wait(&bars[SB_OFULL + ob], (c >> 1) & 1, abort_flag, err, 128u)) break;
         tc_fence_after();
-        if (!sync(abort_flag, err)) break;  // staging free (previous copy-out done)
-        const float* sg = reinterpret_cast<const float*>(smem + S_SGATE) + ob * SG_FLOATS;
-        const float sc = p.scale;
-#pragma unroll 1
-        for (int q4 = 0; q4 < 4; ++q4) {
-          float o1[16], o2[16];
-          tmem_ld16(tmem + lane_off + ST_O1 + 64u * ob + 16u * q4, o1);
-          tmem_ld16(tmem + lane_off + ST_O2 + 64u * ob + 16u * q4, o2);
-          tmem_ld_wait();
-          if (e < D) {
+        // The gate factors are the last thing read from slot ob: take a copy
+        // and hand the slot back to the TMA warp.
+        const float* sg = reinterpret_cast<const float*>(smem + S_SGATE + ob * G_GATE_BYTES);
+        float eg[64];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int r = 16 * q4 + i;
-              const float val = fmaf(sg[r] * sc, o1[i], o2[i]);
-              *reinterpret_cast<uint16_t*>(ost + r * row_bytes + 2 * e) =
-                  __bfloat16_as_ushort(__float2bfloat16_rn(val));
+        for (int r = 0; r < 64; r += 4) {
+          const float4 v4 = *reinterpret_cast<const float4*>(sg + r);
+          eg[r] = v4.x * p.scale;
+          eg[r + 1] = v4.y * p.scale;
+          eg[r + 2] = v4.z * p.scale;
+          eg[r + 3] = v4.w * p.scale;
+        }
+        mbar_arrive(&bars[SB_SFREE + ob]);
+        uint16_t* orow = p.o + (size_t(it.t0) * p.H_v + it.h) * D + e;
+        const size_t rstride = size_t(p.H_v) * D;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float o1[32], o2[32];
+          tmem_ld32(tmem + lane_off + ST_O1 + 64u * ob + 32u * hf, o1);
+          tmem_ld32(tmem + lane_off + ST_O2 + 64u * ob + 32u * hf, o2);
+          tmem_ld_wait();
+          if (hf == 1) {
+            tc_fence_before();
+            mbar_arrive(&bars[SB_OFREE + ob]);
+          }
+          if (ev) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int r = 32 * hf + i;
+              if (r < L)
+                orow[size_t(r) * rstride] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(eg[r], o1[i], o2[i])));
             }
           }
-        }
-        tc_fence_before();
-        mbar_arrive(&bars[SB_OFREE + ob]);
-        // The slot of chunk c is no longer needed by anyone: hand it to the prep
-        // group that fills it next.
-        const int next_group = ((c >> 1) + 1) & 1;
-        mbar_arrive_remote(
-            mapa_shared(sbase + P_BARS + (PB_SLOTFREE + next_group) * 8, 1 + (c & 1)));
-        if (!sync(abort_flag, err)) break;  // staging complete
-        const int per_row = row_bytes / 16;
-        for (int q = e; q < L * per_row; q += 128) {
-          const int r = q / per_row, cc = q % per_row;
-          const uint4 v = *reinterpret_cast<const uint4*>(ost + r * row_bytes + cc * 16);
-          *reinterpret_cast<uint4*>(p.o + (size_t(it.t0 + r) * p.H_v + it.h) * D + cc * 8) = v;
         }
         it_next(it, p, ustep);
       }
     }
   } else {
     // =====================================================================
-    // PREP (rank 1: even chunks, rank 2: odd chunks; group w takes every
-    // other one of those)
+    // PREP (with P prep CTAs, chunk c goes to prep rank 1 + c % P, and there
+    // to group (c / P) & 1; its results go to ring entry c & 3)
     // =====================================================================
     const int par = int(rank) - 1;
-    const uint32_t spine_slot = mapa_shared(sbase + S_SLOT + par * SL_BYTES, 0);
-    const uint32_t spine_gate = mapa_shared(sbase + S_SGATE + par * SG_FLOATS * 4, 0);
-    const uint32_t spine_slotf = mapa_shared(sbase + S_BARS + (SB_SLOTF + par) * 8, 0);
     if (warp == 8) {
       // ---------------- TMA: K, Q, V of each item into its group's buffers
       if (elect_one()) {
@@ -684,17 +732,17 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
         int last_k[2] = {-1, -1};
         while (it.ok) {
           const int c = it.c;
-          if ((c & 1) == par) {
-            const int w = (c >> 1) & 1, k = c >> 2;
+          if (c % P == par) {
+            const int w = (c / P) & 1, k = (c / P) >> 1;
             if (!mbar_wait(&bars[PB_KQVE + w], (k & 1) ^ 1, abort_flag, err, 1u)) break;
             uint64_t* fb = &bars[PB_KQVF + w];
             mbar_arrive_expect_tx(fb, uint32_t(nbox) * 3 * 8192);
             uint8_t* gsm = smem + w * P_WG;
             const int hk = it.h / (p.H_v / p.H_k);
-            for (int b = 0; b < nbox; ++b) {
-              tma_load_3d(gsm + P_KQ + b * 16384, &tm_k, fb, b * 64, hk, it.t0);
-              tma_load_3d(gsm + P_KQ + b * 16384 + 8192, &tm_q, fb, b * 64, hk, it.t0);
-              tma_load_3d(gsm + P_V + b * 8192, &tm_v, fb, b * 64, it.h, it.t0);
+            for (int b2 = 0; b2 < nbox; ++b2) {
+              tma_load_3d(gsm + P_KQ + b2 * 16384, &tm_k, fb, b2 * 64, hk, it.t0);
+              tma_load_3d(gsm + P_KQ + b2 * 16384 + 8192, &tm_q, fb, b2 * 64, hk, it.t0);
+              tma_load_3d(gsm + P_V + b2 * 8192, &tm_v, fb, b2 * 64, it.h, it.t0);
             }
             last_k[w] = k;
           }
@@ -711,20 +759,21 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t id_wu = make_idesc_bf16(128, 64, 1, 0);
         ChunkIter itp[2];
         int kp[2] = {0, 0}, kw[2] = {0, 0};
-        for (int w = 0; w < 2; ++w) {
-          it_start(itp[w], p, u0, ustep);
-          it_align(itp[w], p, ustep, par + 2 * w);
-        }
+        it_start(itp[0], p, u0, ustep);
+        it_align(itp[0], p, ustep, P, par, 0);
+        it_start(itp[1], p, u0, ustep);
+        it_align(itp[1], p, ustep, P, par, 1);
         long long last = clock64();
         while (true) {
           bool pending = false, prog = false;
+#pragma unroll
           for (int w = 0; w < 2; ++w) {
             const uint32_t g = sbase + w * P_WG;
             const uint32_t tm = tmem + PT_WG * w;
             if (itp[w].ok) {
               pending = true;
-              if (mbar_try_wait(&bars[PB_KQVF + w], kp[w] & 1) &&
-                  (kp[w] == 0 || mbar_try_wait(&bars[PB_P1FREE + w], (kp[w] - 1) & 1))) {
+              if (mbar_test_wait(&bars[PB_KQVF + w], kp[w] & 1) &&
+                  (kp[w] == 0 || mbar_test_wait(&bars[PB_P1FREE + w], (kp[w] - 1) & 1))) {
                 tc_fence_after();
                 for (int kk = 0; kk < ksteps_d; ++kk) {
                   const uint32_t a = g + P_KQ + (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -734,13 +783,13 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
                 mma_commit(&bars[PB_P1F + w]);
                 ++kp[w];
                 it_next(itp[w], p, ustep);
-                it_align(itp[w], p, ustep, par + 2 * w);
+                it_align(itp[w], p, ustep, P, par, w);
                 prog = true;
               }
             }
             if (kw[w] < kp[w]) {
               pending = true;
-              if (mbar_try_wait(&bars[PB_TREADY + w], kw[w] & 1)) {
+              if (mbar_test_wait(&bars[PB_TREADY + w], kw[w] & 1)) {
                 tc_fence_after();
                 for (int kk = 0; kk < 4; ++kk)
                   mma_bf16_ss(tm + PT_W, make_sdesc_sw128(g + P_KQ + kk * 2048, 16384, 1024),
@@ -758,17 +807,20 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
           if (!pending || *abort_flag) break;
           if (prog) {
             last = clock64();
-          } else if (clock64() - last > kSpinLimitCycles) {
-            *abort_flag = 1;
-            atomicOr(err, 2u);
-            break;
+          } else {
+            if (clock64() - last > kSpinLimitCycles) {
+              *abort_flag = 1;
+              atomicOr(err, 2u);
+              break;
+            }
+            __nanosleep(20);
           }
         }
         mma_commit(&bars[PB_DRAIN]);
         mbar_wait(&bars[PB_DRAIN], 0, nullptr, err, 8u);
       }
       __syncwarp();
-    } else {
+    } else if (warp < 8) {
       // ---------------- prep groups: 128 threads each, one item at a time
       const int w = warp >> 2;
       const int pt = tid & 127;
@@ -780,10 +832,10 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
       float* Xs = reinterpret_cast<float*>(gs + P_XS);
       float* gt = reinterpret_cast<float*>(gs + P_GATE);
       const uint32_t tm = tmem + PT_WG * w;
-      WgSync sync{&bars[PB_SYNC + w], 0};
+      const int gbar = 1 + 3 * w;  // this group's named barriers: gbar (all), gbar+1, gbar+2
       ChunkIter it;
       it_start(it, p, u0, ustep);
-      it_align(it, p, ustep, par + 2 * w);
+      it_align(it, p, ustep, P, par, w);
       int k = 0;
       while (it.ok) {
         const int c = it.c;
@@ -795,20 +847,20 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
           gt[PG_G + pt] = valid ? p.g[size_t(it.t0 + pt) * p.gb_stride + h] : 0.f;
           gt[PG_BET + pt] = valid ? p.beta[size_t(it.t0 + pt) * p.gb_stride + h] : 0.f;
         }
-        if (!sync(abort_flag, err)) break;
+        named_sync(gbar, 128);
         if (pt < 32) {  // inclusive scan of g over 64 rows (2 per lane)
           const float a0 = gt[PG_G + 2 * pt], a1 = gt[PG_G + 2 * pt + 1];
-          float s = a0 + a1;
+          float s2 = a0 + a1;
 #pragma unroll
           for (int off = 1; off < 32; off <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, s, off);
-            if (pt >= off) s += y;
+            const float y = __shfl_up_sync(0xffffffffu, s2, off);
+            if (pt >= off) s2 += y;
           }
-          const float excl = s - (a0 + a1);
+          const float excl = s2 - (a0 + a1);
           gt[PG_G + 2 * pt] = excl + a0;
           gt[PG_G + 2 * pt + 1] = excl + a0 + a1;
         }
-        if (!sync(abort_flag, err)) break;
+        named_sync(gbar, 128);
         {
           const float GC = gt[PG_G + 63];
           if (pt < 64) {
@@ -820,123 +872,150 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
             gt[PG_E1 + pt] = __expf(Gr - gt[PG_G + (pt & ~15)]);
           }
           for (int e = pt; e < 256; e += 128) {  // E2[b][s] = e^{G_{16b} - G_s}, s < 16b
-            const int bb = e >> 6, s = e & 63;
-            gt[PG_E2 + e] = (s < 16 * bb) ? __expf(gt[PG_G + 16 * bb] - gt[PG_G + s]) : 0.f;
+            const int bb = e >> 6, s2 = e & 63;
+            gt[PG_E2 + e] = (s2 < 16 * bb) ? __expf(gt[PG_G + 16 * bb] - gt[PG_G + s2]) : 0.f;
           }
           if (pt == 0) gt[PG_DEC] = __expf(GC);
         }
-        if (!sync(abort_flag, err)) break;
-        // ---- P1 row pt: K K^T (pt < 64) or Q K^T (pt >= 64)
-        if (!mbar_wait(&bars[PB_P1F + w], k & 1, abort_flag, err, 4u)) break;
+        named_sync(gbar, 128);
+        // ---- P1 row pt: K K^T (pt < 64) or Q K^T (pt >= 64), times e^{G_r - G_s}
+        // (s <= r): two factors <= 1 for the blocks of s before r's 16-row
+        // block, a direct exponential inside it.
+        if (!named_all(gbar, 128, mbar_wait(&bars[PB_P1F + w], k & 1, abort_flag, err, 4u))) break;
         tc_fence_after();
         {
-          float row[64];
-          tmem_ld64(tm + lane_off + PT_P1, row);
-          tc_fence_before();
-          mbar_arrive(&bars[PB_P1FREE + w]);
-          // row[s] *= e^{G_r - G_s} (s <= r): two factors <= 1 for the blocks of s
-          // before r's 16-row block, a direct exponential inside it.
           const int r = pt & 63, rb = r >> 4;
           const float Gr = gt[PG_G + r];
           const float e1 = gt[PG_E1 + r];
+          const float br = gt[PG_BET + r];
           const float* e2 = gt + PG_E2 + 64 * rb;
+          float v[64];
+          tmem_ld32(tm + lane_off + PT_P1, *reinterpret_cast<float(*)[32]>(v));
+          tmem_ld32(tm + lane_off + PT_P1 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(&bars[PB_P1FREE + w]);
 #pragma unroll
           for (int sb = 0; sb < 4; ++sb) {
+            float f[16];
             if (sb < rb) {
 #pragma unroll
-              for (int jj = 0; jj < 16; ++jj) row[16 * sb + jj] *= e1 * e2[16 * sb + jj];
+              for (int jj = 0; jj < 16; jj += 4) {
+                const float4 e4 = *reinterpret_cast<const float4*>(e2 + 16 * sb + jj);
+                f[jj] = e1 * e4.x;
+                f[jj + 1] = e1 * e4.y;
+                f[jj + 2] = e1 * e4.z;
+                f[jj + 3] = e1 * e4.w;
+              }
             } else if (sb == rb) {
 #pragma unroll
-              for (int jj = 0; jj < 16; ++jj) {
-                const int s = 16 * sb + jj;
-                row[s] = (s <= r) ? row[s] * __expf(Gr - gt[PG_G + s]) : 0.f;
+              for (int jj = 0; jj < 16; jj += 4) {
+                const int s2 = 16 * sb + jj;
+                const float4 g4 = *reinterpret_cast<const float4*>(gt + PG_G + s2);
+                f[jj] = (s2 <= r) ? __expf(Gr - g4.x) : 0.f;
+                f[jj + 1] = (s2 + 1 <= r) ? __expf(Gr - g4.y) : 0.f;
+                f[jj + 2] = (s2 + 2 <= r) ? __expf(Gr - g4.z) : 0.f;
+                f[jj + 3] = (s2 + 3 <= r) ? __expf(Gr - g4.w) : 0.f;
               }
             } else {
 #pragma unroll
-              for (int jj = 0; jj < 16; ++jj) row[16 * sb + jj] = 0.f;
+              for (int jj = 0; jj < 16; ++jj) f[jj] = 0.f;
+            }
+            if (pt < 64) {  // A[r][s] = beta_r e^{G_r-G_s} k_r.k_s, s < r
+#pragma unroll
+              for (int jj = 0; jj < 16; jj += 4) {
+                const int s2 = 16 * sb + jj;
+                *reinterpret_cast<float4*>(Af + r * kAS + s2) = make_float4(
+                    s2 + 0 < r ? br * f[jj] * v[s2] : 0.f,
+                    s2 + 1 < r ? br * f[jj + 1] * v[s2 + 1] : 0.f,
+                    s2 + 2 < r ? br * f[jj + 2] * v[s2 + 2] : 0.f,
+                    s2 + 3 < r ? br * f[jj + 3] * v[s2 + 3] : 0.f);
+              }
+            } else {  // Aqk[r][s] = scale e^{G_r-G_s} q_r.k_s, s <= r  (bf16, swizzled)
+              const float sc = p.scale;
+#pragma unroll
+              for (int hc = 0; hc < 2; ++hc) {
+                const int s2 = 16 * sb + 8 * hc;
+                st_shared_v4(
+                    g + P_AQK + sw128_offset(r, (2 * sb + hc) * 16),
+                    pack_bf16x2(sc * f[8 * hc] * v[s2], sc * f[8 * hc + 1] * v[s2 + 1]),
+                    pack_bf16x2(sc * f[8 * hc + 2] * v[s2 + 2], sc * f[8 * hc + 3] * v[s2 + 3]),
+                    pack_bf16x2(sc * f[8 * hc + 4] * v[s2 + 4], sc * f[8 * hc + 5] * v[s2 + 5]),
+                    pack_bf16x2(sc * f[8 * hc + 6] * v[s2 + 6], sc * f[8 * hc + 7] * v[s2 + 7]));
+              }
             }
           }
-          if (pt < 64) {
-            const float br = gt[PG_BET + r];
-#pragma unroll
-            for (int s = 0; s < 64; s += 4)
-              *reinterpret_cast<float4*>(Af + r * kAS + s) =
-                  make_float4(s + 0 < r ? br * row[s] : 0.f, s + 1 < r ? br * row[s + 1] : 0.f,
-                              s + 2 < r ? br * row[s + 2] : 0.f, s + 3 < r ? br * row[s + 3] : 0.f);
-          } else {
-            const float sc = p.scale;
-#pragma unroll
-            for (int s = 0; s < 64; ++s) row[s] *= sc;
-            uint32_t pk[32];
-            pack_chunks<8>(row, pk);
-            uint4* dst = reinterpret_cast<uint4*>(gs + P_AQK + r * 128);
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc)
-              dst[cc] = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-          }
         }
-        if (!sync(abort_flag, err)) break;
+        named_sync(gbar, 128);
         // ---- T = (I + A)^{-1}
-        if (!invert_unit_lower64(Af, Tf, Xs, pt, sync, abort_flag, err)) break;
+        invert_unit_lower64(Af, Tf, Xs, pt, gbar);
         // ---- T1 = T diag(beta e^G) (rows pt < 64), T2 = T diag(beta) (rows pt >= 64)
         {
           const int r = pt & 63;
           const float* scv = gt + (pt < 64 ? PG_BEG : PG_BET);
-          float row[64];
-#pragma unroll
-          for (int s = 0; s < 64; s += 4) {
-            const float4 t4 = *reinterpret_cast<const float4*>(Tf + r * kAS + s);
-            const float4 s4 = *reinterpret_cast<const float4*>(scv + s);
-            row[s] = s + 0 <= r ? t4.x * s4.x : 0.f;
-            row[s + 1] = s + 1 <= r ? t4.y * s4.y : 0.f;
-            row[s + 2] = s + 2 <= r ? t4.z * s4.z : 0.f;
-            row[s + 3] = s + 3 <= r ? t4.w * s4.w : 0.f;
+          const uint32_t tile = g + (pt < 64 ? P_T1B : P_T2B);
+#pragma unroll 1
+          for (int cc = 0; cc < 8; ++cc) {
+            const float4 ta = *reinterpret_cast<const float4*>(Tf + r * kAS + 8 * cc);
+            const float4 tb2 = *reinterpret_cast<const float4*>(Tf + r * kAS + 8 * cc + 4);
+            const float4 sa = *reinterpret_cast<const float4*>(scv + 8 * cc);
+            const float4 sb2 = *reinterpret_cast<const float4*>(scv + 8 * cc + 4);
+            const int s0 = 8 * cc;
+            st_shared_v4(tile + sw128_offset(r, cc * 16),
+                         pack_bf16x2(s0 + 0 <= r ? ta.x * sa.x : 0.f, s0 + 1 <= r ? ta.y * sa.y : 0.f),
+                         pack_bf16x2(s0 + 2 <= r ? ta.z * sa.z : 0.f, s0 + 3 <= r ? ta.w * sa.w : 0.f),
+                         pack_bf16x2(s0 + 4 <= r ? tb2.x * sb2.x : 0.f,
+                                     s0 + 5 <= r ? tb2.y * sb2.y : 0.f),
+                         pack_bf16x2(s0 + 6 <= r ? tb2.z * sb2.z : 0.f,
+                                     s0 + 7 <= r ? tb2.w * sb2.w : 0.f));
           }
-          st_row64_bf16(g + (pt < 64 ? P_T1B : P_T2B), uint32_t(r), row);
         }
         fence_proxy_async_smem();
         mbar_arrive(&bars[PB_TREADY + w]);
-        // ---- W^T, U^T, Aqk and the gate factors into the spine's slot
-        // group 0 writes slot items 0, 2, 4 (the first needs no release), group 1
-        // items 1, 3, 5 (each needs the release of the item before it)
-        if (!mbar_wait_cluster(&bars[PB_SLOTFREE + w], (k + 1 + w) & 1, abort_flag, err, 4u))
-          break;
-        if (!mbar_wait(&bars[PB_WUF + w], k & 1, abort_flag, err, 4u)) break;
+        // ---- W^T, U^T rows into the staging (the A / T scratch is free now),
+        // then the whole entry to global ring slot c & 3
+        if (!named_all(gbar, 128, mbar_wait(&bars[PB_WUF + w], k & 1, abort_flag, err, 4u))) break;
         tc_fence_after();
-        {
-          float row[64];
-          uint32_t pk[32];
-          tmem_ld64(tm + lane_off + PT_W, row);  // W^T row pt (d_k index)
-          pack_chunks<8>(row, pk);
-          st_row64_remote(spine_slot + SL_W, uint32_t(pt), pk);
-          tmem_ld64(tm + lane_off + PT_U, row);  // U^T row pt (d_v index)
-          pack_chunks<8>(row, pk);
-          st_row64_remote(spine_slot + SL_U, uint32_t(pt), pk);
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {  // W^T row pt (d_k index), U^T row pt (d_v index)
+          float wv[32], uv[32];
+          tmem_ld32(tm + lane_off + PT_W + 32u * hf, wv);
+          tmem_ld32(tm + lane_off + PT_U + 32u * hf, uv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int hc = 0; hc < 4; ++hc) {
+            const uint32_t off = sw128_offset(pt, (4 * hf + hc) * 16);
+            st_shared_v4(g + P_AF + G_W + off, pack_bf16x2(wv[8 * hc], wv[8 * hc + 1]),
+                         pack_bf16x2(wv[8 * hc + 2], wv[8 * hc + 3]),
+                         pack_bf16x2(wv[8 * hc + 4], wv[8 * hc + 5]),
+                         pack_bf16x2(wv[8 * hc + 6], wv[8 * hc + 7]));
+            st_shared_v4(g + P_AF + G_U + off, pack_bf16x2(uv[8 * hc], uv[8 * hc + 1]),
+                         pack_bf16x2(uv[8 * hc + 2], uv[8 * hc + 3]),
+                         pack_bf16x2(uv[8 * hc + 4], uv[8 * hc + 5]),
+                         pack_bf16x2(uv[8 * hc + 6], uv[8 * hc + 7]));
+          }
         }
         tc_fence_before();
-        if (pt >= 64) {
-          const uint4* src = reinterpret_cast<const uint4*>(gs + P_AQK + (pt - 64) * 128);
-          uint32_t pk[32];
-#pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            const uint4 v4 = src[cc];
-            pk[4 * cc] = v4.x;
-            pk[4 * cc + 1] = v4.y;
-            pk[4 * cc + 2] = v4.z;
-            pk[4 * cc + 3] = v4.w;
+        fence_proxy_async_smem();
+        named_sync(gbar, 128);
+        if (pt == 0) {
+          // ring entry c & 3 is free once the spine has loaded chunk c - 4
+          bool okr = mbar_wait_cluster(&bars[PB_GFREE + (c & 3)], ((c >> 2) & 1) ^ 1, abort_flag,
+                                       err, 4u);
+          if (okr) {
+            uint8_t* dst = ring + (c & 3) * SLOT_G;
+            bulk_store_s2g(dst + G_W, gs + P_AF, 32768);
+            bulk_store_s2g(dst + G_AQK, gs + P_AQK, 8192);
+            bulk_store_s2g(dst + G_GATE, gs + P_GATE + PG_EG * 4, G_GATE_BYTES);
+            tma_store_commit();
+            tma_store_wait_all<0>();
+            fence_proxy_async_global();
+            mbar_arrive_remote(mapa_shared(sbase + S_BARS + (SB_GREADY + (c & 3)) * 8, 0));
           }
-          st_row64_remote(spine_slot + SL_AQK, uint32_t(pt - 64), pk);
         }
-        if (pt < 33) {  // e^{G_r} [0, 64), e^{G_C - G_r} [64, 128), e^{G_C} at 128
-          const float* src = gt + PG_EG + 4 * pt;  // PG_EG, PG_ECG, PG_DEC are contiguous
-          st_cluster_v4(spine_gate + 16 * pt, __float_as_uint(src[0]), __float_as_uint(src[1]),
-                        __float_as_uint(src[2]), __float_as_uint(src[3]));
-        }
-        fence_proxy_async_cluster();
-        mbar_arrive_remote(spine_slotf);
         ++k;
         it_next(it, p, ustep);
-        it_align(it, p, ustep, par + 2 * w);
+        it_align(it, p, ustep, P, par, w);
       }
     }
   }
@@ -947,7 +1026,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     const int exit_bar = spine ? SB_EXIT : PB_EXIT;
     mbar_arrive(&bars[exit_bar]);
-    for (uint32_t r = 0; r < kCluster; ++r) {
+    for (uint32_t r = 0; r < ncta; ++r) {
       if (r == rank) continue;
       const uint32_t off = (r == 0 ? S_BARS + SB_EXIT * 8 : P_BARS + PB_EXIT * 8);
       mbar_arrive_remote(mapa_shared(sbase + off, r));
@@ -958,14 +1037,68 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-size_t prefill_workspace_bytes(int, int, int, int, int) { return 0; }
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+namespace {
+
+// Resident clusters of `ncta` CTAs for this kernel on the current device.
+int max_active_clusters(int ncta) {
+  static int cache[64][4] = {{0}};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int* slot = (dev >= 0 && dev < 64) ? &cache[dev][ncta] : nullptr;
+  if (slot != nullptr && *slot > 0) return *slot;
+  int m = 0;
+  cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       int(kSmemAlloc));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ncta * (sm_count() / ncta));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemAlloc;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = ncta;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  if (cudaOccupancyMaxActiveClusters(&m, prefill_kernel, &cfg) != cudaSuccess || m <= 0) {
+    cudaGetLastError();
+    m = sm_count() / ncta;
+  }
+  if (slot != nullptr) *slot = m;
+  return m;
+}
+
+// Cluster shape and count for `units` (sequence, v-head) units: three CTAs
+// per unit (two preps) unless that leaves units for a second round of
+// clusters while two-CTA clusters would need fewer rounds.
+void plan(int units, int* ncta, int* clusters) {
+  const int m3 = max_active_clusters(3), m2 = max_active_clusters(2);
+  const int rounds3 = (units + m3 - 1) / m3, rounds2 = (units + m2 - 1) / m2;
+  *ncta = rounds2 < rounds3 ? 2 : 3;
+  const int mc = *ncta == 3 ? m3 : m2;
+  *clusters = units < mc ? units : mc;
+}
+
+}  // namespace
+
+size_t prefill_workspace_bytes(int total_tokens, int num_seqs, int H_k, int H_v, int D) {
+  (void)total_tokens;
+  (void)H_k;
+  (void)D;
+  int ncta = 3, clusters = 0;
+  plan(num_seqs * H_v, &ncta, &clusters);
+  return size_t(clusters) * kRing * SLOT_G;
+}
 
 cudaError_t launch_prefill(const uint16_t* q, const uint16_t* k, int qk_stride,
                            const uint16_t* v, int v_stride, const float* g, const float* beta,
                            int gb_stride, const int32_t* cu_seqlens, int num_seqs,
                            int total_tokens, const float* h0, float* hT, uint16_t* o, int H_k,
                            int H_v, int D, float scale, void* workspace, cudaStream_t s) {
-  (void)workspace;
   CUtensorMap tq, tk, tv;
   {
     uint64_t dims[3] = {uint64_t(D), uint64_t(H_k), uint64_t(total_tokens)};
@@ -987,6 +1120,7 @@ cudaError_t launch_prefill(const uint16_t* q, const uint16_t* k, int qk_stride,
   p.h0 = h0;
   p.hT = hT;
   p.o = o;
+  p.ws = static_cast<uint8_t*>(workspace);
   p.gb_stride = gb_stride;
   p.num_seqs = num_seqs;
   p.total_tokens = total_tokens;
@@ -997,34 +1131,22 @@ cudaError_t launch_prefill(const uint16_t* q, const uint16_t* k, int qk_stride,
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(kSmemAlloc));
   if (e != cudaSuccess) return e;
-  // As many clusters as can be resident at once (each cluster then walks its
-  // share of the units), never more than there are units.
-  static int max_clusters_cache[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  int max_clusters = (dev >= 0 && dev < 64) ? max_clusters_cache[dev] : 0;
-  if (max_clusters <= 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kCluster * (sm_count() / kCluster));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemAlloc;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = kCluster;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&max_clusters, prefill_kernel, &cfg) != cudaSuccess ||
-        max_clusters <= 0) {
-      cudaGetLastError();
-      max_clusters = sm_count() / kCluster;
-    }
-    if (dev >= 0 && dev < 64) max_clusters_cache[dev] = max_clusters;
-  }
-  const int units = num_seqs * H_v;
-  const int clusters = units < max_clusters ? units : max_clusters;
-  prefill_kernel<<<clusters * kCluster, kThreads, kSmemAlloc, s>>>(tq, tk, tv, p);
+  int ncta = 3, clusters = 0;
+  plan(num_seqs * H_v, &ncta, &clusters);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(clusters * ncta);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemAlloc;
+  cfg.stream = s;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = ncta;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, prefill_kernel, tq, tk, tv, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
