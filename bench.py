@@ -65,16 +65,25 @@ def peaks():
 
 
 def profiled_traffic():
-    """dram read+write bytes per prefill launch from the committed ncu summary."""
+    """dram read+write bytes per prefill launch from the committed ncu summary,
+    or None once gdn_prefill.cu no longer matches the source that was profiled."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "prefill_dram_traffic.txt")
+    src = os.path.join(ROOT, "linear_attention_ssm_gdn_b200", "csrc", "gdn_prefill.cu")
     try:
+        vals = {}
         with open(path) as f:
             for line in f:
-                if line.startswith("bytes_per_launch_full_workload"):
-                    return float(line.split("=")[1].split()[0])
+                if "=" in line and not line.startswith("#"):
+                    k, v = line.split("=", 1)
+                    vals[k.strip()] = v.split()[0]
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        if vals.get("source_sha256") != sha:
+            return None
+        return float(vals["bytes_per_launch_full_workload"])
     except Exception:
-        pass
-    return None
+        return None
 
 
 # --------------------------------------------------------------------------
