@@ -307,6 +307,19 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
 }  // namespace gdn
 
 // ---------------------------------------------------------------------------
@@ -425,6 +438,37 @@ __device__ __forceinline__ void bulk_store_s2g(void* dst, const void* src, uint3
 
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// gpu-scope acquire load / release store of a 32-bit flag in global memory.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Poll a flag in global memory until it reaches `target` (values only grow).
+// Gives up when *gabort becomes nonzero or after kSpinLimitCycles; on a
+// timeout it sets *gabort and ORs `err_bit` into *err.
+static __device__ __noinline__ bool poll_geq(const uint32_t* flag, uint32_t target,
+                                             volatile uint32_t* gabort, uint32_t* err,
+                                             uint32_t err_bit) {
+  if (ld_acquire_gpu(flag) >= target) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (ld_acquire_gpu(flag) >= target) return true;
+    if (*gabort != 0u) return false;
+    if (clock64() - t0 > kSpinLimitCycles) {
+      atomicExch(const_cast<uint32_t*>(gabort), 1u);
+      if (err != nullptr) atomicOr(err, err_bit);
+      return false;
+    }
+    __nanosleep(32);
+  }
 }
 
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {

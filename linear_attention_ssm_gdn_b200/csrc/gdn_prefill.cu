@@ -2,25 +2,28 @@
 //
 // Page "ssm_gdn_tc_route.rs" names the piece this kernel replaces: the prefill
 // "state spine" (chunk_delta_h) that carries the f32 recurrent state across
-// chunks with bf16 tensor-core operands and an f32 accumulator.  Here the whole
-// chunk step is one kernel, and each (sequence, v-head) unit is handled by a
-// cluster of two or three CTAs on as many SMs:
+// chunks with bf16 tensor-core operands and an f32 accumulator.  Here the
+// whole chunk step is one persistent kernel with one CTA per SM (a cooperative
+// launch, so that every CTA is resident) in two roles:
 //
-//   rank 0, the SPINE, runs the per-chunk critical chain on tcgen05 MMAs with
-//     TMEM accumulators (M = d_v = 128 lanes), keeping H^T in TMEM (f32):
+//   SPINES (the first S CTAs) each own (sequence, v-head) units u = s, s+S, ...
+//     and run their per-chunk critical chain on tcgen05 MMAs with TMEM
+//     accumulators (M = d_v = 128 lanes), keeping H^T in TMEM (f32):
 //       Vn^T = U^T - H^T W^T,   H^T <- e^{G_C} H^T + (e^{G_C - G_r} Vn)^T K,
 //     and the outputs  o_r = e^{G_r} scale (Q H)_r + (Aqk Vn)_r;
-//   ranks 1 (and 2), the PREPS, compute everything that does not depend on H,
-//     each for its share of the chunks, two chunks at a time per CTA:
+//   PREPS (all other CTAs) compute everything that does not depend on H, for
+//     chunk items taken from one global order (chunk index major, spine minor;
+//     prep p takes every Pn-th item), two items at a time per CTA:
 //       P1 = [K;Q] K^T                                 (MMA)
 //       A[r][s]   = beta_r e^{G_r-G_s} k_r.k_s, s < r   (f32)
 //       Aqk[r][s] = scale e^{G_r-G_s} q_r.k_s, s <= r
 //       T = (I + A)^{-1}                               (blocked, f32, CUDA cores)
 //       W^T = K^T (T diag(beta e^G))^T,  U^T = V^T (T diag(beta))^T   (MMAs)
-//     and bulk-store W^T, U^T, Aqk (bf16) and the gate factors into a 4-entry
-//     ring in global memory (the workspace; it stays in L2), from where the
-//     spine's TMA warp bulk-loads them into one of two shared-memory slots.
-//     Hand-offs are mbarrier arrivals across the cluster.
+//     and bulk-store W^T, U^T, Aqk (bf16) and the gate factors into the
+//     owning spine's ring of kRing entries in the workspace (it stays in L2).
+//   Hand-offs are release/acquire flags in the workspace: a prep publishes
+//   entry j of spine s after its bulk store completed; the spine publishes that
+//   it has copied the entry out, which frees it for item j + kRing.
 //
 // This is the WY/UT chunk form: within a chunk of rows r = 0..L-1 with
 // G_r = g_0 + ... + g_r, (I + A) Vn = diag(beta) V - diag(beta e^G) K H, the
@@ -30,9 +33,14 @@
 // d_k = d_v = 64 runs the same code with the upper halves of every tile zero.
 //
 // No TMA multicast: every CTA loads its own K/Q/V tiles (L2 serves re-reads).
-// Every mbarrier wait is bounded (gdn_device.cuh); a timeout sets
-// g_err_prefill and the kernel returns instead of hanging.  Named barriers are
-// used only among threads that are all guaranteed to arrive.
+// Every wait is bounded (gdn_device.cuh): a timeout sets g_err_prefill and a
+// grid-wide abort word, and every CTA then returns instead of waiting.  Named
+// barriers are used only among threads that are all guaranteed to arrive.
+//
+// Progress: prep items are produced in increasing global index and consumed by
+// each spine in increasing chunk order; the oldest unfinished item never waits
+// on a younger one (its ring entry was freed by an older, already produced
+// item), so the pipeline cannot deadlock while all CTAs are resident.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -47,15 +55,19 @@ __device__ uint32_t g_err_prefill;
 namespace pf {
 
 constexpr int C = 64;          // chunk rows
-constexpr int kThreads = 320;  // 10 warps
+constexpr int kThreads = 384;  // 12 warps
 constexpr int kAS = 68;        // f32 row stride of the A / T scratch (16-byte rows)
+constexpr int kRing = 4;       // ring entries per spine
+constexpr int kMaxSpines = 256;
 
-// ---- global slot-ring entry (workspace): W^T | U^T | Aqk | gate factors
+// ---- ring entry (workspace): W^T | U^T | Aqk | gate factors
 constexpr uint32_t G_W = 0, G_U = 16384, G_AQK = 32768, G_GATE = 40960;
 constexpr uint32_t G_GATE_BYTES = 528;  // e^{G_r} 64 | e^{G_C-G_r} 64 | e^{G_C} | pad
 constexpr uint32_t SLOT_G = 41984;      // 41 KB, a multiple of 1024
 constexpr uint32_t SLOT_TX = G_GATE + G_GATE_BYTES;
-constexpr int kRing = 4;
+// ---- flags (workspace head): one 64-byte line for the abort word, then one
+// line per (spine, ring entry): ready count at +0, free count at +32 bytes.
+constexpr uint32_t kFlagLine = 64;
 
 // ---- spine shared memory (bytes from a 1024-aligned base)
 constexpr uint32_t S_KQ = 0;            // [2 stages][2 boxes][K 64x128B | Q 64x128B]
@@ -64,9 +76,9 @@ constexpr uint32_t S_VN = 98304;        // Vn^T bf16 [128 x 128B]
 constexpr uint32_t S_VNS = 114688;      // scaled Vn^T bf16
 constexpr uint32_t S_SLOT = 131072;     // 2 slots of {W^T, U^T, Aqk}, same layout as G_*
 constexpr uint32_t SL_BYTES = 40960;
-constexpr uint32_t S_SGATE = S_SLOT + 2 * SL_BYTES;  // 2 x 528 B of gate factors
-constexpr uint32_t SG_FLOATS = 132;
-constexpr uint32_t S_BARS = S_SGATE + 2 * G_GATE_BYTES;
+constexpr uint32_t S_SGATE = S_SLOT + 2 * SL_BYTES;      // 2 x 528 B of gate factors
+constexpr uint32_t S_OSTG = S_SGATE + 2 * G_GATE_BYTES;  // output transpose: 4 warps x 2 x 1 KB
+constexpr uint32_t S_BARS = S_OSTG + 8192;
 // ---- prep shared memory: two item groups of P_WG bytes
 constexpr uint32_t P_KQ = 0;        // [2 boxes][K | Q]
 constexpr uint32_t P_V = 32768;     // [2 boxes][64 x 128B]
@@ -75,42 +87,45 @@ constexpr uint32_t P_T2B = 57344;   // T diag(beta) bf16
 constexpr uint32_t P_AF = 65536;    // A f32 [64][kAS]; later the W^T | U^T staging
 constexpr uint32_t P_TF = P_AF + 64 * kAS * 4;  // T f32 [64][kAS]
 constexpr uint32_t P_XS = P_T1B;    // inverse scratch (32x32 f32), in the T1/T2 tiles' space
-constexpr uint32_t P_GATE = P_TF + 64 * kAS * 4;
+constexpr uint32_t P_GATE = P_TF + 64 * kAS * 4;  // 2 gate blocks of PG_BYTES
 constexpr int PG_G = 0, PG_BET = 64, PG_E1 = 128, PG_E2 = 192, PG_BEG = 448, PG_EG = 512,
-              PG_ECG = 576, PG_DEC = 640;  // floats; PG_EG..PG_DEC+3 is the gate block
-constexpr uint32_t P_AQK = (P_GATE + 644 * 4 + 1023) / 1024 * 1024;  // Aqk bf16 staging
+              PG_ECG = 576, PG_DEC = 640;  // floats; PG_EG..PG_DEC+3 is the published block
+constexpr uint32_t PG_BYTES = 644 * 4;
+constexpr uint32_t P_AQK = (P_GATE + 2 * PG_BYTES + 1023) / 1024 * 1024;  // Aqk bf16 staging
 constexpr uint32_t P_WG = P_AQK + 8192;
 constexpr uint32_t P_BARS = 2 * P_WG;
-constexpr uint32_t BAR_BYTES = 24 * 8;
+constexpr uint32_t BAR_BYTES = 32 * 8;
+constexpr uint32_t kMiscBytes = 16 + 4 * kMaxSpines;  // TMEM base, abort word, chunks per spine
 constexpr uint32_t kSmemBytes =
-    ((S_BARS > P_BARS ? S_BARS : P_BARS) + BAR_BYTES + 16 + 15) / 16 * 16;
+    ((S_BARS > P_BARS ? S_BARS : P_BARS) + BAR_BYTES + kMiscBytes + 15) / 16 * 16;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 static_assert(S_BARS % 8 == 0 && P_BARS % 8 == 0, "barrier alignment");
 static_assert(P_AF + 32768 <= P_GATE, "W^T | U^T staging fits in the A / T scratch");
+static_assert((P_GATE + PG_EG * 4) % 16 == 0 && (P_GATE + PG_BYTES + PG_EG * 4) % 16 == 0,
+              "gate blocks are bulk-copy sources");
 
 // ---- barriers (spine)
 enum {
   SB_KQF = 0,      // +stage: K/Q tiles landed (TMA)
   SB_KQE = 2,      // +stage: K/Q tiles free (MMA commit)
   SB_SLOTF = 4,    // +slot: slot data landed (bulk loads)
-  SB_SFREE = 6,    // +slot: slot no longer read (128, epilogue warps)
-  SB_GREADY = 8,   // +ring: a prep stored this ring entry (1 remote arrival)
-  SB_VNFULL = 12,  // -H^T W^T done (commit)
-  SB_DHFULL = 13,  // H += dH done (commit)
-  SB_OFULL = 14,   // +buf: O1, O2 done (commit)
-  SB_OFREE = 16,   // +buf: O1, O2 read back (128)
-  SB_DRAIN = 18,
-  SB_EXIT = 19,
-  SB_COUNT = 20
+  SB_VNFULL = 6,   // -H^T W^T done (commit)
+  SB_DHFULL = 7,   // H += dH done (commit)
+  SB_OFULL = 8,    // +buf: O1, O2 done (commit)
+  SB_OFREE = 10,   // +buf: O1, O2 read back (128)
+  SB_DRAIN = 12,
+  SB_COUNT = 13
 };
-// ---- barriers (prep); per group w: base + w
+// ---- barriers (prep); per group w: base + w (GATEF / GATEE: base + 2w + b)
 enum {
   PB_KQVF = 0, PB_KQVE = 2, PB_P1F = 4, PB_P1FREE = 6, PB_TREADY = 8, PB_WUF = 10,
-  PB_GFREE = 12,  // +ring: the spine has loaded this ring entry (1 remote arrival)
-  PB_DRAIN = 16,
-  PB_EXIT = 17,
-  PB_COUNT = 18
+  PB_GATEF = 12,   // gate block (w, b) written (32, the loader warp)
+  PB_GATEE = 16,   // gate block (w, b) free again (1, the store warp)
+  PB_STAGED = 20,  // +w: W^T | U^T, Aqk staged (1)
+  PB_STGE = 22,    // +w: staging read by the bulk store (1)
+  PB_DRAIN = 24,
+  PB_COUNT = 25
 };
 
 // ---- TMEM columns
@@ -125,22 +140,40 @@ struct Params {
   const float* h0;
   float* hT;
   uint16_t* o;
-  uint8_t* ws;  // 4 global slot-ring entries of SLOT_G bytes per cluster
+  uint32_t* flags;  // abort line + S * kRing flag lines
+  uint8_t* ring;    // S * kRing entries of SLOT_G bytes
   int gb_stride, num_seqs, total_tokens, H_k, H_v, D;
+  int S;  // spine CTAs: blockIdx.x < S; the others are preps
   float scale;
 };
 
-// Walks the chunks of the units this cluster owns (u = cluster, += clusters);
-// `c` counts chunks over all of them and is the same in every role.
-struct ChunkIter {
-  int u, n, h, t0, tb, te, c;
-  bool ok;
-};
+__device__ __forceinline__ uint32_t* ready_flag(const Params& p, int s, int e) {
+  return p.flags + (1 + s * kRing + e) * (kFlagLine / 4);
+}
+__device__ __forceinline__ uint32_t* free_flag(const Params& p, int s, int e) {
+  return ready_flag(p, s, e) + 8;
+}
+__device__ __forceinline__ uint8_t* ring_entry(const Params& p, int s, int e) {
+  return p.ring + size_t(s * kRing + e) * SLOT_G;
+}
 
 __device__ __forceinline__ void seq_range(const Params& p, int n, int& b, int& e) {
   b = min(max(p.cu_seqlens[n], 0), p.total_tokens);
   e = min(max(p.cu_seqlens[n + 1], b), p.total_tokens);
 }
+
+__device__ __forceinline__ int unit_chunks(const Params& p, int u) {
+  int b, e;
+  seq_range(p, u / p.H_v, b, e);
+  return (e - b + C - 1) / C;
+}
+
+// Walks the chunks of the units a spine owns (u = s, s + S, ...); `c` counts
+// chunks over all of them.
+struct ChunkIter {
+  int u, n, h, t0, tb, te, c;
+  bool ok;
+};
 
 __device__ __forceinline__ void it_load_unit(ChunkIter& it, const Params& p) {
   it.n = it.u / p.H_v;
@@ -149,10 +182,10 @@ __device__ __forceinline__ void it_load_unit(ChunkIter& it, const Params& p) {
   it.t0 = it.tb;
 }
 
-__device__ __forceinline__ void it_skip_empty(ChunkIter& it, const Params& p, int ustep) {
+__device__ __forceinline__ void it_skip_empty(ChunkIter& it, const Params& p) {
   const int units = p.num_seqs * p.H_v;
   while (it.ok && it.t0 >= it.te) {
-    it.u += ustep;
+    it.u += p.S;
     if (it.u >= units) {
       it.ok = false;
       break;
@@ -161,31 +194,69 @@ __device__ __forceinline__ void it_skip_empty(ChunkIter& it, const Params& p, in
   }
 }
 
-__device__ __forceinline__ void it_start(ChunkIter& it, const Params& p, int u0, int ustep) {
-  it.u = u0;
+__device__ __forceinline__ void it_start(ChunkIter& it, const Params& p, int s) {
+  it.u = s;
   it.c = 0;
-  it.ok = u0 < p.num_seqs * p.H_v;
+  it.ok = s < p.num_seqs * p.H_v;
   if (it.ok) it_load_unit(it, p);
-  it_skip_empty(it, p, ustep);
+  it_skip_empty(it, p);
 }
 
-__device__ __forceinline__ void it_next(ChunkIter& it, const Params& p, int ustep) {
+__device__ __forceinline__ void it_next(ChunkIter& it, const Params& p) {
   it.t0 += C;
   ++it.c;
-  it_skip_empty(it, p, ustep);
+  it_skip_empty(it, p);
 }
 
-// Advance to the first chunk at or after the current one that prep rank
-// 1 + par (of P) hands to its group w: c % P == par and (c / P) % 2 == w.
-__device__ __forceinline__ void it_align(ChunkIter& it, const Params& p, int ustep, int P, int par,
+// The items of one prep CTA: global item i = j * S + s (chunk j of spine s),
+// i = prank, prank + Pn, ...; k counts the valid ones (k & 1 picks the group).
+struct PrepIter {
+  int i, k, s, j, h, t0, L;
+  bool ok;
+};
+
+__device__ __forceinline__ bool pi_fill(PrepIter& it, const Params& p, const int* sJ, int iend) {
+  while (it.i < iend) {
+    const int s = it.i % p.S, j = it.i / p.S;
+    if (j < sJ[s]) {
+      const int units = p.num_seqs * p.H_v;
+      int jj = j;
+      for (int u = s; u < units; u += p.S) {
+        const int nc = unit_chunks(p, u);
+        if (jj < nc) {
+          int tb, te;
+          seq_range(p, u / p.H_v, tb, te);
+          it.s = s;
+          it.j = j;
+          it.h = u % p.H_v;
+          it.t0 = tb + jj * C;
+          it.L = min(C, te - it.t0);
+          return true;
+        }
+        jj -= nc;
+      }
+    }
+    it.i += gridDim.x - p.S;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void pi_start(PrepIter& it, const Params& p, const int* sJ, int iend,
+                                         int prank) {
+  it.i = prank;
+  it.k = 0;
+  it.ok = pi_fill(it, p, sJ, iend);
+}
+
+__device__ __forceinline__ void pi_next(PrepIter& it, const Params& p, const int* sJ, int iend) {
+  it.i += gridDim.x - p.S;
+  ++it.k;
+  it.ok = pi_fill(it, p, sJ, iend);
+}
+
+__device__ __forceinline__ void pi_align(PrepIter& it, const Params& p, const int* sJ, int iend,
                                          int w) {
-  while (it.ok && (it.c % P != par || ((it.c / P) & 1) != w)) it_next(it, p, ustep);
-}
-
-template <int NCH>
-__device__ __forceinline__ void pack_chunks(const float* x, uint32_t* out) {
-#pragma unroll
-  for (int c = 0; c < 4 * NCH; ++c) out[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
+  while (it.ok && (it.k & 1) != w) pi_next(it, p, sJ, iend);
 }
 
 // Write 64 bf16 values as a 128-byte row of a 128B-swizzled tile (local smem).
@@ -197,45 +268,10 @@ __device__ __forceinline__ void st_row64_bf16(uint32_t tile, uint32_t row, const
                  pack_bf16x2(x[8 * c + 6], x[8 * c + 7]));
 }
 
-// Same, from 32 packed words, into another CTA's shared memory.
-__device__ __forceinline__ void st_row64_remote(uint32_t tile_cluster, uint32_t row,
-                                                const uint32_t* w) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c)
-    st_cluster_v4(tile_cluster + sw128_offset(row, c * 16), w[4 * c], w[4 * c + 1], w[4 * c + 2],
-                  w[4 * c + 3]);
-}
-
-// Read 64 bf16 of a swizzled row back as f32.
-__device__ __forceinline__ void ld_row64_bf16(const uint8_t* tile, uint32_t row, float* x) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const uint4 v = *reinterpret_cast<const uint4*>(tile + sw128_offset(row, c * 16));
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      x[8 * c + 2 * k] = __uint_as_float(w[k] << 16);
-      x[8 * c + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-    }
-  }
-}
-
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* x) {
-  float a[32], b[32];
-  tmem_ld32(taddr, a);
-  tmem_ld32(taddr + 32, b);
-  tmem_ld_wait();
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    x[i] = a[i];
-    x[32 + i] = b[i];
-  }
-}
-
 // ---------------------------------------------------------------------------
-// Named (hardware) barriers among the threads of one prep group.  Used only
+// Named (hardware) barriers among a fixed set of warps.  Used only
 // where every thread of the group is guaranteed to arrive (no early exits in
-// between); after a bounded wait that may fail, group_all() first agrees on
+// between); after a bounded wait that may fail, named_all() first agrees on
 // the outcome so that all threads leave together.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
@@ -407,39 +443,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t rank = cluster_ctarank();
-  const uint32_t ncta = cluster_nctarank();  // 2 or 3: the spine and P = ncta - 1 preps
-  const int P = int(ncta) - 1;
-  const bool spine = rank == 0;
+  const bool spine = int(blockIdx.x) < p.S;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (spine ? S_BARS : P_BARS));
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);  // after 24 barrier slots
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 24) + 1;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + 32);
+  uint32_t* tmem_slot = misc;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  int* sJ = reinterpret_cast<int*>(misc + 4);  // chunks per spine (preps only)
+  volatile uint32_t* gabort = p.flags;
   uint32_t* err = &g_err_prefill;
 
   const int warp = int(warp_id_sync());
   const int tid = threadIdx.x;
+  const int lane = tid & 31;
   const int D = p.D;
   const int nbox = D / 64;
-  const int u0 = int(cluster_id_x());
-  const int ustep = int(num_clusters_x());
-  uint8_t* ring = p.ws + size_t(cluster_id_x()) * kRing * SLOT_G;
+  const int units = p.num_seqs * p.H_v;
+  const int vpg = p.H_v / p.H_k;
 
   for (uint32_t i = tid * 16; i < kSmemBytes; i += kThreads * 16)
     *reinterpret_cast<uint4*>(smem + i) = make_uint4(0, 0, 0, 0);
   __syncthreads();
   if (tid == 0) {
     if (spine) {
-      for (int b = 0; b < SB_COUNT; ++b) {
-        uint32_t cnt = 1;
-        if (b == SB_SFREE || b == SB_SFREE + 1 || b == SB_OFREE || b == SB_OFREE + 1) cnt = 128;
-        if (b == SB_EXIT) cnt = ncta;
-        mbar_init(&bars[b], cnt);
-      }
+      for (int b = 0; b < SB_COUNT; ++b)
+        mbar_init(&bars[b], (b == SB_OFREE || b == SB_OFREE + 1) ? 128u : 1u);
     } else {
       for (int b = 0; b < PB_COUNT; ++b) {
         uint32_t cnt = 1;
         if (b == PB_P1FREE || b == PB_P1FREE + 1 || b == PB_TREADY || b == PB_TREADY + 1) cnt = 128;
-        if (b == PB_EXIT) cnt = ncta;
+        if (b >= PB_GATEF && b < PB_GATEF + 4) cnt = 32;
         mbar_init(&bars[b], cnt);
       }
     }
@@ -449,86 +481,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
+  // Chunks per spine, for the preps' item walk.
+  int Jmax = 0;
+  if (!spine) {
+    for (int s = tid; s < p.S; s += kThreads) {
+      int J = 0;
+      for (int u = s; u < units; u += p.S) J += unit_chunks(p, u);
+      sJ[s] = J;
+    }
+  }
   if (warp == 0) tmem_alloc(tmem_slot, 512);
   __syncthreads();
-  cluster_sync_start();  // every CTA's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int ksteps_d = D / 16;
+  if (!spine)
+    for (int s = 0; s < p.S; ++s) Jmax = max(Jmax, sJ[s]);
+  const int iend = Jmax * p.S;  // items i < iend (some invalid: chunk j beyond its spine)
 
   if (spine) {
     // =====================================================================
-    // SPINE
+    // SPINE s = blockIdx.x
     // =====================================================================
-    if (warp == 8) {
-      // ---------------- TMA: K and Q tiles (2 stages) and the slot data of
-      // every chunk (2 shared-memory slots fed from the 4-entry global ring)
-      if (elect_one()) {
-        ChunkIter it;
-        it_start(it, p, u0, ustep);
-        int issued = 0;
-        while (it.ok) {
-          const int c = it.c, st = c & 1;
-          if (!mbar_wait(&bars[SB_KQE + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 1u)) break;
-          uint64_t* fb = &bars[SB_KQF + st];
-          mbar_arrive_expect_tx(fb, uint32_t(nbox) * 2 * 8192);
-          uint8_t* kq = smem + S_KQ + st * 32768;
-          const int hk = it.h / (p.H_v / p.H_k);
-          for (int b = 0; b < nbox; ++b) {
-            tma_load_3d(kq + b * 16384, &tm_k, fb, b * 64, hk, it.t0);
-            tma_load_3d(kq + b * 16384 + 8192, &tm_q, fb, b * 64, hk, it.t0);
-          }
-          // slot st: free once the epilogue is done with chunk c-2; the ring
-          // entry once a prep has stored chunk c there
-          if (!mbar_wait(&bars[SB_SFREE + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 1u)) break;
-          if (!mbar_wait_cluster(&bars[SB_GREADY + (c & 3)], (c >> 2) & 1, abort_flag, err, 1u))
-            break;
-          fence_proxy_async_global();
-          uint64_t* sb = &bars[SB_SLOTF + st];
-          mbar_arrive_expect_tx(sb, SLOT_TX);
-          const uint8_t* src = ring + (c & 3) * SLOT_G;
-          bulk_load_g2s(smem + S_SLOT + st * SL_BYTES, src, G_GATE, sb);
-          bulk_load_g2s(smem + S_SGATE + st * G_GATE_BYTES, src + G_GATE, G_GATE_BYTES, sb);
-          issued = c + 1;
-          it_next(it, p, ustep);
-        }
-        for (int cc = issued - 2; cc < issued; ++cc) {
-          if (cc < 0) continue;
-          mbar_wait(&bars[SB_KQF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
-          mbar_wait(&bars[SB_SLOTF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
-        }
-      }
-      __syncwarp();
-    } else if (warp < 4) {
-      // ---------------- state warps: thread j owns row j of H^T, kept in TMEM
-      // (f32, 128 columns at ST_H).  Per chunk: read H^T, write its bf16 copy
-      // (the A operand of Vn and O1) and write back e^{G_C} H^T, so that the dH
-      // MMA accumulates H_{c+1} = e^{G_C} H_c + dH in place.  Thread 0 also
-      // issues the chunk's MMAs right after the group's named barriers.
-      const int j = tid;
-      const bool issuer = j == 0;
-      const uint32_t lane_off = uint32_t(warp * 32) << 16;
-      const uint32_t th = tmem + lane_off + ST_H;
+    const int s = int(blockIdx.x);
+    if (warp < 8) {
+      // ---------------- state warps: warp w serves TMEM lane quadrant w & 3
+      // (row j of H^T) and half w >> 2 of the columns: d_k 64 hh .. 64 hh + 63
+      // of H^T, chunk rows 32 hh .. 32 hh + 31 of Vn^T.  Per chunk: read H^T,
+      // write its bf16 copy (the A operand of Vn and O1), write back
+      // e^{G_C} H^T so that the dH MMA accumulates H_{c+1} = e^{G_C} H_c + dH
+      // in place.  Thread 0 also issues the chunk's MMAs.
+      const int qd = warp & 3, hh = warp >> 2;
+      const int j = 32 * qd + lane;
+      const bool issuer = tid == 0;
+      const uint32_t lane_off = uint32_t(32 * qd) << 16;
+      const uint32_t th = tmem + lane_off + ST_H + 64u * uint32_t(hh);
       const bool jv = j < D;
-      const int units = p.num_seqs * p.H_v;
       const uint32_t id_vn = make_idesc_bf16(128, 64, 0, 1, /*b_neg=*/1);
       const uint32_t id_o = make_idesc_bf16(128, 64, 0, 0);
       const uint32_t id_dh = make_idesc_bf16(128, 128, 0, 1);
       int c = 0;
       bool ok = true;
-      for (int u = u0; u < units && ok; u += ustep) {
+      for (int u = s; u < units && ok; u += p.S) {
         const int n = u / p.H_v, h = u % p.H_v;
         int tb, te;
         seq_range(p, n, tb, te);
         const size_t state_off = (size_t(n) * p.H_v + h) * size_t(D) * D;
         const float* h0 = (p.h0 != nullptr && jv) ? p.h0 + state_off + j : nullptr;
 #pragma unroll 1
-        for (int q4 = 0; q4 < 4; ++q4) {  // H^T row j <- h0 (or zeros)
+        for (int q2 = 0; q2 < 2; ++q2) {  // H^T row j, this warp's 64 columns <- h0 (or zeros)
           float x[32];
+          const int k0 = 64 * hh + 32 * q2;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            x[i] = (h0 != nullptr && 32 * q4 + i < D) ? h0[size_t(32 * q4 + i) * D] : 0.f;
-          tmem_st32(th + 32u * q4, x);
+            x[i] = (h0 != nullptr && k0 + i < D) ? h0[size_t(k0 + i) * D] : 0.f;
+          tmem_st32(th + 32u * q2, x);
         }
         tmem_st_wait();
         for (int t0 = tb; t0 < te && ok; t0 += C, ++c) {
@@ -540,92 +547,87 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
           }
           ok = ok && mbar_wait(&bars[SB_SLOTF + st], (c >> 1) & 1, abort_flag, err, 16u);
-          if (ok && issuer)  // ring entry c & 3 has been copied in: the prep may reuse it
-            mbar_arrive_remote(
-                mapa_shared(sbase + P_BARS + (PB_GFREE + (c & 3)) * 8, 1 + uint32_t(c % P)));
+          if (issuer && ok) {
+            st_release_gpu(free_flag(p, s, c % kRing), uint32_t(c + 1));  // ring entry copied out
+            ok = mbar_wait(&bars[SB_KQF + st], (c >> 1) & 1, abort_flag, err, 2u);
+          }
           const float* sg = reinterpret_cast<const float*>(smem + S_SGATE + st * G_GATE_BYTES);
           const float dec = sg[128];
-#pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {  // 64 columns = one 128-byte box row at a time
+          {
             float x[64];
-            tmem_ld32(th + 64u * hh, *reinterpret_cast<float(*)[32]>(x));
-            tmem_ld32(th + 64u * hh + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+            tmem_ld32(th, *reinterpret_cast<float(*)[32]>(x));
+            tmem_ld32(th + 32, *reinterpret_cast<float(*)[32]>(x + 32));
             tmem_ld_wait();
-            st_row64_bf16(sbase + S_HT + hh * 16384, uint32_t(j), x);
+            st_row64_bf16(sbase + S_HT + uint32_t(hh) * 16384, uint32_t(j), x);
 #pragma unroll
             for (int i = 0; i < 64; ++i) x[i] *= dec;
-            tmem_st32(th + 64u * hh, *reinterpret_cast<float(*)[32]>(x));
-            tmem_st32(th + 64u * hh + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+            tmem_st32(th, *reinterpret_cast<float(*)[32]>(x));
+            tmem_st32(th + 32, *reinterpret_cast<float(*)[32]>(x + 32));
           }
           tmem_st_wait();
           fence_proxy_async_smem();
           tc_fence_before();
-          if (!named_all(1, 128, ok)) {
+          if (!named_all(1, 256, ok)) {
             ok = false;
             break;
           }
           if (issuer) {
             tc_fence_after();
-            ok = mbar_wait(&bars[SB_KQF + st], (c >> 1) & 1, abort_flag, err, 2u);
-            if (ok) {  // Vn^T := -H^T W^T   (U^T is added below)
+            // Vn^T := -H^T W^T   (U^T is added below)
+            for (int kk = 0; kk < ksteps_d; ++kk) {
+              const uint32_t a = sbase + S_HT + (kk >> 2) * 16384 + (kk & 3) * 32;
+              mma_bf16_ss(tmem + ST_VN, make_sdesc_sw128(a, 16, 1024),
+                          make_sdesc_sw128(slot + G_W + kk * 2048, 8192, 1024), id_vn, kk > 0);
+            }
+            mma_commit(&bars[SB_VNFULL]);
+            // O1^T = H^T Q^T into buffer st (free once the epilogue read chunk c-2)
+            ok = c < 2 || mbar_wait(&bars[SB_OFREE + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 2u);
+            if (ok) {
+              tc_fence_after();
               for (int kk = 0; kk < ksteps_d; ++kk) {
                 const uint32_t a = sbase + S_HT + (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16_ss(tmem + ST_VN, make_sdesc_sw128(a, 16, 1024),
-                            make_sdesc_sw128(slot + G_W + kk * 2048, 8192, 1024), id_vn, kk > 0);
-              }
-              mma_commit(&bars[SB_VNFULL]);
-              // O1^T = H^T Q^T into buffer st (free once the epilogue read chunk c-2)
-              ok = c < 2 ||
-                   mbar_wait(&bars[SB_OFREE + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 2u);
-              if (ok) {
-                tc_fence_after();
-                for (int kk = 0; kk < ksteps_d; ++kk) {
-                  const uint32_t a = sbase + S_HT + (kk >> 2) * 16384 + (kk & 3) * 32;
-                  const uint32_t b = kq + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32;
-                  mma_bf16_ss(tmem + ST_O1 + 64u * st, make_sdesc_sw128(a, 16, 1024),
-                              make_sdesc_sw128(b, 16, 1024), id_o, kk > 0);
-                }
+                const uint32_t b = kq + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32;
+                mma_bf16_ss(tmem + ST_O1 + 64u * st, make_sdesc_sw128(a, 16, 1024),
+                            make_sdesc_sw128(b, 16, 1024), id_o, kk > 0);
               }
             }
           }
-          // Vn = U - (H W)  ->  Vn^T and e^{G_C - G_r} Vn^T rows in bf16
+          // Vn = U - (H W)  ->  Vn^T and e^{G_C - G_r} Vn^T rows in bf16 (this
+          // warp: chunk rows 32 hh .. 32 hh + 31)
           ok = ok && mbar_wait(&bars[SB_VNFULL], c & 1, abort_flag, err, 16u);
           tc_fence_after();
           if (ok) {
             const uint8_t* urow = smem + S_SLOT + st * SL_BYTES + G_U;
-#pragma unroll 1
-            for (int hf = 0; hf < 2; ++hf) {  // 32 columns (four 16-byte chunks) at a time
-              float vn[32];
-              tmem_ld32(tmem + lane_off + ST_VN + 32u * hf, vn);
-              tmem_ld_wait();
+            float vn[32];
+            tmem_ld32(tmem + lane_off + ST_VN + 32u * uint32_t(hh), vn);
+            tmem_ld_wait();
 #pragma unroll
-              for (int hc = 0; hc < 4; ++hc) {
-                const int cc = 4 * hf + hc;
-                const uint4 uv = *reinterpret_cast<const uint4*>(urow + sw128_offset(j, cc * 16));
-                const float4 e0 = *reinterpret_cast<const float4*>(sg + 64 + 8 * cc);
-                const float4 e1 = *reinterpret_cast<const float4*>(sg + 64 + 8 * cc + 4);
-                const float ec[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-                const uint32_t uw[4] = {uv.x, uv.y, uv.z, uv.w};
-                float x[8], y[8];
+            for (int hc = 0; hc < 4; ++hc) {
+              const int cc = 4 * hh + hc;
+              const uint4 uv = *reinterpret_cast<const uint4*>(urow + sw128_offset(j, cc * 16));
+              const float4 e0 = *reinterpret_cast<const float4*>(sg + 64 + 8 * cc);
+              const float4 e1 = *reinterpret_cast<const float4*>(sg + 64 + 8 * cc + 4);
+              const float ec[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+              const uint32_t uw[4] = {uv.x, uv.y, uv.z, uv.w};
+              float x[8], y[8];
 #pragma unroll
-                for (int kq2 = 0; kq2 < 4; ++kq2) {
-                  x[2 * kq2] = vn[8 * hc + 2 * kq2] + __uint_as_float(uw[kq2] << 16);
-                  x[2 * kq2 + 1] = vn[8 * hc + 2 * kq2 + 1] + __uint_as_float(uw[kq2] & 0xFFFF0000u);
-                }
-#pragma unroll
-                for (int m = 0; m < 8; ++m) y[m] = x[m] * ec[m];
-                st_shared_v4(sbase + S_VN + sw128_offset(j, cc * 16), pack_bf16x2(x[0], x[1]),
-                             pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                             pack_bf16x2(x[6], x[7]));
-                st_shared_v4(sbase + S_VNS + sw128_offset(j, cc * 16), pack_bf16x2(y[0], y[1]),
-                             pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                             pack_bf16x2(y[6], y[7]));
+              for (int k2 = 0; k2 < 4; ++k2) {
+                x[2 * k2] = vn[8 * hc + 2 * k2] + __uint_as_float(uw[k2] << 16);
+                x[2 * k2 + 1] = vn[8 * hc + 2 * k2 + 1] + __uint_as_float(uw[k2] & 0xFFFF0000u);
               }
+#pragma unroll
+              for (int m = 0; m < 8; ++m) y[m] = x[m] * ec[m];
+              st_shared_v4(sbase + S_VN + sw128_offset(j, cc * 16), pack_bf16x2(x[0], x[1]),
+                           pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                           pack_bf16x2(x[6], x[7]));
+              st_shared_v4(sbase + S_VNS + sw128_offset(j, cc * 16), pack_bf16x2(y[0], y[1]),
+                           pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                           pack_bf16x2(y[6], y[7]));
             }
           }
           fence_proxy_async_smem();
           tc_fence_before();
-          if (!named_all(1, 128, ok)) {
+          if (!named_all(1, 256, ok)) {
             ok = false;
             break;
           }
@@ -653,13 +655,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p.hT != nullptr && jv) {
           float* hT = p.hT + state_off + j;
 #pragma unroll 1
-          for (int q4 = 0; q4 < 4; ++q4) {
+          for (int q2 = 0; q2 < 2; ++q2) {
             float x[32];
-            tmem_ld32(th + 32u * q4, x);
+            const int k0 = 64 * hh + 32 * q2;
+            tmem_ld32(th + 32u * q2, x);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              if (32 * q4 + i < D) hT[size_t(32 * q4 + i) * D] = x[i];
+              if (k0 + i < D) hT[size_t(k0 + i) * D] = x[i];
           }
         }
         tc_fence_before();
@@ -668,20 +671,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bars[SB_DRAIN]);
         mbar_wait(&bars[SB_DRAIN], 0, nullptr, err, 8u);
       }
-    } else if (warp < 8) {
-      // ---------------- epilogue warps: o_r = e^{G_r} scale O1[r] + O2[r]
-      const int e = tid - 128;
-      const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
-      const bool ev = e < D;
+    } else {
+      // ---------------- epilogue warps 8..11: o_r = e^{G_r} scale O1[r] + O2[r].
+      // Lane 0 of warp 8 also feeds the pipeline: K/Q tiles (TMA) and the ring
+      // entry of chunk c + 2 once the epilogue of chunk c has freed its slot.
+      const int qd = warp & 3;
+      const int e = 32 * qd + lane;
+      const uint32_t lane_off = uint32_t(32 * qd) << 16;
+      const bool ev = e < D;  // warp-uniform (D is a multiple of 32)
+      const bool feeder = warp == 8 && lane == 0;
+      int kq_issued = 0, slot_issued = 0;  // chunks whose K/Q, slot loads were issued
+      ChunkIter fd;
+      it_start(fd, p, s);
+      // Issue the loads of chunk fd.c into stage / slot fd.c & 1.
+      auto feed = [&]() -> bool {
+        const int cc = fd.c, st = cc & 1;
+        if (cc >= 2 &&
+            !mbar_wait(&bars[SB_KQE + st], ((cc >> 1) & 1) ^ 1, abort_flag, err, 1u))
+          return false;
+        uint64_t* fb = &bars[SB_KQF + st];
+        mbar_arrive_expect_tx(fb, uint32_t(nbox) * 2 * 8192);
+        uint8_t* kqp = smem + S_KQ + st * 32768;
+        const int hk = fd.h / vpg;
+        for (int b = 0; b < nbox; ++b) {
+          tma_load_3d(kqp + b * 16384, &tm_k, fb, b * 64, hk, fd.t0);
+          tma_load_3d(kqp + b * 16384 + 8192, &tm_q, fb, b * 64, hk, fd.t0);
+        }
+        kq_issued = cc + 1;
+        if (!poll_geq(ready_flag(p, s, cc % kRing), uint32_t(cc + 1), gabort, err, 1u)) {
+          *abort_flag = 1;
+          return false;
+        }
+        fence_proxy_async_global();
+        uint64_t* sb = &bars[SB_SLOTF + st];
+        mbar_arrive_expect_tx(sb, SLOT_TX);
+        const uint8_t* src = ring_entry(p, s, cc % kRing);
+        bulk_load_g2s(smem + S_SLOT + st * SL_BYTES, src, G_GATE, sb);
+        bulk_load_g2s(smem + S_SGATE + st * G_GATE_BYTES, src + G_GATE, G_GATE_BYTES, sb);
+        slot_issued = cc + 1;
+        it_next(fd, p);
+        return true;
+      };
+      bool fok = true;
+      if (feeder)
+        for (int k2 = 0; k2 < 2 && fd.ok && fok; ++k2) fok = feed();
       ChunkIter it;
-      it_start(it, p, u0, ustep);
+      it_start(it, p, s);
       while (it.ok) {
         const int c = it.c, ob = c & 1;
         const int L = min(C, it.te - it.t0);
-        if (!mbar_wait(&bars[SB_OFULL + ob], (c >> 1) & 1, abort_flag, err, 128u)) break;
+        // All four warps agree on the outcome before any named barrier.
+        if (!named_all(2, 128, mbar_wait(&bars[SB_OFULL + ob], (c >> 1) & 1, abort_flag, err, 128u)))
+          break;
         tc_fence_after();
-        // The gate factors are the last thing read from slot ob: take a copy
-        // and hand the slot back to the TMA warp.
+        // The gate factors are the last thing read from slot ob: take a copy,
+        // then (all four warps done) the feeder refills the slot.
         const float* sg = reinterpret_cast<const float*>(smem + S_SGATE + ob * G_GATE_BYTES);
         float eg[64];
 #pragma unroll
@@ -692,77 +736,152 @@ __global__ void __launch_bounds__(kThreads, 1)
           eg[r + 2] = v4.z * p.scale;
           eg[r + 3] = v4.w * p.scale;
         }
-        mbar_arrive(&bars[SB_SFREE + ob]);
-        uint16_t* orow = p.o + (size_t(it.t0) * p.H_v + it.h) * D + e;
-        const size_t rstride = size_t(p.H_v) * D;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float o1[32], o2[32];
-          tmem_ld32(tmem + lane_off + ST_O1 + 64u * ob + 32u * hf, o1);
-          tmem_ld32(tmem + lane_off + ST_O2 + 64u * ob + 32u * hf, o2);
+        named_sync(2, 128);
+        if (feeder && fok && fd.ok) fok = feed();
+        __syncwarp();
+        // o^T sits in TMEM (lane = d_v index e, column = row r).  Per 16-row
+        // piece: transpose through this warp's 1 KB buffer [16 rows][32 e]
+        // bf16, then write each row's 64-byte segment with 16-byte stores.
+        const uint32_t stg = sbase + S_OSTG + uint32_t(qd) * 2048;
+        const int e0 = qd * 32;
+#pragma unroll 1
+        for (int pc = 0; pc < 4; ++pc) {
+          float o1[16], o2[16];
+          tmem_ld16(tmem + lane_off + ST_O1 + 64u * ob + 16u * pc, o1);
+          tmem_ld16(tmem + lane_off + ST_O2 + 64u * ob + 16u * pc, o2);
           tmem_ld_wait();
-          if (hf == 1) {
+          if (pc == 3) {
             tc_fence_before();
             mbar_arrive(&bars[SB_OFREE + ob]);
           }
-          if (ev) {
+          const uint32_t buf = stg + uint32_t(pc & 1) * 1024;
+          __syncwarp();  // the reads of this buffer two pieces ago are done
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int r = 32 * hf + i;
-              if (r < L)
-                orow[size_t(r) * rstride] =
-                    __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(eg[r], o1[i], o2[i])));
-            }
+          for (int i = 0; i < 16; ++i)
+            st_shared_u16(buf + uint32_t(i) * 64 + uint32_t(lane) * 2,
+                          __bfloat16_as_ushort(
+                              __float2bfloat16_rn(fmaf(eg[16 * pc + i], o1[i], o2[i]))));
+          __syncwarp();
+#pragma unroll
+          for (int m = 0; m < 2; ++m) {
+            const int id = lane + 32 * m, i = id >> 2, seg = id & 3;
+            const int r = 16 * pc + i;
+            const uint4 val = ld_shared_v4(buf + uint32_t(i) * 64 + uint32_t(seg) * 16);
+            if (r < L && ev)
+              *reinterpret_cast<uint4*>(p.o + (size_t(it.t0 + r) * p.H_v + it.h) * D + e0 +
+                                        seg * 8) = val;
           }
         }
-        it_next(it, p, ustep);
+        it_next(it, p);
       }
+      if (feeder) {  // nothing may still be landing in shared memory at exit
+        for (int cc = kq_issued - 2; cc < kq_issued; ++cc)
+          if (cc >= 0) mbar_wait(&bars[SB_KQF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
+        for (int cc = slot_issued - 2; cc < slot_issued; ++cc)
+          if (cc >= 0) mbar_wait(&bars[SB_SLOTF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
+      }
+      __syncwarp();
     }
   } else {
     // =====================================================================
-    // PREP (with P prep CTAs, chunk c goes to prep rank 1 + c % P, and there
-    // to group (c / P) & 1; its results go to ring entry c & 3)
+    // PREP prank = blockIdx.x - S
     // =====================================================================
-    const int par = int(rank) - 1;
+    const int prank = int(blockIdx.x) - p.S;
     if (warp == 8) {
-      // ---------------- TMA: K, Q, V of each item into its group's buffers
-      if (elect_one()) {
-        ChunkIter it;
-        it_start(it, p, u0, ustep);
-        int last_k[2] = {-1, -1};
-        while (it.ok) {
-          const int c = it.c;
-          if (c % P == par) {
-            const int w = (c / P) & 1, k = (c / P) >> 1;
-            if (!mbar_wait(&bars[PB_KQVE + w], (k & 1) ^ 1, abort_flag, err, 1u)) break;
+      // ---------------- loader: K, Q, V tiles (TMA, lane 0) and the gate
+      // factors (whole warp) of each item, for its group
+      PrepIter it;
+      pi_start(it, p, sJ, iend, prank);
+      int last_kw[2] = {-1, -1};
+      bool ok = true;
+      while (it.ok && ok) {
+        const int w = it.k & 1, kw = it.k >> 1, b = kw & 1;
+        if (lane == 0) {
+          ok = mbar_wait(&bars[PB_KQVE + w], (kw & 1) ^ 1, abort_flag, err, 1u);
+          if (ok) {
             uint64_t* fb = &bars[PB_KQVF + w];
             mbar_arrive_expect_tx(fb, uint32_t(nbox) * 3 * 8192);
             uint8_t* gsm = smem + w * P_WG;
-            const int hk = it.h / (p.H_v / p.H_k);
+            const int hk = it.h / vpg;
             for (int b2 = 0; b2 < nbox; ++b2) {
               tma_load_3d(gsm + P_KQ + b2 * 16384, &tm_k, fb, b2 * 64, hk, it.t0);
               tma_load_3d(gsm + P_KQ + b2 * 16384 + 8192, &tm_q, fb, b2 * 64, hk, it.t0);
               tma_load_3d(gsm + P_V + b2 * 8192, &tm_v, fb, b2 * 64, it.h, it.t0);
             }
-            last_k[w] = k;
+            last_kw[w] = kw;
           }
-          it_next(it, p, ustep);
         }
-        for (int w = 0; w < 2; ++w)
-          if (last_k[w] >= 0) mbar_wait(&bars[PB_KQVF + w], last_k[w] & 1, nullptr, err, 32u);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        ok = ok && mbar_wait(&bars[PB_GATEE + 2 * w + b], ((kw >> 1) & 1) ^ 1, abort_flag, err, 1u);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        // Gates of this item (padded rows: g = beta = 0); lane l owns rows 2l, 2l+1.
+        float* gt = reinterpret_cast<float*>(smem + w * P_WG + P_GATE + b * PG_BYTES);
+        {
+          const int r0 = 2 * lane;
+          const float* gsrc = p.g + size_t(it.t0) * p.gb_stride + it.h;
+          const float* bsrc = p.beta + size_t(it.t0) * p.gb_stride + it.h;
+          const float a0 = r0 < it.L ? gsrc[size_t(r0) * p.gb_stride] : 0.f;
+          const float a1 = r0 + 1 < it.L ? gsrc[size_t(r0 + 1) * p.gb_stride] : 0.f;
+          const float b0 = r0 < it.L ? bsrc[size_t(r0) * p.gb_stride] : 0.f;
+          const float b1 = r0 + 1 < it.L ? bsrc[size_t(r0 + 1) * p.gb_stride] : 0.f;
+          float s2 = a0 + a1;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, s2, off);
+            if (lane >= off) s2 += y;
+          }
+          const float G1 = s2, G0 = s2 - a1;       // G_{r0+1}, G_{r0}
+          const float GC = __shfl_sync(0xffffffffu, G1, 31);
+          // G at the start of this pair's 16-row block: row r0 & ~15 is the
+          // first row of lane (r0 & ~15) / 2
+          const float Gb = __shfl_sync(0xffffffffu, G0, (r0 & ~15) >> 1);
+          gt[PG_G + r0] = G0;
+          gt[PG_G + r0 + 1] = G1;
+          gt[PG_BET + r0] = b0;
+          gt[PG_BET + r0 + 1] = b1;
+          const float eg0 = __expf(G0), eg1 = __expf(G1);
+          gt[PG_EG + r0] = eg0;
+          gt[PG_EG + r0 + 1] = eg1;
+          gt[PG_BEG + r0] = b0 * eg0;
+          gt[PG_BEG + r0 + 1] = b1 * eg1;
+          gt[PG_ECG + r0] = __expf(GC - G0);
+          gt[PG_ECG + r0 + 1] = __expf(GC - G1);
+          gt[PG_E1 + r0] = __expf(G0 - Gb);
+          gt[PG_E1 + r0 + 1] = __expf(G1 - Gb);
+          if (lane == 0) gt[PG_DEC] = __expf(GC);
+          __syncwarp();
+          // E2[bb][s2] = e^{G_{16 bb} - G_s2}, s2 < 16 bb
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int e2 = lane + 32 * q, bb = e2 >> 6, sx = e2 & 63;
+            gt[PG_E2 + e2] = (sx < 16 * bb) ? __expf(gt[PG_G + 16 * bb] - gt[PG_G + sx]) : 0.f;
+          }
+        }
+        mbar_arrive(&bars[PB_GATEF + 2 * w + b]);  // release: this lane's gate writes
+        pi_next(it, p, sJ, iend);
       }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicExch(const_cast<uint32_t*>(gabort), 1u);
+      }
+      if (lane == 0)  // nothing may still be landing in shared memory at exit
+        for (int w = 0; w < 2; ++w)
+          if (last_kw[w] >= 0) mbar_wait(&bars[PB_KQVF + w], last_kw[w] & 1, nullptr, err, 32u);
       __syncwarp();
     } else if (warp == 9) {
       // ---------------- MMA issue for both groups, whichever is ready
       if (elect_one()) {
         const uint32_t id_p1 = make_idesc_bf16(128, 64, 0, 0);
         const uint32_t id_wu = make_idesc_bf16(128, 64, 1, 0);
-        ChunkIter itp[2];
+        PrepIter itp[2];
         int kp[2] = {0, 0}, kw[2] = {0, 0};
-        it_start(itp[0], p, u0, ustep);
-        it_align(itp[0], p, ustep, P, par, 0);
-        it_start(itp[1], p, u0, ustep);
-        it_align(itp[1], p, ustep, P, par, 1);
+        for (int w = 0; w < 2; ++w) {
+          pi_start(itp[w], p, sJ, iend, prank);
+          pi_align(itp[w], p, sJ, iend, w);
+        }
         long long last = clock64();
         while (true) {
           bool pending = false, prog = false;
@@ -782,8 +901,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mma_commit(&bars[PB_P1F + w]);
                 ++kp[w];
-                it_next(itp[w], p, ustep);
-                it_align(itp[w], p, ustep, P, par, w);
+                pi_next(itp[w], p, sJ, iend);
+                pi_align(itp[w], p, sJ, iend, w);
                 prog = true;
               }
             }
@@ -810,6 +929,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             if (clock64() - last > kSpinLimitCycles) {
               *abort_flag = 1;
+              atomicExch(const_cast<uint32_t*>(gabort), 1u);
               atomicOr(err, 2u);
               break;
             }
@@ -818,6 +938,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&bars[PB_DRAIN]);
         mbar_wait(&bars[PB_DRAIN], 0, nullptr, err, 8u);
+      }
+      __syncwarp();
+    } else if (warp == 10) {
+      // ---------------- store: each staged item to its spine's ring entry
+      if (lane == 0) {
+        PrepIter it;
+        pi_start(it, p, sJ, iend, prank);
+        bool ok = true;
+        while (it.ok && ok) {
+          const int w = it.k & 1, kw = it.k >> 1, b = kw & 1;
+          const int e = it.j % kRing;
+          ok = mbar_wait(&bars[PB_STAGED + w], kw & 1, abort_flag, err, 4u);
+          if (ok && it.j >= kRing)  // entry e is free once the spine copied item j - kRing
+            ok = poll_geq(free_flag(p, it.s, e), uint32_t(it.j - kRing + 1), gabort, err, 4u);
+          if (!ok) break;
+          fence_proxy_async_global();
+          uint8_t* dst = ring_entry(p, it.s, e);
+          const uint8_t* gs = smem + w * P_WG;
+          bulk_store_s2g(dst + G_W, gs + P_AF, 32768);
+          bulk_store_s2g(dst + G_AQK, gs + P_AQK, 8192);
+          bulk_store_s2g(dst + G_GATE, gs + P_GATE + b * PG_BYTES + PG_EG * 4, G_GATE_BYTES);
+          tma_store_commit();
+          tma_store_wait_read<0>();
+          mbar_arrive(&bars[PB_STGE + w]);
+          mbar_arrive(&bars[PB_GATEE + 2 * w + b]);
+          tma_store_wait_all<0>();
+          fence_proxy_async_global();
+          st_release_gpu(ready_flag(p, it.s, e), uint32_t(it.j + 1));
+          pi_next(it, p, sJ, iend);
+        }
+        if (!ok) {
+          *abort_flag = 1;
+          atomicExch(const_cast<uint32_t*>(gabort), 1u);
+        }
       }
       __syncwarp();
     } else if (warp < 8) {
@@ -830,59 +984,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* Af = reinterpret_cast<float*>(gs + P_AF);
       float* Tf = reinterpret_cast<float*>(gs + P_TF);
       float* Xs = reinterpret_cast<float*>(gs + P_XS);
-      float* gt = reinterpret_cast<float*>(gs + P_GATE);
       const uint32_t tm = tmem + PT_WG * w;
       const int gbar = 1 + 3 * w;  // this group's named barriers: gbar (all), gbar+1, gbar+2
-      ChunkIter it;
-      it_start(it, p, u0, ustep);
-      it_align(it, p, ustep, P, par, w);
-      int k = 0;
+      PrepIter it;
+      pi_start(it, p, sJ, iend, prank);
+      pi_align(it, p, sJ, iend, w);
+      int kw = 0;
       while (it.ok) {
-        const int c = it.c;
-        const int L = min(C, it.te - it.t0);
-        const int h = it.h;
-        // ---- gates of this chunk (padded rows: g = beta = 0)
-        if (pt < 64) {
-          const bool valid = pt < L;
-          gt[PG_G + pt] = valid ? p.g[size_t(it.t0 + pt) * p.gb_stride + h] : 0.f;
-          gt[PG_BET + pt] = valid ? p.beta[size_t(it.t0 + pt) * p.gb_stride + h] : 0.f;
-        }
-        named_sync(gbar, 128);
-        if (pt < 32) {  // inclusive scan of g over 64 rows (2 per lane)
-          const float a0 = gt[PG_G + 2 * pt], a1 = gt[PG_G + 2 * pt + 1];
-          float s2 = a0 + a1;
-#pragma unroll
-          for (int off = 1; off < 32; off <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, s2, off);
-            if (pt >= off) s2 += y;
-          }
-          const float excl = s2 - (a0 + a1);
-          gt[PG_G + 2 * pt] = excl + a0;
-          gt[PG_G + 2 * pt + 1] = excl + a0 + a1;
-        }
-        named_sync(gbar, 128);
-        {
-          const float GC = gt[PG_G + 63];
-          if (pt < 64) {
-            const float Gr = gt[PG_G + pt];
-            const float eg = __expf(Gr);
-            gt[PG_EG + pt] = eg;
-            gt[PG_ECG + pt] = __expf(GC - Gr);
-            gt[PG_BEG + pt] = gt[PG_BET + pt] * eg;
-            gt[PG_E1 + pt] = __expf(Gr - gt[PG_G + (pt & ~15)]);
-          }
-          for (int e = pt; e < 256; e += 128) {  // E2[b][s] = e^{G_{16b} - G_s}, s < 16b
-            const int bb = e >> 6, s2 = e & 63;
-            gt[PG_E2 + e] = (s2 < 16 * bb) ? __expf(gt[PG_G + 16 * bb] - gt[PG_G + s2]) : 0.f;
-          }
-          if (pt == 0) gt[PG_DEC] = __expf(GC);
-        }
-        named_sync(gbar, 128);
+        const int b = kw & 1;
+        const float* gt = reinterpret_cast<const float*>(gs + P_GATE + b * PG_BYTES);
+        // gates written, P1 = [K;Q] K^T done, staging free (previous store read it)
+        const bool ready = mbar_wait(&bars[PB_GATEF + 2 * w + b], (kw >> 1) & 1, abort_flag, err, 4u) &&
+                           mbar_wait(&bars[PB_P1F + w], kw & 1, abort_flag, err, 4u) &&
+                           mbar_wait(&bars[PB_STGE + w], (kw & 1) ^ 1, abort_flag, err, 4u);
+        if (!named_all(gbar, 128, ready)) break;
+        tc_fence_after();
         // ---- P1 row pt: K K^T (pt < 64) or Q K^T (pt >= 64), times e^{G_r - G_s}
         // (s <= r): two factors <= 1 for the blocks of s before r's 16-row
         // block, a direct exponential inside it.
-        if (!named_all(gbar, 128, mbar_wait(&bars[PB_P1F + w], k & 1, abort_flag, err, 4u))) break;
-        tc_fence_after();
         {
           const int r = pt & 63, rb = r >> 4;
           const float Gr = gt[PG_G + r];
@@ -972,9 +1091,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         mbar_arrive(&bars[PB_TREADY + w]);
-        // ---- W^T, U^T rows into the staging (the A / T scratch is free now),
-        // then the whole entry to global ring slot c & 3
-        if (!named_all(gbar, 128, mbar_wait(&bars[PB_WUF + w], k & 1, abort_flag, err, 4u))) break;
+        // ---- W^T, U^T rows into the staging (the A / T scratch is free now)
+        if (!named_all(gbar, 128, mbar_wait(&bars[PB_WUF + w], kw & 1, abort_flag, err, 4u))) break;
         tc_fence_after();
 #pragma unroll 1
         for (int hf = 0; hf < 2; ++hf) {  // W^T row pt (d_k index), U^T row pt (d_v index)
@@ -998,42 +1116,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         fence_proxy_async_smem();
         named_sync(gbar, 128);
-        if (pt == 0) {
-          // ring entry c & 3 is free once the spine has loaded chunk c - 4
-          bool okr = mbar_wait_cluster(&bars[PB_GFREE + (c & 3)], ((c >> 2) & 1) ^ 1, abort_flag,
-                                       err, 4u);
-          if (okr) {
-            uint8_t* dst = ring + (c & 3) * SLOT_G;
-            bulk_store_s2g(dst + G_W, gs + P_AF, 32768);
-            bulk_store_s2g(dst + G_AQK, gs + P_AQK, 8192);
-            bulk_store_s2g(dst + G_GATE, gs + P_GATE + PG_EG * 4, G_GATE_BYTES);
-            tma_store_commit();
-            tma_store_wait_all<0>();
-            fence_proxy_async_global();
-            mbar_arrive_remote(mapa_shared(sbase + S_BARS + (SB_GREADY + (c & 3)) * 8, 0));
-          }
-        }
-        ++k;
-        it_next(it, p, ustep);
-        it_align(it, p, ustep, P, par, w);
+        if (pt == 0) mbar_arrive(&bars[PB_STAGED + w]);
+        ++kw;
+        pi_next(it, p, sJ, iend);
+        pi_align(it, p, sJ, iend, w);
       }
     }
   }
 
-  // ---- teardown: wait for the whole cluster, then release TMEM
+  // ---- teardown: publish an abort to the grid, release TMEM
   tc_fence_before();
   __syncthreads();
-  if (tid == 0) {
-    const int exit_bar = spine ? SB_EXIT : PB_EXIT;
-    mbar_arrive(&bars[exit_bar]);
-    for (uint32_t r = 0; r < ncta; ++r) {
-      if (r == rank) continue;
-      const uint32_t off = (r == 0 ? S_BARS + SB_EXIT * 8 : P_BARS + PB_EXIT * 8);
-      mbar_arrive_remote(mapa_shared(sbase + off, r));
-    }
-    mbar_wait_cluster(&bars[exit_bar], 0, nullptr, err, 256u);
-  }
-  __syncthreads();
+  if (tid == 0 && *abort_flag) atomicExch(const_cast<uint32_t*>(gabort), 1u);
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
@@ -1043,45 +1137,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 namespace {
 
-// Resident clusters of `ncta` CTAs for this kernel on the current device.
-int max_active_clusters(int ncta) {
-  static int cache[64][4] = {{0}};
+// CTAs of this kernel that can be resident at once on the current device.
+int resident_ctas() {
+  static int cache[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
-  int* slot = (dev >= 0 && dev < 64) ? &cache[dev][ncta] : nullptr;
+  int* slot = (dev >= 0 && dev < 64) ? &cache[dev] : nullptr;
   if (slot != nullptr && *slot > 0) return *slot;
-  int m = 0;
+  int per_sm = 0;
   cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        int(kSmemAlloc));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ncta * (sm_count() / ncta));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemAlloc;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = ncta;
-  attr.val.clusterDim.y = 1;
-  attr.val.clusterDim.z = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  if (cudaOccupancyMaxActiveClusters(&m, prefill_kernel, &cfg) != cudaSuccess || m <= 0) {
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prefill_kernel, kThreads,
+                                                    kSmemAlloc) != cudaSuccess) {
     cudaGetLastError();
-    m = sm_count() / ncta;
+    per_sm = 0;
   }
-  if (slot != nullptr) *slot = m;
+  const int m = per_sm * sm_count();
+  if (slot != nullptr && m > 0) *slot = m;
   return m;
 }
 
-// Cluster shape and count for `units` (sequence, v-head) units: three CTAs
-// per unit (two preps) unless that leaves units for a second round of
-// clusters while two-CTA clusters would need fewer rounds.
-void plan(int units, int* ncta, int* clusters) {
-  const int m3 = max_active_clusters(3), m2 = max_active_clusters(2);
-  const int rounds3 = (units + m3 - 1) / m3, rounds2 = (units + m2 - 1) / m2;
-  *ncta = rounds2 < rounds3 ? 2 : 3;
-  const int mc = *ncta == 3 ? m3 : m2;
-  *clusters = units < mc ? units : mc;
+// Grid and spine count for `units` (sequence, v-head) units: one CTA per SM,
+// about a third of them spines (each prep serves two spines' worth of
+// chunks), never more spines than units.
+void plan(int units, int* grid, int* spines) {
+  const int G = resident_ctas();
+  *grid = G;
+  int S = G / 3;
+  if (S > units) S = units;
+  if (S > kMaxSpines) S = kMaxSpines;
+  if (S < 1) S = 1;
+  *spines = S;
 }
+
+size_t flag_bytes(int S) { return (size_t(1 + S * kRing) * kFlagLine + 1023) / 1024 * 1024; }
 
 }  // namespace
 
@@ -1089,9 +1178,9 @@ size_t prefill_workspace_bytes(int total_tokens, int num_seqs, int H_k, int H_v,
   (void)total_tokens;
   (void)H_k;
   (void)D;
-  int ncta = 3, clusters = 0;
-  plan(num_seqs * H_v, &ncta, &clusters);
-  return size_t(clusters) * kRing * SLOT_G;
+  int G = 0, S = 0;
+  plan(num_seqs * H_v, &G, &S);
+  return flag_bytes(S) + size_t(S) * kRing * SLOT_G;
 }
 
 cudaError_t launch_prefill(const uint16_t* q, const uint16_t* k, int qk_stride,
@@ -1113,6 +1202,12 @@ cudaError_t launch_prefill(const uint16_t* q, const uint16_t* k, int qk_stride,
     uint32_t box[3] = {64, 1, 64};
     if (!encode_tmap_bf16(&tv, v, 3, dims, strides, box, true)) return cudaErrorInvalidValue;
   }
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(kSmemAlloc));
+  if (e != cudaSuccess) return e;
+  int G = 0, S = 0;
+  plan(num_seqs * H_v, &G, &S);
+  if (G < 2) return cudaErrorCooperativeLaunchTooLarge;
   Params p;
   p.g = g;
   p.beta = beta;
@@ -1120,29 +1215,27 @@ cudaError_t launch_prefill(const uint16_t* q, const uint16_t* k, int qk_stride,
   p.h0 = h0;
   p.hT = hT;
   p.o = o;
-  p.ws = static_cast<uint8_t*>(workspace);
+  p.flags = static_cast<uint32_t*>(workspace);
+  p.ring = static_cast<uint8_t*>(workspace) + flag_bytes(S);
   p.gb_stride = gb_stride;
   p.num_seqs = num_seqs;
   p.total_tokens = total_tokens;
   p.H_k = H_k;
   p.H_v = H_v;
   p.D = D;
+  p.S = S;
   p.scale = scale;
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(kSmemAlloc));
+  // The hand-off counters start from zero on every launch.
+  e = cudaMemsetAsync(workspace, 0, flag_bytes(S), s);
   if (e != cudaSuccess) return e;
-  int ncta = 3, clusters = 0;
-  plan(num_seqs * H_v, &ncta, &clusters);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(clusters * ncta);
+  cfg.gridDim = dim3(G);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemAlloc;
   cfg.stream = s;
   cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = ncta;
-  attr.val.clusterDim.y = 1;
-  attr.val.clusterDim.z = 1;
+  attr.id = cudaLaunchAttributeCooperative;  // every CTA resident: spines and preps wait on each other
+  attr.val.cooperative = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, prefill_kernel, tq, tk, tv, p);
