@@ -8,9 +8,10 @@
 //
 //   SPINES (the first S CTAs) each own (sequence, v-head) units u = s, s+S, ...
 //     and run their per-chunk critical chain on tcgen05 MMAs with TMEM
-//     accumulators (M = d_v = 128 lanes), keeping H^T in TMEM (f32):
-//       Vn^T = U^T - H^T W^T,   H^T <- e^{G_C} H^T + (e^{G_C - G_r} Vn)^T K,
-//     and the outputs  o_r = e^{G_r} scale (Q H)_r + (Aqk Vn)_r;
+//     accumulators (M = d_v = 128 lanes), keeping H^T in registers (f32):
+//       [Vn' | O1]^T = H^T [W; Q]^T,  Vn = U - Vn',
+//       H^T <- e^{G_C} H^T + (e^{G_C - G_r} Vn)^T K,
+//     and the outputs  o_r = e^{G_r} scale O1_r + (Aqk Vn)_r;
 //   PREPS (all other CTAs) compute everything that does not depend on H, for
 //     chunk items taken from one global order (chunk index major, spine minor;
 //     prep p takes every Pn-th item), two items at a time per CTA:
@@ -19,7 +20,7 @@
 //       Aqk[r][s] = scale e^{G_r-G_s} q_r.k_s, s <= r
 //       T = (I + A)^{-1}                               (blocked, f32, CUDA cores)
 //       W^T = K^T (T diag(beta e^G))^T,  U^T = V^T (T diag(beta))^T   (MMAs)
-//     and bulk-store W^T, U^T, Aqk (bf16) and the gate factors into the
+//     and bulk-store W (row-major), U^T, Aqk (bf16) and the gate factors into the
 //     owning spine's ring of kRing entries in the workspace (it stays in L2).
 //   Hand-offs are release/acquire flags in the workspace: a prep publishes
 //   entry j of spine s after its bulk store completed; the spine publishes that
@@ -60,7 +61,7 @@ constexpr int kAS = 68;        // f32 row stride of the A / T scratch (16-byte r
 constexpr int kRing = 4;       // ring entries per spine
 constexpr int kMaxSpines = 256;
 
-// ---- ring entry (workspace): W^T | U^T | Aqk | gate factors
+// ---- ring entry (workspace): W (rows r, two 64-column d_k boxes) | U^T | Aqk | gate factors
 constexpr uint32_t G_W = 0, G_U = 16384, G_AQK = 32768, G_GATE = 40960;
 constexpr uint32_t G_GATE_BYTES = 528;  // e^{G_r} 64 | e^{G_C-G_r} 64 | e^{G_C} | pad
 constexpr uint32_t SLOT_G = 41984;      // 41 KB, a multiple of 1024
@@ -69,22 +70,27 @@ constexpr uint32_t SLOT_TX = G_GATE + G_GATE_BYTES;
 // line per (spine, ring entry): ready count at +0, free count at +32 bytes.
 constexpr uint32_t kFlagLine = 64;
 
-// ---- spine shared memory (bytes from a 1024-aligned base)
-constexpr uint32_t S_KQ = 0;            // [2 stages][2 boxes][K 64x128B | Q 64x128B]
-constexpr uint32_t S_HT = 65536;        // H^T bf16, [2 boxes][128 x 128B]
-constexpr uint32_t S_VN = 98304;        // Vn^T bf16 [128 x 128B]
-constexpr uint32_t S_VNS = 114688;      // scaled Vn^T bf16
-constexpr uint32_t S_SLOT = 131072;     // 2 slots of {W^T, U^T, Aqk}, same layout as G_*
-constexpr uint32_t SL_BYTES = 40960;
-constexpr uint32_t S_SGATE = S_SLOT + 2 * SL_BYTES;      // 2 x 528 B of gate factors
-constexpr uint32_t S_OSTG = S_SGATE + 2 * G_GATE_BYTES;  // output transpose: 4 warps x 2 x 1 KB
+// ---- spine shared memory (bytes from a 1024-aligned base): two chunk stages
+// of STG_BYTES, each holding everything one chunk step reads:
+//   [box b: W rows 64x128B | Q rows 64x128B] x 2  (the N = 128 B operand [W; Q])
+//   K [box b: 64 x 128B] x 2,  U^T [128 x 128B],  Aqk [64 x 128B],  gate factors
+constexpr uint32_t STG_WQ = 0, STG_K = 32768, STG_U = 49152, STG_AQK = 65536, STG_GATE = 73728;
+constexpr uint32_t STG_BYTES = 74752;  // 73 KB
+constexpr uint32_t S_STG = 0;
+constexpr uint32_t S_HT = S_STG + 2 * STG_BYTES;  // H^T bf16, [2 boxes][128 x 128B]
+constexpr uint32_t S_VN = S_HT + 32768;           // Vn^T bf16 [128 x 128B]
+constexpr uint32_t S_VNS = S_VN + 16384;          // e^{G_C - G_r} Vn^T bf16
+constexpr uint32_t S_EG = S_VNS + 16384;          // 2 x 64 f32: scale e^{G_r} per chunk
+constexpr uint32_t S_OSTG = S_EG + 512;           // output transpose: 8 warps x 1 KB
 constexpr uint32_t S_BARS = S_OSTG + 8192;
+static_assert(S_HT % 1024 == 0 && STG_BYTES % 1024 == 0, "swizzled tiles are 1024-aligned");
+static_assert(STG_GATE + G_GATE_BYTES <= STG_BYTES, "stage layout");
 // ---- prep shared memory: two item groups of P_WG bytes
 constexpr uint32_t P_KQ = 0;        // [2 boxes][K | Q]
 constexpr uint32_t P_V = 32768;     // [2 boxes][64 x 128B]
 constexpr uint32_t P_T1B = 49152;   // T diag(beta e^G) bf16 [64 x 128B]
 constexpr uint32_t P_T2B = 57344;   // T diag(beta) bf16
-constexpr uint32_t P_AF = 65536;    // A f32 [64][kAS]; later the W^T | U^T staging
+constexpr uint32_t P_AF = 65536;    // A f32 [64][kAS]; later the W | U^T staging
 constexpr uint32_t P_TF = P_AF + 64 * kAS * 4;  // T f32 [64][kAS]
 constexpr uint32_t P_XS = P_T1B;    // inverse scratch (32x32 f32), in the T1/T2 tiles' space
 constexpr uint32_t P_GATE = P_TF + 64 * kAS * 4;  // 2 gate blocks of PG_BYTES
@@ -101,36 +107,34 @@ constexpr uint32_t kSmemBytes =
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 static_assert(S_BARS % 8 == 0 && P_BARS % 8 == 0, "barrier alignment");
-static_assert(P_AF + 32768 <= P_GATE, "W^T | U^T staging fits in the A / T scratch");
+static_assert(P_AF + 32768 <= P_GATE, "W | U^T staging fits in the A / T scratch");
 static_assert((P_GATE + PG_EG * 4) % 16 == 0 && (P_GATE + PG_BYTES + PG_EG * 4) % 16 == 0,
               "gate blocks are bulk-copy sources");
 
 // ---- barriers (spine)
 enum {
-  SB_KQF = 0,      // +stage: K/Q tiles landed (TMA)
-  SB_KQE = 2,      // +stage: K/Q tiles free (MMA commit)
-  SB_SLOTF = 4,    // +slot: slot data landed (bulk loads)
-  SB_VNFULL = 6,   // -H^T W^T done (commit)
-  SB_DHFULL = 7,   // H += dH done (commit)
-  SB_OFULL = 8,    // +buf: O1, O2 done (commit)
-  SB_OFREE = 10,   // +buf: O1, O2 read back (128)
-  SB_DRAIN = 12,
-  SB_COUNT = 13
+  SB_STGF = 0,     // +stage: every tile of the chunk landed (TMA + bulk loads)
+  SB_STGE = 2,     // +stage: the chunk's MMAs are done, the stage is free (commit)
+  SB_VOFULL = 4,   // H^T [W; Q]^T done (commit)
+  SB_DHFULL = 5,   // dH = Vns^T K done (commit)
+  SB_OFULL = 6,    // +buf: O2 (and so O1) done (commit)
+  SB_DRAIN = 8,
+  SB_COUNT = 9
 };
 // ---- barriers (prep); per group w: base + w (GATEF / GATEE: base + 2w + b)
 enum {
   PB_KQVF = 0, PB_KQVE = 2, PB_P1F = 4, PB_P1FREE = 6, PB_TREADY = 8, PB_WUF = 10,
   PB_GATEF = 12,   // gate block (w, b) written (32, the loader warp)
   PB_GATEE = 16,   // gate block (w, b) free again (1, the store warp)
-  PB_STAGED = 20,  // +w: W^T | U^T, Aqk staged (1)
+  PB_STAGED = 20,  // +w: W | U^T, Aqk staged (1)
   PB_STGE = 22,    // +w: staging read by the bulk store (1)
   PB_DRAIN = 24,
   PB_COUNT = 25
 };
 
 // ---- TMEM columns
-// spine: Vn, O1 x2, O2 x2, and the state H^T itself (f32, lane j = row j)
-constexpr uint32_t ST_VN = 0, ST_O1 = 64, ST_O2 = 192, ST_H = 320;
+// spine: [H^T W^T | O1^T] x2 (128 columns each), O2^T x2, dH^T (lane j = row j of H^T)
+constexpr uint32_t ST_VO = 0, ST_O2 = 256, ST_DH = 384;
 constexpr uint32_t PT_P1 = 0, PT_W = 64, PT_U = 128, PT_WG = 192;  // prep, per group
 
 struct Params {
@@ -465,8 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (tid == 0) {
     if (spine) {
-      for (int b = 0; b < SB_COUNT; ++b)
-        mbar_init(&bars[b], (b == SB_OFREE || b == SB_OFREE + 1) ? 128u : 1u);
+      for (int b = 0; b < SB_COUNT; ++b) mbar_init(&bars[b], 1u);
     } else {
       for (int b = 0; b < PB_COUNT; ++b) {
         uint32_t cnt = 1;
@@ -506,20 +509,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int s = int(blockIdx.x);
     if (warp < 8) {
       // ---------------- state warps: warp w serves TMEM lane quadrant w & 3
-      // (row j of H^T) and half w >> 2 of the columns: d_k 64 hh .. 64 hh + 63
-      // of H^T, chunk rows 32 hh .. 32 hh + 31 of Vn^T.  Per chunk: read H^T,
-      // write its bf16 copy (the A operand of Vn and O1), write back
-      // e^{G_C} H^T so that the dH MMA accumulates H_{c+1} = e^{G_C} H_c + dH
-      // in place.  Thread 0 also issues the chunk's MMAs.
+      // (row j of H^T) and half hh = w >> 2: columns d_k 64 hh .. 64 hh + 63 of
+      // H^T (kept in registers, f32) and chunk rows 32 hh .. 32 hh + 31 of Vn^T
+      // and of the outputs.  Per chunk c:
+      //   H <- e^{G_C} H + dH (dH of chunk c-1, from TMEM); bf16 copy -> S_HT;
+      //   [Vn' | O1]^T = H^T [W; Q]^T  (one N = 128 MMA);
+      //   outputs of chunk c-1 while it runs;
+      //   Vn = U - Vn' -> Vn^T, e^{G_C - G_r} Vn^T (bf16);
+      //   dH = Vns^T K,  O2^T = Vn^T Aqk^T.
+      // Thread 0 issues the MMAs right after the named barriers.
       const int qd = warp & 3, hh = warp >> 2;
       const int j = 32 * qd + lane;
       const bool issuer = tid == 0;
       const uint32_t lane_off = uint32_t(32 * qd) << 16;
-      const uint32_t th = tmem + lane_off + ST_H + 64u * uint32_t(hh);
       const bool jv = j < D;
-      const uint32_t id_vn = make_idesc_bf16(128, 64, 0, 1, /*b_neg=*/1);
-      const uint32_t id_o = make_idesc_bf16(128, 64, 0, 0);
+      const uint32_t id_vo = make_idesc_bf16(128, 128, 0, 0);
       const uint32_t id_dh = make_idesc_bf16(128, 128, 0, 1);
+      const uint32_t id_o2 = make_idesc_bf16(128, 64, 0, 0);
+      const uint32_t ostg = sbase + S_OSTG + uint32_t(warp) * 1024;
+      float* eg_s = reinterpret_cast<float*>(smem + S_EG);
+      // Outputs of chunk cl (rows 32 hh .. + 31 of this warp, d_v lanes of its
+      // quadrant): o_r = scale e^{G_r} O1[r] + O2[r], transposed through this
+      // warp's 1 KB buffer and written as 64-byte row segments.
+      auto epilogue = [&](int cl, int t0l, int Ll, int hl) -> bool {
+        const int ob = cl & 1;
+        const bool okE = mbar_wait(&bars[SB_OFULL + ob], (cl >> 1) & 1, abort_flag, err, 128u);
+        tc_fence_after();
+        const float* egp = eg_s + 64 * ob;
+        const int e0 = 32 * qd;
+#pragma unroll 1
+        for (int pc = 0; pc < 2; ++pc) {
+          const int r0 = 32 * hh + 16 * pc;
+          float o1[16], o2[16];
+          tmem_ld16(tmem + lane_off + ST_VO + 128u * ob + 64u + uint32_t(r0), o1);
+          tmem_ld16(tmem + lane_off + ST_O2 + 64u * ob + uint32_t(r0), o2);
+          tmem_ld_wait();
+          __syncwarp();  // the previous piece's reads of the buffer are done
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            st_shared_u16(ostg + uint32_t(i) * 64 + uint32_t(lane) * 2,
+                          __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(egp[r0 + i], o1[i], o2[i]))));
+          __syncwarp();
+#pragma unroll
+          for (int m = 0; m < 2; ++m) {
+            const int id = lane + 32 * m, i = id >> 2, seg = id & 3;
+            const int r = r0 + i;
+            const uint4 val = ld_shared_v4(ostg + uint32_t(i) * 64 + uint32_t(seg) * 16);
+            if (okE && r < Ll && e0 < D)
+              *reinterpret_cast<uint4*>(p.o + (size_t(t0l + r) * p.H_v + hl) * D + e0 + seg * 8) = val;
+          }
+        }
+        return okE;
+      };
       int c = 0;
       bool ok = true;
       for (int u = s; u < units && ok; u += p.S) {
@@ -527,79 +568,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         int tb, te;
         seq_range(p, n, tb, te);
         const size_t state_off = (size_t(n) * p.H_v + h) * size_t(D) * D;
-        const float* h0 = (p.h0 != nullptr && jv) ? p.h0 + state_off + j : nullptr;
-#pragma unroll 1
-        for (int q2 = 0; q2 < 2; ++q2) {  // H^T row j, this warp's 64 columns <- h0 (or zeros)
-          float x[32];
-          const int k0 = 64 * hh + 32 * q2;
+        float H[64];
+        {
+          const float* h0 = (p.h0 != nullptr && jv) ? p.h0 + state_off + j : nullptr;
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            x[i] = (h0 != nullptr && k0 + i < D) ? h0[size_t(k0 + i) * D] : 0.f;
-          tmem_st32(th + 32u * q2, x);
+          for (int i = 0; i < 64; ++i)
+            H[i] = (h0 != nullptr && 64 * hh + i < D) ? h0[size_t(64 * hh + i) * D] : 0.f;
         }
-        tmem_st_wait();
+        const int c_first = c;
+        float dec_prev = 1.f;
+        int prev_t0 = tb, prev_L = 0;
         for (int t0 = tb; t0 < te && ok; t0 += C, ++c) {
           const int st = c & 1;
-          const uint32_t kq = sbase + S_KQ + st * 32768;
-          const uint32_t slot = sbase + S_SLOT + st * SL_BYTES;
-          if (t0 > tb) {  // H = e^{G_C} H_{c-1} + dH landed
+          const uint32_t stg = sbase + S_STG + uint32_t(st) * STG_BYTES;
+          const float* sg = reinterpret_cast<const float*>(smem + S_STG + st * STG_BYTES + STG_GATE);
+          if (c > c_first) {  // dH of the previous chunk landed
             ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u);
             tc_fence_after();
           }
-          ok = ok && mbar_wait(&bars[SB_SLOTF + st], (c >> 1) & 1, abort_flag, err, 16u);
-          if (issuer && ok) {
-            st_release_gpu(free_flag(p, s, c % kRing), uint32_t(c + 1));  // ring entry copied out
-            ok = mbar_wait(&bars[SB_KQF + st], (c >> 1) & 1, abort_flag, err, 2u);
-          }
-          const float* sg = reinterpret_cast<const float*>(smem + S_SGATE + st * G_GATE_BYTES);
-          const float dec = sg[128];
-          {
-            float x[64];
-            tmem_ld32(th, *reinterpret_cast<float(*)[32]>(x));
-            tmem_ld32(th + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-            tmem_ld_wait();
-            st_row64_bf16(sbase + S_HT + uint32_t(hh) * 16384, uint32_t(j), x);
+          ok = ok && mbar_wait(&bars[SB_STGF + st], (c >> 1) & 1, abort_flag, err, 16u);
+          if (c > c_first) {  // H <- e^{G_C} H + dH
 #pragma unroll
-            for (int i = 0; i < 64; ++i) x[i] *= dec;
-            tmem_st32(th, *reinterpret_cast<float(*)[32]>(x));
-            tmem_st32(th + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+            for (int q2 = 0; q2 < 2; ++q2) {
+              float d[32];
+              tmem_ld32(tmem + lane_off + ST_DH + 64u * uint32_t(hh) + 32u * uint32_t(q2), d);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) H[32 * q2 + i] = fmaf(dec_prev, H[32 * q2 + i], d[i]);
+            }
           }
-          tmem_st_wait();
+          const float dec_cur = sg[128];
+          if (tid < 64) eg_s[64 * st + tid] = sg[tid] * p.scale;
+          st_row64_bf16(sbase + S_HT + uint32_t(hh) * 16384, uint32_t(j), H);
           fence_proxy_async_smem();
           tc_fence_before();
           if (!named_all(1, 256, ok)) {
             ok = false;
             break;
           }
-          if (issuer) {
+          if (issuer) {  // [Vn' | O1]^T = H^T [W; Q]^T
             tc_fence_after();
-            // Vn^T := -H^T W^T   (U^T is added below)
             for (int kk = 0; kk < ksteps_d; ++kk) {
-              const uint32_t a = sbase + S_HT + (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_bf16_ss(tmem + ST_VN, make_sdesc_sw128(a, 16, 1024),
-                          make_sdesc_sw128(slot + G_W + kk * 2048, 8192, 1024), id_vn, kk > 0);
+              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+              mma_bf16_ss(tmem + ST_VO + 128u * st, make_sdesc_sw128(sbase + S_HT + off, 16, 1024),
+                          make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_vo, kk > 0);
             }
-            mma_commit(&bars[SB_VNFULL]);
-            // O1^T = H^T Q^T into buffer st (free once the epilogue read chunk c-2)
-            ok = c < 2 || mbar_wait(&bars[SB_OFREE + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 2u);
-            if (ok) {
-              tc_fence_after();
-              for (int kk = 0; kk < ksteps_d; ++kk) {
-                const uint32_t a = sbase + S_HT + (kk >> 2) * 16384 + (kk & 3) * 32;
-                const uint32_t b = kq + (kk >> 2) * 16384 + 8192 + (kk & 3) * 32;
-                mma_bf16_ss(tmem + ST_O1 + 64u * st, make_sdesc_sw128(a, 16, 1024),
-                            make_sdesc_sw128(b, 16, 1024), id_o, kk > 0);
-              }
-            }
+            mma_commit(&bars[SB_VOFULL]);
           }
-          // Vn = U - (H W)  ->  Vn^T and e^{G_C - G_r} Vn^T rows in bf16 (this
-          // warp: chunk rows 32 hh .. 32 hh + 31)
-          ok = ok && mbar_wait(&bars[SB_VNFULL], c & 1, abort_flag, err, 16u);
+          if (c > c_first) ok = epilogue(c - 1, prev_t0, prev_L, h) && ok;
+          // Vn = U - Vn'  ->  Vn^T and e^{G_C - G_r} Vn^T rows in bf16
+          ok = mbar_wait(&bars[SB_VOFULL], c & 1, abort_flag, err, 16u) && ok;
           tc_fence_after();
-          if (ok) {
-            const uint8_t* urow = smem + S_SLOT + st * SL_BYTES + G_U;
+          {
+            const uint8_t* urow = smem + S_STG + st * STG_BYTES + STG_U;
             float vn[32];
-            tmem_ld32(tmem + lane_off + ST_VN + 32u * uint32_t(hh), vn);
+            tmem_ld32(tmem + lane_off + ST_VO + 128u * st + 32u * uint32_t(hh), vn);
             tmem_ld_wait();
 #pragma unroll
             for (int hc = 0; hc < 4; ++hc) {
@@ -612,8 +635,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               float x[8], y[8];
 #pragma unroll
               for (int k2 = 0; k2 < 4; ++k2) {
-                x[2 * k2] = vn[8 * hc + 2 * k2] + __uint_as_float(uw[k2] << 16);
-                x[2 * k2 + 1] = vn[8 * hc + 2 * k2 + 1] + __uint_as_float(uw[k2] & 0xFFFF0000u);
+                x[2 * k2] = __uint_as_float(uw[k2] << 16) - vn[8 * hc + 2 * k2];
+                x[2 * k2 + 1] = __uint_as_float(uw[k2] & 0xFFFF0000u) - vn[8 * hc + 2 * k2 + 1];
               }
 #pragma unroll
               for (int m = 0; m < 8; ++m) y[m] = x[m] * ec[m];
@@ -633,37 +656,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (issuer) {
             tc_fence_after();
-            // H^T (already scaled by e^{G_C} in TMEM) += Vns^T K ; O2^T = Vn^T Aqk^T
+            // dH^T = Vns^T K (fresh), then O2^T = Vn^T Aqk^T
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(tmem + ST_H, make_sdesc_sw128(sbase + S_VNS + kk * 32, 16, 1024),
-                          make_sdesc_sw128(kq + kk * 2048, 16384, 1024), id_dh, 1);
+              mma_bf16_ss(tmem + ST_DH, make_sdesc_sw128(sbase + S_VNS + kk * 32, 16, 1024),
+                          make_sdesc_sw128(stg + STG_K + kk * 2048, 8192, 1024), id_dh, kk > 0);
             mma_commit(&bars[SB_DHFULL]);
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(tmem + ST_O2 + 64u * st,
-                          make_sdesc_sw128(sbase + S_VN + kk * 32, 16, 1024),
-                          make_sdesc_sw128(slot + G_AQK + kk * 32, 16, 1024), id_o, kk > 0);
+              mma_bf16_ss(tmem + ST_O2 + 64u * st, make_sdesc_sw128(sbase + S_VN + kk * 32, 16, 1024),
+                          make_sdesc_sw128(stg + STG_AQK + kk * 32, 16, 1024), id_o2, kk > 0);
             mma_commit(&bars[SB_OFULL + st]);
-            mma_commit(&bars[SB_KQE + st]);
+            mma_commit(&bars[SB_STGE + st]);
           }
+          dec_prev = dec_cur;
+          prev_t0 = t0;
+          prev_L = min(C, te - t0);
         }
         if (!ok) break;
-        if (te > tb) {  // the last chunk's update
+        if (te > tb) {  // the last chunk: its update and its outputs
           ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u);
-          if (!ok) break;
           tc_fence_after();
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) {
+            float d[32];
+            tmem_ld32(tmem + lane_off + ST_DH + 64u * uint32_t(hh) + 32u * uint32_t(q2), d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) H[32 * q2 + i] = fmaf(dec_prev, H[32 * q2 + i], d[i]);
+          }
+          ok = epilogue(c - 1, prev_t0, prev_L, h) && ok;
+          if (!named_all(1, 256, ok)) {
+            ok = false;
+            break;
+          }
         }
         if (p.hT != nullptr && jv) {
           float* hT = p.hT + state_off + j;
-#pragma unroll 1
-          for (int q2 = 0; q2 < 2; ++q2) {
-            float x[32];
-            const int k0 = 64 * hh + 32 * q2;
-            tmem_ld32(th + 32u * q2, x);
-            tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (k0 + i < D) hT[size_t(k0 + i) * D] = x[i];
-          }
+          for (int i = 0; i < 64; ++i)
+            if (64 * hh + i < D) hT[size_t(64 * hh + i) * D] = H[i];
         }
         tc_fence_before();
       }
@@ -671,114 +701,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bars[SB_DRAIN]);
         mbar_wait(&bars[SB_DRAIN], 0, nullptr, err, 8u);
       }
-    } else {
-      // ---------------- epilogue warps 8..11: o_r = e^{G_r} scale O1[r] + O2[r].
-      // Lane 0 of warp 8 also feeds the pipeline: K/Q tiles (TMA) and the ring
-      // entry of chunk c + 2 once the epilogue of chunk c has freed its slot.
-      const int qd = warp & 3;
-      const int e = 32 * qd + lane;
-      const uint32_t lane_off = uint32_t(32 * qd) << 16;
-      const bool ev = e < D;  // warp-uniform (D is a multiple of 32)
-      const bool feeder = warp == 8 && lane == 0;
-      int kq_issued = 0, slot_issued = 0;  // chunks whose K/Q, slot loads were issued
-      ChunkIter fd;
-      it_start(fd, p, s);
-      // Issue the loads of chunk fd.c into stage / slot fd.c & 1.
-      auto feed = [&]() -> bool {
-        const int cc = fd.c, st = cc & 1;
-        if (cc >= 2 &&
-            !mbar_wait(&bars[SB_KQE + st], ((cc >> 1) & 1) ^ 1, abort_flag, err, 1u))
-          return false;
-        uint64_t* fb = &bars[SB_KQF + st];
-        mbar_arrive_expect_tx(fb, uint32_t(nbox) * 2 * 8192);
-        uint8_t* kqp = smem + S_KQ + st * 32768;
-        const int hk = fd.h / vpg;
-        for (int b = 0; b < nbox; ++b) {
-          tma_load_3d(kqp + b * 16384, &tm_k, fb, b * 64, hk, fd.t0);
-          tma_load_3d(kqp + b * 16384 + 8192, &tm_q, fb, b * 64, hk, fd.t0);
+    } else if (warp == 8) {
+      // ---------------- feeder: the tiles of chunk c into stage c & 1 once the
+      // chunk c - 2 MMAs released it: K and Q by TMA, then (when a prep has
+      // published it) the ring entry: W next to Q, U^T, Aqk and the gates.
+      // It also hands chunk c - 2's ring entry back to the preps.
+      if (lane == 0) {
+        ChunkIter fd;
+        it_start(fd, p, s);
+        int issued = 0;
+        bool ok = true;
+        while (fd.ok && ok) {
+          const int cc = fd.c, st = cc & 1;
+          if (cc >= 2) {
+            ok = mbar_wait(&bars[SB_STGE + st], ((cc >> 1) & 1) ^ 1, abort_flag, err, 1u);
+            if (!ok) break;
+            // chunk cc - 2 is fully consumed: its ring entry may be reused
+            st_release_gpu(free_flag(p, s, (cc - 2) % kRing), uint32_t(cc - 1));
+          }
+          uint8_t* stg = smem + S_STG + st * STG_BYTES;
+          uint64_t* fb = &bars[SB_STGF + st];
+          // The phase completes on the one arrival (made with the ring bytes, or
+          // bare on an abort) plus every byte announced before it.
+          mbar_expect_tx(fb, uint32_t(nbox) * 2 * 8192);
+          const int hk = fd.h / vpg;
+          for (int b = 0; b < nbox; ++b) {
+            tma_load_3d(stg + STG_K + b * 8192, &tm_k, fb, b * 64, hk, fd.t0);
+            tma_load_3d(stg + STG_WQ + b * 16384 + 8192, &tm_q, fb, b * 64, hk, fd.t0);
+          }
+          issued = cc + 1;
+          ok = poll_geq(ready_flag(p, s, cc % kRing), uint32_t(cc + 1), gabort, err, 1u);
+          if (!ok) {  // the phase still completes once the K/Q tiles landed
+            mbar_arrive(fb);
+            break;
+          }
+          fence_proxy_async_global();
+          mbar_arrive_expect_tx(fb, 2 * 8192 + 16384 + 8192 + G_GATE_BYTES);
+          const uint8_t* src = ring_entry(p, s, cc % kRing);
+          bulk_load_g2s(stg + STG_WQ, src + G_W, 8192, fb);
+          bulk_load_g2s(stg + STG_WQ + 16384, src + G_W + 8192, 8192, fb);
+          bulk_load_g2s(stg + STG_U, src + G_U, 16384, fb);
+          bulk_load_g2s(stg + STG_AQK, src + G_AQK, 8192, fb);
+          bulk_load_g2s(stg + STG_GATE, src + G_GATE, G_GATE_BYTES, fb);
+          it_next(fd, p);
         }
-        kq_issued = cc + 1;
-        if (!poll_geq(ready_flag(p, s, cc % kRing), uint32_t(cc + 1), gabort, err, 1u)) {
+        if (!ok) {
           *abort_flag = 1;
-          return false;
+          atomicExch(const_cast<uint32_t*>(gabort), 1u);
         }
-        fence_proxy_async_global();
-        uint64_t* sb = &bars[SB_SLOTF + st];
-        mbar_arrive_expect_tx(sb, SLOT_TX);
-        const uint8_t* src = ring_entry(p, s, cc % kRing);
-        bulk_load_g2s(smem + S_SLOT + st * SL_BYTES, src, G_GATE, sb);
-        bulk_load_g2s(smem + S_SGATE + st * G_GATE_BYTES, src + G_GATE, G_GATE_BYTES, sb);
-        slot_issued = cc + 1;
-        it_next(fd, p);
-        return true;
-      };
-      bool fok = true;
-      if (feeder)
-        for (int k2 = 0; k2 < 2 && fd.ok && fok; ++k2) fok = feed();
-      ChunkIter it;
-      it_start(it, p, s);
-      while (it.ok) {
-        const int c = it.c, ob = c & 1;
-        const int L = min(C, it.te - it.t0);
-        // All four warps agree on the outcome before any named barrier.
-        if (!named_all(2, 128, mbar_wait(&bars[SB_OFULL + ob], (c >> 1) & 1, abort_flag, err, 128u)))
-          break;
-        tc_fence_after();
-        // The gate factors are the last thing read from slot ob: take a copy,
-        // then (all four warps done) the feeder refills the slot.
-        const float* sg = reinterpret_cast<const float*>(smem + S_SGATE + ob * G_GATE_BYTES);
-        float eg[64];
-#pragma unroll
-        for (int r = 0; r < 64; r += 4) {
-          const float4 v4 = *reinterpret_cast<const float4*>(sg + r);
-          eg[r] = v4.x * p.scale;
-          eg[r + 1] = v4.y * p.scale;
-          eg[r + 2] = v4.z * p.scale;
-          eg[r + 3] = v4.w * p.scale;
-        }
-        named_sync(2, 128);
-        if (feeder && fok && fd.ok) fok = feed();
-        __syncwarp();
-        // o^T sits in TMEM (lane = d_v index e, column = row r).  Per 16-row
-        // piece: transpose through this warp's 1 KB buffer [16 rows][32 e]
-        // bf16, then write each row's 64-byte segment with 16-byte stores.
-        const uint32_t stg = sbase + S_OSTG + uint32_t(qd) * 2048;
-        const int e0 = qd * 32;
-#pragma unroll 1
-        for (int pc = 0; pc < 4; ++pc) {
-          float o1[16], o2[16];
-          tmem_ld16(tmem + lane_off + ST_O1 + 64u * ob + 16u * pc, o1);
-          tmem_ld16(tmem + lane_off + ST_O2 + 64u * ob + 16u * pc, o2);
-          tmem_ld_wait();
-          if (pc == 3) {
-            tc_fence_before();
-            mbar_arrive(&bars[SB_OFREE + ob]);
-          }
-          const uint32_t buf = stg + uint32_t(pc & 1) * 1024;
-          __syncwarp();  // the reads of this buffer two pieces ago are done
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            st_shared_u16(buf + uint32_t(i) * 64 + uint32_t(lane) * 2,
-                          __bfloat16_as_ushort(
-                              __float2bfloat16_rn(fmaf(eg[16 * pc + i], o1[i], o2[i]))));
-          __syncwarp();
-#pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            const int id = lane + 32 * m, i = id >> 2, seg = id & 3;
-            const int r = 16 * pc + i;
-            const uint4 val = ld_shared_v4(buf + uint32_t(i) * 64 + uint32_t(seg) * 16);
-            if (r < L && ev)
-              *reinterpret_cast<uint4*>(p.o + (size_t(it.t0 + r) * p.H_v + it.h) * D + e0 +
-                                        seg * 8) = val;
-          }
-        }
-        it_next(it, p);
-      }
-      if (feeder) {  // nothing may still be landing in shared memory at exit
-        for (int cc = kq_issued - 2; cc < kq_issued; ++cc)
-          if (cc >= 0) mbar_wait(&bars[SB_KQF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
-        for (int cc = slot_issued - 2; cc < slot_issued; ++cc)
-          if (cc >= 0) mbar_wait(&bars[SB_SLOTF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
+        // nothing may still be landing in shared memory at exit
+        for (int cc = issued - 2; cc < issued; ++cc)
+          if (cc >= 0) mbar_wait(&bars[SB_STGF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
       }
       __syncwarp();
     }
@@ -1091,26 +1064,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         mbar_arrive(&bars[PB_TREADY + w]);
-        // ---- W^T, U^T rows into the staging (the A / T scratch is free now)
+        // ---- W, U^T into the staging (the A / T scratch is free now)
         if (!named_all(gbar, 128, mbar_wait(&bars[PB_WUF + w], kw & 1, abort_flag, err, 4u))) break;
         tc_fence_after();
+        // U^T row pt (d_v index) as a 128-byte swizzled row; W column pt (d_k
+        // index) into the row-major W tile [box pt / 64][row r][d_k % 64].
+        {
+          const uint32_t wcol = g + P_AF + G_W + uint32_t(pt >> 6) * 8192;
+          const uint32_t wbyte = uint32_t(pt & 63) * 2;
 #pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {  // W^T row pt (d_k index), U^T row pt (d_v index)
-          float wv[32], uv[32];
-          tmem_ld32(tm + lane_off + PT_W + 32u * hf, wv);
-          tmem_ld32(tm + lane_off + PT_U + 32u * hf, uv);
-          tmem_ld_wait();
+          for (int hf = 0; hf < 2; ++hf) {
+            float wv[32], uv[32];
+            tmem_ld32(tm + lane_off + PT_W + 32u * hf, wv);
+            tmem_ld32(tm + lane_off + PT_U + 32u * hf, uv);
+            tmem_ld_wait();
 #pragma unroll
-          for (int hc = 0; hc < 4; ++hc) {
-            const uint32_t off = sw128_offset(pt, (4 * hf + hc) * 16);
-            st_shared_v4(g + P_AF + G_W + off, pack_bf16x2(wv[8 * hc], wv[8 * hc + 1]),
-                         pack_bf16x2(wv[8 * hc + 2], wv[8 * hc + 3]),
-                         pack_bf16x2(wv[8 * hc + 4], wv[8 * hc + 5]),
-                         pack_bf16x2(wv[8 * hc + 6], wv[8 * hc + 7]));
-            st_shared_v4(g + P_AF + G_U + off, pack_bf16x2(uv[8 * hc], uv[8 * hc + 1]),
-                         pack_bf16x2(uv[8 * hc + 2], uv[8 * hc + 3]),
-                         pack_bf16x2(uv[8 * hc + 4], uv[8 * hc + 5]),
-                         pack_bf16x2(uv[8 * hc + 6], uv[8 * hc + 7]));
+            for (int hc = 0; hc < 4; ++hc) {
+              const uint32_t off = sw128_offset(pt, (4 * hf + hc) * 16);
+              st_shared_v4(g + P_AF + G_U + off, pack_bf16x2(uv[8 * hc], uv[8 * hc + 1]),
+                           pack_bf16x2(uv[8 * hc + 2], uv[8 * hc + 3]),
+                           pack_bf16x2(uv[8 * hc + 4], uv[8 * hc + 5]),
+                           pack_bf16x2(uv[8 * hc + 6], uv[8 * hc + 7]));
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              st_shared_u16(wcol + sw128_offset(uint32_t(32 * hf + i), wbyte),
+                            __bfloat16_as_ushort(__float2bfloat16_rn(wv[i])));
           }
         }
         tc_fence_before();
