@@ -6,14 +6,20 @@
 // kernels (the gb10 parent and the Hopper twin) do this on CUDA cores and read
 // the row 96x resp. 12x; here it is a bf16 GEMM with f32 accumulation:
 //
-//   D[128 tokens x N] = X[128 x K] * W[N x K]^T     (one CTA per 128 tokens)
+//   D[128 tokens x N] = X[128 x K] * W[N x K]^T
 //
+// One cluster of KS CTAs per 128 tokens, each CTA over its own K / KS slice
+// (split-K, so that the 4576 x 5120 activation streams through ~all SMs).
 // TMA streams 128x64 X tiles and Nx64 W tiles (128-byte swizzle) through a
 // STAGES-deep mbarrier ring; one thread issues tcgen05.mma (M=128, N=N_pad,
-// K=16 steps) into a TMEM accumulator; four warps then read their 32 TMEM
-// lanes (one token each) and apply the gate epilogue in f32:
+// K=16 steps) into a TMEM accumulator.  Each CTA then stages its f32 partial
+// in its own (now idle) pipeline shared memory; after a cluster barrier, rank
+// r reduces rows r*128/KS .. of all KS partials in rank order (distributed
+// shared memory reads, deterministic) and applies the gate epilogue in f32:
 //   beta = sigmoid(ba),  gate = -exp(A_log) * softplus(ba + dt_bias).
+// A second cluster barrier keeps every partial alive until it has been read.
 // Every activation byte is read from HBM once; W (N*K*2 bytes) stays in L2.
+// No multicast: each CTA loads its own tiles.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -35,7 +41,24 @@ struct BaParams {
   float* out;
   int gate_stride, M, N, K, nv, vpg;
   int n_pad, stages, tmem_cols;
+  int ks;  // CTAs per cluster (K split)
 };
+
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// Hardware cluster barrier; every thread of every CTA of the cluster reaches
+// each call exactly once (no early exits in this kernel).
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
 
 __global__ void __launch_bounds__(kBaThreads, 1)
     ba_gates_kernel(const __grid_constant__ CUtensorMap tmap_x,
@@ -56,8 +79,11 @@ __global__ void __launch_bounds__(kBaThreads, 1)
 
   const uint32_t warp = warp_id_sync();
   const uint32_t lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kBaBM;
-  const int num_kb = (p.K + kBaBK - 1) / kBaBK;
+  const int rank = int(cluster_ctarank());
+  const int m0 = int(cluster_id_x()) * kBaBM;
+  const int kb_all = (p.K + kBaBK - 1) / kBaBK;
+  const int kb_begin = kb_all * rank / p.ks, kb_end = kb_all * (rank + 1) / p.ks;
+  const int num_kb = kb_end - kb_begin;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -82,8 +108,8 @@ __global__ void __launch_bounds__(kBaThreads, 1)
         const uint32_t ph = (kb / stages) & 1;
         if (!mbar_wait(&empty_bar[s], ph ^ 1, abort_flag, &g_err_ba_gates, 1u)) break;
         mbar_arrive_expect_tx(&full_bar[s], a_bytes + b_bytes);
-        tma_load_2d(a_s + s * a_bytes, &tmap_x, &full_bar[s], kb * kBaBK, m0);
-        tma_load_2d(b_s + s * b_bytes, &tmap_w, &full_bar[s], kb * kBaBK, 0);
+        tma_load_2d(a_s + s * a_bytes, &tmap_x, &full_bar[s], (kb_begin + kb) * kBaBK, m0);
+        tma_load_2d(b_s + s * b_bytes, &tmap_w, &full_bar[s], (kb_begin + kb) * kBaBK, 0);
       }
     }
     __syncwarp();
@@ -111,20 +137,51 @@ __global__ void __launch_bounds__(kBaThreads, 1)
     __syncwarp();
   }
 
-  // Epilogue: warp w owns TMEM lanes 32w..32w+31, i.e. tokens m0+32w+lane.
-  const bool ok = mbar_wait(done_bar, 0, abort_flag, &g_err_ba_gates, 4u);
+  // Partial sums: warp w owns TMEM lanes 32w..32w+31 (tokens m0+32w+lane);
+  // each row goes to the partial buffer P[128][n_pad + 4] f32 that reuses the
+  // pipeline's shared memory (every MMA has completed once done_bar fired).
+  const bool ok = num_kb == 0 || mbar_wait(done_bar, 0, abort_flag, &g_err_ba_gates, 4u);
   tc_fence_after();
-  const int m = m0 + int(warp * 32 + lane);
-  if (ok && !*abort_flag) {
-    const int group_dim = 2 * p.vpg;
-    float* row = p.out + size_t(m) * p.gate_stride;
+  const int pstride = p.n_pad + 4;
+  float* part = reinterpret_cast<float*>(smem);
+  {
+    float* prow = part + size_t(warp * 32 + lane) * pstride;
     for (int c = 0; c < p.n_pad; c += 16) {
       float acc[16];
       tmem_ld16(tmem + ((warp * 32u) << 16) + uint32_t(c), acc);
       tmem_ld_wait();
-      if (m < p.M) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<float4*>(prow + c + j) =
+            (ok && num_kb > 0) ? make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3])
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  tc_fence_before();
+  cluster_barrier();  // every partial of the cluster is written
+  // Reduction + epilogue: this CTA's rows r0 .. r0 + rows - 1; thread t takes
+  // row r0 + t / tpr and a run of 4-column groups.
+  {
+    const int rows = kBaBM / p.ks;
+    const int tpr = kBaThreads / rows;  // threads per row
+    const int r = rank * rows + int(threadIdx.x) / tpr;
+    const int m = m0 + r;
+    const int group_dim = 2 * p.vpg;
+    const uint32_t prow = smem_u32(part + size_t(r) * pstride);
+    float* row = p.out + size_t(m) * p.gate_stride;
+    for (int c = 4 * (int(threadIdx.x) % tpr); c < p.n_pad; c += 4 * tpr) {
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < p.ks; ++q) {  // fixed order: deterministic
+        const float4 v = ld_cluster_f4(mapa_shared(prow + uint32_t(c) * 4, uint32_t(q)));
+        sum.x += v.x;
+        sum.y += v.y;
+        sum.z += v.z;
+        sum.w += v.w;
+      }
+      const float acc[4] = {sum.x, sum.y, sum.z, sum.w};
+      if (m < p.M && ok && !*abort_flag) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
           const int n = c + j;
           if (n < p.N) {
             const int within = n % group_dim, grp = n / group_dim;
@@ -143,6 +200,7 @@ __global__ void __launch_bounds__(kBaThreads, 1)
       }
     }
   }
+  cluster_barrier();  // no CTA leaves while its partial may still be read
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, p.tmem_cols);
@@ -175,6 +233,9 @@ cudaError_t launch_ba_gates(const uint16_t* x, int k_stride, const uint16_t* w,
   p.stages = (200 * 1024) / stage_bytes;
   if (p.stages > 6) p.stages = 6;
   if (p.stages < 2) p.stages = 2;
+  // The pipeline buffers double as the f32 partial [128][n_pad + 4] afterwards.
+  const size_t part_bytes = size_t(kBaBM) * (p.n_pad + 4) * 4;
+  if (size_t(p.stages) * stage_bytes < part_bytes) return cudaErrorInvalidValue;
   const size_t smem = 1024 + size_t(p.stages) * stage_bytes + (2 * p.stages + 1) * 8 + 16;
 
   CUtensorMap tx, tw;
@@ -193,8 +254,27 @@ cudaError_t launch_ba_gates(const uint16_t* x, int k_stride, const uint16_t* w,
   cudaError_t e =
       cudaFuncSetAttribute(ba_gates_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid((M + kBaBM - 1) / kBaBM);
-  ba_gates_kernel<<<grid, kBaThreads, smem, s>>>(tx, tw, p);
+  // K split: the largest power of two <= 8 that keeps the grid within the SMs
+  // and leaves every CTA at least one K block (KS = 4 for 4576 tokens).
+  const int mtiles = (M + kBaBM - 1) / kBaBM;
+  const int kb_all = (K + kBaBK - 1) / kBaBK;
+  int ks = 1;
+  while (ks < 8 && mtiles * ks * 2 <= sm_count() && ks * 2 <= kb_all) ks *= 2;
+  p.ks = ks;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(mtiles * ks);
+  cfg.blockDim = dim3(kBaThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = ks;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, ba_gates_kernel, tx, tw, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

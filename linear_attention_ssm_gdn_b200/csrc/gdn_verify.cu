@@ -11,8 +11,9 @@
 //                          - sum_{s<r} e^{G_r - G_s} kk[s][r] delta_s[j])
 //   o_r[j] = scale (e^{G_r} b_r[j] + sum_{s<=r} e^{G_r - G_s} kq[s][r] delta_s[j])
 // which is the token recurrence unrolled over four rows.  H0 is read once
-// (16-byte loads, 4 columns per thread, 4 row groups per CTA); nothing is
-// written to it.  delta_r and G_r go to the stash for the fold.
+// (16-byte loads, 4 columns per thread, 8 row groups per CTA, every load of a
+// thread in flight at once); nothing is written to it.  delta_r and G_r go to
+// the stash for the fold.
 //
 // Fold.  With na = na_tab[b] in 1..4 (and the engaged bit set):
 //   H[i][j] <- e^{G_{na-1}} H[i][j] + sum_{r<na} e^{G_{na-1} - G_r} k_r[i] delta_r[j]
@@ -48,18 +49,21 @@ __global__ void flag_clear_kernel(uint32_t* flag) {
   if (threadIdx.x == 0) *flag = 0u;
 }
 
-// grid = (H_v, batch); block = 128 = 4 row groups x 32 column quads (d_v = 128)
-// or 4 row groups x 16 column quads with 16 idle lanes... (d_v = 64: see below)
+constexpr int kVThreads = 256;
+
+// grid = (H_v, batch); block = 256 threads = GROUPS row groups x QUADS column
+// quads.  Every thread issues all of its state loads (16 x 16 bytes at
+// d = 128) before it needs any of them, so a CTA waits for memory about once.
 template <int D>
-__global__ void __launch_bounds__(128) verify_kernel(
+__global__ void __launch_bounds__(kVThreads) verify_kernel(
     float* const* __restrict__ h_table, const uint16_t* __restrict__ q,
     const uint16_t* __restrict__ k, int qk_stride, const uint16_t* __restrict__ v, int v_stride,
     const float* __restrict__ g, const float* __restrict__ beta, int gb_stride,
     uint16_t* __restrict__ o, float* __restrict__ stash, int stash_seq_floats, int H_k, int H_v,
     float scale, uint32_t* flag) {
-  constexpr int QUADS = D / 4;             // column quads per row
-  constexpr int GROUPS = 128 / QUADS;      // row groups (4 for D=128, 8 for D=64)
-  constexpr int ROWS_PER_GROUP = D / GROUPS;
+  constexpr int QUADS = D / 4;              // column quads per row
+  constexpr int GROUPS = kVThreads / QUADS;  // row groups (8 for D=128, 16 for D=64)
+  constexpr int RPG = D / GROUPS;            // rows per group (16 resp. 4)
   __shared__ float ks[kRows][D], qs[kRows][D];
   __shared__ float4 part[GROUPS][2 * kRows][QUADS];  // partial a_r, b_r per row group
   __shared__ float kk[kRows][kRows], kq[kRows][kRows], G[kRows], bt[kRows];
@@ -73,13 +77,23 @@ __global__ void __launch_bounds__(128) verify_kernel(
 
   const size_t row0 = size_t(b) * kRows;
   if (H0 == nullptr) {  // padding sequence: zero outputs, nothing else
-    for (int idx = tid; idx < kRows * D; idx += 128) {
+    for (int idx = tid; idx < kRows * D; idx += kVThreads) {
       const int r = idx / D, j = idx % D;
       o[((row0 + r) * H_v + h) * D + j] = 0;
     }
     return;
   }
-  for (int idx = tid; idx < kRows * D; idx += 128) {
+  // This thread's rows of the state, all loads in flight at once.
+  const float4* H4 = reinterpret_cast<const float4*>(H0 + size_t(h) * D * D);
+  float4 hv[RPG];
+#pragma unroll
+  for (int ii = 0; ii < RPG; ++ii) hv[ii] = __ldg(&H4[(grp * RPG + ii) * QUADS + quad]);
+  // v for the recurrence (thread j < D owns column j)
+  float vr[kRows];
+#pragma unroll
+  for (int r = 0; r < kRows; ++r)
+    vr[r] = tid < D ? bf16_at(v + (row0 + r) * v_stride + size_t(h) * D + tid) : 0.f;
+  for (int idx = tid; idx < kRows * D; idx += kVThreads) {
     const int r = idx / D, i = idx % D;
     ks[r][i] = bf16_at(k + (row0 + r) * qk_stride + size_t(hk) * D + i);
     qs[r][i] = bf16_at(q + (row0 + r) * qk_stride + size_t(hk) * D + i);
@@ -96,8 +110,9 @@ __global__ void __launch_bounds__(128) verify_kernel(
       G[r] = run;
     }
   }
-  if (tid < 2 * kRows * kRows) {  // 16 k.k and 16 k.q dot products
-    const int which = tid / (kRows * kRows), s = (tid / kRows) % kRows, r = tid % kRows;
+  if (tid >= 64 && tid < 64 + 2 * kRows * kRows) {  // 16 k.k and 16 k.q dot products
+    const int t = tid - 64;
+    const int which = t / (kRows * kRows), s = (t / kRows) % kRows, r = t % kRows;
     float acc = 0.f;
     const float* other = which == 0 ? ks[r] : qs[r];
     for (int i = 0; i < D; ++i) acc = fmaf(ks[s][i], other[i], acc);
@@ -110,33 +125,33 @@ __global__ void __launch_bounds__(128) verify_kernel(
   float4 acc[2 * kRows];
 #pragma unroll
   for (int r = 0; r < 2 * kRows; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float4* H4 = reinterpret_cast<const float4*>(H0 + size_t(h) * D * D);
-#pragma unroll 4
-  for (int ii = 0; ii < ROWS_PER_GROUP; ++ii) {
-    const int i = grp * ROWS_PER_GROUP + ii;
-    const float4 hv = __ldg(&H4[i * QUADS + quad]);
+#pragma unroll
+  for (int ii = 0; ii < RPG; ++ii) {
+    const int i = grp * RPG + ii;
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
       const float kv = ks[r][i], qv = qs[r][i];
-      acc[r].x = fmaf(hv.x, kv, acc[r].x);
-      acc[r].y = fmaf(hv.y, kv, acc[r].y);
-      acc[r].z = fmaf(hv.z, kv, acc[r].z);
-      acc[r].w = fmaf(hv.w, kv, acc[r].w);
-      acc[kRows + r].x = fmaf(hv.x, qv, acc[kRows + r].x);
-      acc[kRows + r].y = fmaf(hv.y, qv, acc[kRows + r].y);
-      acc[kRows + r].z = fmaf(hv.z, qv, acc[kRows + r].z);
-      acc[kRows + r].w = fmaf(hv.w, qv, acc[kRows + r].w);
+      acc[r].x = fmaf(hv[ii].x, kv, acc[r].x);
+      acc[r].y = fmaf(hv[ii].y, kv, acc[r].y);
+      acc[r].z = fmaf(hv[ii].z, kv, acc[r].z);
+      acc[r].w = fmaf(hv[ii].w, kv, acc[r].w);
+      acc[kRows + r].x = fmaf(hv[ii].x, qv, acc[kRows + r].x);
+      acc[kRows + r].y = fmaf(hv[ii].y, qv, acc[kRows + r].y);
+      acc[kRows + r].z = fmaf(hv[ii].z, qv, acc[kRows + r].z);
+      acc[kRows + r].w = fmaf(hv[ii].w, qv, acc[kRows + r].w);
     }
   }
 #pragma unroll
   for (int r = 0; r < 2 * kRows; ++r) part[grp][r][quad] = acc[r];
   __syncthreads();
   // One thread per column: reduce the row groups, run the 4-step recurrence.
-  for (int j = tid; j < D; j += 128) {
+  if (tid < D) {
+    const int j = tid;
     float a[kRows], bq[kRows], delta[kRows];
 #pragma unroll
     for (int r = 0; r < 2 * kRows; ++r) {
       float s = 0.f;
+#pragma unroll
       for (int gg = 0; gg < GROUPS; ++gg) {
         const float* pp = reinterpret_cast<const float*>(&part[gg][r][j / 4]);
         s += pp[j % 4];
@@ -148,14 +163,12 @@ __global__ void __launch_bounds__(128) verify_kernel(
     }
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
-      const float vr = bf16_at(v + (row0 + r) * v_stride + size_t(h) * D + j);
       float pred = __expf(G[r]) * a[r];
       for (int s2 = 0; s2 < r; ++s2) pred += __expf(G[r] - G[s2]) * kk[s2][r] * delta[s2];
-      delta[r] = bt[r] * (vr - pred);
+      delta[r] = bt[r] * (vr[r] - pred);
       float out = __expf(G[r]) * bq[r];
       for (int s2 = 0; s2 <= r; ++s2) out += __expf(G[r] - G[s2]) * kq[s2][r] * delta[s2];
-      o[((row0 + r) * H_v + h) * D + j] =
-          __bfloat16_as_ushort(__float2bfloat16_rn(scale * out));
+      o[((row0 + r) * H_v + h) * D + j] = __bfloat16_as_ushort(__float2bfloat16_rn(scale * out));
       stash[size_t(b) * stash_seq_floats + size_t(h) * kRows * (D + 4) + r * D + j] = delta[r];
     }
   }
@@ -163,15 +176,17 @@ __global__ void __launch_bounds__(128) verify_kernel(
     stash[size_t(b) * stash_seq_floats + size_t(h) * kRows * (D + 4) + kRows * D + tid] = G[tid];
 }
 
-// grid = (H_v, batch); block = 128.
+// grid = (H_v, batch); block = 256.  Each thread loads all of its 16-byte
+// state quads (16 at d = 128) before updating and storing them.
 template <int D>
-__global__ void __launch_bounds__(128) fold_kernel(float* const* __restrict__ h_table,
-                                                   const float* __restrict__ stash,
-                                                   const int32_t* __restrict__ na_tab,
-                                                   const uint16_t* __restrict__ k, int qk_stride,
-                                                   uint32_t* flag, int H_k, int H_v,
-                                                   int stash_seq_floats) {
+__global__ void __launch_bounds__(kVThreads) fold_kernel(float* const* __restrict__ h_table,
+                                                         const float* __restrict__ stash,
+                                                         const int32_t* __restrict__ na_tab,
+                                                         const uint16_t* __restrict__ k,
+                                                         int qk_stride, uint32_t* flag, int H_k,
+                                                         int H_v, int stash_seq_floats) {
   constexpr int QUADS = D / 4;
+  constexpr int PER = D * QUADS / kVThreads;  // quads per thread (16 resp. 4)
   __shared__ float ks[kRows][D], dl[kRows][D], coef[kRows], cdecay;
   const int h = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x;
@@ -183,9 +198,13 @@ __global__ void __launch_bounds__(128) fold_kernel(float* const* __restrict__ h_
     if (h == 0 && tid == 0) atomicOr(flag, kFlagError);
     return;
   }
+  float4* H4 = reinterpret_cast<float4*>(H + size_t(h) * D * D);
+  float4 hv[PER];
+#pragma unroll
+  for (int m = 0; m < PER; ++m) hv[m] = H4[tid + kVThreads * m];
   const int hk = h / (H_v / H_k);
   const float* st = stash + size_t(b) * stash_seq_floats + size_t(h) * kRows * (D + 4);
-  for (int idx = tid; idx < kRows * D; idx += 128) {
+  for (int idx = tid; idx < kRows * D; idx += kVThreads) {
     const int r = idx / D, i = idx % D;
     ks[r][i] = bf16_at(k + (size_t(b) * kRows + r) * qk_stride + size_t(hk) * D + i);
     dl[r][i] = st[r * D + i];
@@ -196,22 +215,23 @@ __global__ void __launch_bounds__(128) fold_kernel(float* const* __restrict__ h_
     cdecay = __expf(Gl);
   }
   __syncthreads();
-  float4* H4 = reinterpret_cast<float4*>(H + size_t(h) * D * D);
-  for (int idx = tid; idx < D * QUADS; idx += 128) {
+#pragma unroll
+  for (int m = 0; m < PER; ++m) {
+    const int idx = tid + kVThreads * m;
     const int i = idx / QUADS, j4 = idx % QUADS;
-    float4 hv = H4[idx];
-    hv.x *= cdecay;
-    hv.y *= cdecay;
-    hv.z *= cdecay;
-    hv.w *= cdecay;
+    float4 x = hv[m];
+    x.x *= cdecay;
+    x.y *= cdecay;
+    x.z *= cdecay;
+    x.w *= cdecay;
     for (int r = 0; r < na; ++r) {
       const float c = coef[r] * ks[r][i];
-      hv.x = fmaf(c, dl[r][4 * j4 + 0], hv.x);
-      hv.y = fmaf(c, dl[r][4 * j4 + 1], hv.y);
-      hv.z = fmaf(c, dl[r][4 * j4 + 2], hv.z);
-      hv.w = fmaf(c, dl[r][4 * j4 + 3], hv.w);
+      x.x = fmaf(c, dl[r][4 * j4 + 0], x.x);
+      x.y = fmaf(c, dl[r][4 * j4 + 1], x.y);
+      x.z = fmaf(c, dl[r][4 * j4 + 2], x.z);
+      x.w = fmaf(c, dl[r][4 * j4 + 3], x.w);
     }
-    H4[idx] = hv;
+    H4[idx] = x;
   }
 }
 
@@ -228,11 +248,11 @@ cudaError_t launch_verify(float* const* h_table, const uint16_t* q, const uint16
   if (batch == 0) return cudaSuccess;
   dim3 grid(H_v, batch);
   if (D == 128)
-    verify_kernel<128><<<grid, 128, 0, s>>>(h_table, q, k, qk_stride, v, v_stride, g, beta,
+    verify_kernel<128><<<grid, kVThreads, 0, s>>>(h_table, q, k, qk_stride, v, v_stride, g, beta,
                                             gb_stride, o, stash, stash_seq_floats, H_k, H_v,
                                             scale, flag);
   else
-    verify_kernel<64><<<grid, 128, 0, s>>>(h_table, q, k, qk_stride, v, v_stride, g, beta,
+    verify_kernel<64><<<grid, kVThreads, 0, s>>>(h_table, q, k, qk_stride, v, v_stride, g, beta,
                                            gb_stride, o, stash, stash_seq_floats, H_k, H_v,
                                            scale, flag);
   return cudaGetLastError();
@@ -245,10 +265,10 @@ cudaError_t launch_fold(float* const* h_table, const float* stash, const int32_t
   if (batch == 0) return cudaSuccess;
   dim3 grid(H_v, batch);
   if (D == 128)
-    fold_kernel<128><<<grid, 128, 0, s>>>(h_table, stash, na_tab, k, qk_stride, flag, H_k, H_v,
+    fold_kernel<128><<<grid, kVThreads, 0, s>>>(h_table, stash, na_tab, k, qk_stride, flag, H_k, H_v,
                                           stash_seq_floats);
   else
-    fold_kernel<64><<<grid, 128, 0, s>>>(h_table, stash, na_tab, k, qk_stride, flag, H_k, H_v,
+    fold_kernel<64><<<grid, kVThreads, 0, s>>>(h_table, stash, na_tab, k, qk_stride, flag, H_k, H_v,
                                          stash_seq_floats);
   return cudaGetLastError();
 }
