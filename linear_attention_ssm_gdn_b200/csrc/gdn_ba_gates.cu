@@ -32,7 +32,9 @@ namespace gdn {
 __device__ uint32_t g_err_ba_gates;
 
 constexpr int kBaBM = 128;       // tokens per CTA (MMA M)
-constexpr int kBaBK = 64;        // K per pipeline stage (one 128-byte swizzle row)
+constexpr int kBaBK = 64;        // K per TMA box (one 128-byte swizzle row)
+constexpr int kBaNB = 2;         // boxes per pipeline stage: 2 x 128 contiguous bytes per row
+constexpr int kBaMaxKS = 2;      // largest K split (CTAs per cluster): measured best
 constexpr int kBaThreads = 128;  // 4 warps: TMA (warp 0), MMA (warp 1), all: epilogue
 
 struct BaParams {
@@ -67,8 +69,9 @@ __global__ void __launch_bounds__(kBaThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int stages = p.stages;
-  const uint32_t a_bytes = kBaBM * 128;
-  const uint32_t b_bytes = uint32_t(p.n_pad) * 128;
+  const uint32_t a_box = kBaBM * 128, b_box = uint32_t(p.n_pad) * 128;
+  const uint32_t a_bytes = kBaNB * a_box;
+  const uint32_t b_bytes = kBaNB * b_box;
   uint8_t* a_s = smem;
   uint8_t* b_s = a_s + stages * a_bytes;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(b_s + stages * b_bytes);
@@ -81,9 +84,12 @@ __global__ void __launch_bounds__(kBaThreads, 1)
   const uint32_t lane = threadIdx.x & 31;
   const int rank = int(cluster_ctarank());
   const int m0 = int(cluster_id_x()) * kBaBM;
+  // K is split into boxes of kBaBK; this CTA owns boxes [kb_begin, kb_end),
+  // consumed kBaNB boxes per pipeline stage (the last stage may be partial).
   const int kb_all = (p.K + kBaBK - 1) / kBaBK;
   const int kb_begin = kb_all * rank / p.ks, kb_end = kb_all * (rank + 1) / p.ks;
-  const int num_kb = kb_end - kb_begin;
+  const int nbox = kb_end - kb_begin;
+  const int num_kb = (nbox + kBaNB - 1) / kBaNB;  // pipeline stages
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -107,9 +113,13 @@ __global__ void __launch_bounds__(kBaThreads, 1)
         const int s = kb % stages;
         const uint32_t ph = (kb / stages) & 1;
         if (!mbar_wait(&empty_bar[s], ph ^ 1, abort_flag, &g_err_ba_gates, 1u)) break;
-        mbar_arrive_expect_tx(&full_bar[s], a_bytes + b_bytes);
-        tma_load_2d(a_s + s * a_bytes, &tmap_x, &full_bar[s], (kb_begin + kb) * kBaBK, m0);
-        tma_load_2d(b_s + s * b_bytes, &tmap_w, &full_bar[s], (kb_begin + kb) * kBaBK, 0);
+        const int nb = min(kBaNB, nbox - kb * kBaNB);
+        mbar_arrive_expect_tx(&full_bar[s], uint32_t(nb) * (a_box + b_box));
+        for (int x = 0; x < nb; ++x) {
+          const int kx = (kb_begin + kb * kBaNB + x) * kBaBK;
+          tma_load_2d(a_s + s * a_bytes + x * a_box, &tmap_x, &full_bar[s], kx, m0);
+          tma_load_2d(b_s + s * b_bytes + x * b_box, &tmap_w, &full_bar[s], kx, 0);
+        }
       }
     }
     __syncwarp();
@@ -123,12 +133,15 @@ __global__ void __launch_bounds__(kBaThreads, 1)
         ok = mbar_wait(&full_bar[s], ph, abort_flag, &g_err_ba_gates, 2u);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(a_s + s * a_bytes);
-        const uint32_t b0 = smem_u32(b_s + s * b_bytes);
+        const int nb = min(kBaNB, nbox - kb * kBaNB);
+        for (int x = 0; x < nb; ++x) {
+          const uint32_t a0 = smem_u32(a_s + s * a_bytes + x * a_box);
+          const uint32_t b0 = smem_u32(b_s + s * b_bytes + x * b_box);
 #pragma unroll
-        for (int j = 0; j < kBaBK / 16; ++j) {
-          mma_bf16_ss(tmem, make_sdesc_sw128(a0 + j * 32, 16, 1024),
-                      make_sdesc_sw128(b0 + j * 32, 16, 1024), idesc, (kb | j) != 0);
+          for (int j = 0; j < kBaBK / 16; ++j) {
+            mma_bf16_ss(tmem, make_sdesc_sw128(a0 + j * 32, 16, 1024),
+                        make_sdesc_sw128(b0 + j * 32, 16, 1024), idesc, (kb | x | j) != 0);
+          }
         }
         mma_commit(&empty_bar[s]);
       }
@@ -229,7 +242,7 @@ cudaError_t launch_ba_gates(const uint16_t* x, int k_stride, const uint16_t* w,
   p.vpg = vpg;
   p.n_pad = (N + 15) / 16 * 16;
   p.tmem_cols = pow2_at_least(p.n_pad);
-  const int stage_bytes = kBaBM * 128 + p.n_pad * 128;
+  const int stage_bytes = kBaNB * (kBaBM * 128 + p.n_pad * 128);
   p.stages = (200 * 1024) / stage_bytes;
   if (p.stages > 6) p.stages = 6;
   if (p.stages < 2) p.stages = 2;
@@ -254,12 +267,12 @@ cudaError_t launch_ba_gates(const uint16_t* x, int k_stride, const uint16_t* w,
   cudaError_t e =
       cudaFuncSetAttribute(ba_gates_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  // K split: the largest power of two <= 8 that keeps the grid within the SMs
-  // and leaves every CTA at least one K block (KS = 4 for 4576 tokens).
+  // K split: the largest power of two <= kBaMaxKS that keeps the grid within
+  // the SMs and leaves every CTA at least one K box (KS = 2 for 4576 tokens).
   const int mtiles = (M + kBaBM - 1) / kBaBM;
   const int kb_all = (K + kBaBK - 1) / kBaBK;
   int ks = 1;
-  while (ks < 8 && mtiles * ks * 2 <= sm_count() && ks * 2 <= kb_all) ks *= 2;
+  while (ks < kBaMaxKS && mtiles * ks * 2 <= sm_count() && ks * 2 <= kb_all) ks *= 2;
   p.ks = ks;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(mtiles * ks);
