@@ -53,9 +53,11 @@ constexpr int kVThreads = 256;
 
 // grid = (H_v, batch); block = 256 threads = GROUPS row groups x QUADS column
 // quads.  Every thread issues all of its state loads (16 x 16 bytes at
-// d = 128) before it needs any of them, so a CTA waits for memory about once.
+// d = 128) before it needs any of them, so a CTA waits for memory about once;
+// four CTAs per SM (64 registers) keep the loads of one CTA overlapping the
+// recurrence of another (measured: 55.6 us against 75.4 us at two per SM).
 template <int D>
-__global__ void __launch_bounds__(kVThreads) verify_kernel(
+__global__ void __launch_bounds__(kVThreads, 4) verify_kernel(
     float* const* __restrict__ h_table, const uint16_t* __restrict__ q,
     const uint16_t* __restrict__ k, int qk_stride, const uint16_t* __restrict__ v, int v_stride,
     const float* __restrict__ g, const float* __restrict__ beta, int gb_stride,
