@@ -143,6 +143,21 @@ class ClockSampler:
 # Our arm
 # --------------------------------------------------------------------------
 
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's time (every rank calls this; identity for one rank)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, steps: int, tokens_per_step: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank runs `steps` steps of `tokens_per_step`."""
+    return world * steps * tokens_per_step / (max_ms / 1e3)
+
+
 def make_inputs(dev):
     import torch
 
@@ -236,10 +251,7 @@ def run_ours(args, rank, world, dist):
     total_ms = t_start.elapsed_time(t_end)
     per = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
            for j, name in enumerate(["ba_gates", "prefill", "flag_clear", "verify", "fold"])}
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
 
     # ---- end to end through the public API: H2D inputs, the calls, D2H results
     pinned = {k: v.pin_memory() for k, v in host.items()}
@@ -262,17 +274,15 @@ def run_ours(args, rank, world, dist):
     e_e.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e_s.elapsed_time(e_e)
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
 
     if rank != 0:
         return None
     T = meta["T"]
-    value = world * K * T / (total_ms / 1e3)
-    e2e_value = world * K * T / (e2e_ms / 1e3)
+    value = job_value(world, K, T, total_ms)
+    e2e_value = job_value(world, K, T, e2e_ms)
     hbm, tf_burst, tf_sust, src = peaks()
     B = prefill_alg_bytes(T, meta["N"], meta["H_k"], meta["H_v"], meta["d_k"], meta["d_v"])
     F = prefill_alg_flops(T, meta["H_v"], meta["d_k"], meta["d_v"])
