@@ -60,6 +60,7 @@ constexpr int kThreads = 384;  // 12 warps
 constexpr int kAS = 68;        // f32 row stride of the A / T scratch (16-byte rows)
 constexpr int kRing = 4;       // ring entries per spine
 constexpr int kMaxSpines = 256;
+constexpr int kSpineSync = 288;  // the spine's per-chunk barriers: 8 state warps + the issuer warp
 
 // ---- ring entry (workspace): W (rows r, two 64-column d_k boxes) | U^T | Aqk | gate factors
 constexpr uint32_t G_W = 0, G_U = 16384, G_AQK = 32768, G_GATE = 40960;
@@ -516,29 +517,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       //   [Vn' | O1]^T = H^T [W; Q]^T  (one N = 128 MMA);
       //   outputs of chunk c-1 while it runs;
       //   Vn = U - Vn' -> Vn^T, e^{G_C - G_r} Vn^T (bf16);
-      //   dH = Vns^T K,  O2^T = Vn^T Aqk^T.
-      // Thread 0 issues the MMAs right after the named barriers.
+      //   dH = Vns^T K,  O2^T = Vn^T Aqk^T;
+      // warp 9 issues the MMAs right after the two named barriers, and chunk
+      // c-1's outputs are written in two halves, one under each of them.
       const int qd = warp & 3, hh = warp >> 2;
       const int j = 32 * qd + lane;
-      const bool issuer = tid == 0;
       const uint32_t lane_off = uint32_t(32 * qd) << 16;
       const bool jv = j < D;
-      const uint32_t id_vo = make_idesc_bf16(128, 128, 0, 0);
-      const uint32_t id_dh = make_idesc_bf16(128, 128, 0, 1);
-      const uint32_t id_o2 = make_idesc_bf16(128, 64, 0, 0);
       const uint32_t ostg = sbase + S_OSTG + uint32_t(warp) * 1024;
       float* eg_s = reinterpret_cast<float*>(smem + S_EG);
-      // Outputs of chunk cl (rows 32 hh .. + 31 of this warp, d_v lanes of its
-      // quadrant): o_r = scale e^{G_r} O1[r] + O2[r], transposed through this
-      // warp's 1 KB buffer and written as 64-byte row segments.
-      auto epilogue = [&](int cl, int t0l, int Ll, int hl) -> bool {
+      // Outputs of chunk cl, 16 of this warp's rows 32 hh .. + 31 per call
+      // (piece pc), for the d_v lanes of its quadrant: o_r = scale e^{G_r}
+      // O1[r] + O2[r], transposed through this warp's 1 KB buffer and written
+      // as 64-byte row segments.  Piece 0 waits for the chunk's MMAs.
+      auto epilogue = [&](int cl, int pc, int t0l, int Ll, int hl) -> bool {
         const int ob = cl & 1;
-        const bool okE = mbar_wait(&bars[SB_OFULL + ob], (cl >> 1) & 1, abort_flag, err, 128u);
+        bool okE = true;
+        if (pc == 0) okE = mbar_wait(&bars[SB_OFULL + ob], (cl >> 1) & 1, abort_flag, err, 128u);
         tc_fence_after();
         const float* egp = eg_s + 64 * ob;
         const int e0 = 32 * qd;
-#pragma unroll 1
-        for (int pc = 0; pc < 2; ++pc) {
+        {
           const int r0 = 32 * hh + 16 * pc;
           float o1[16], o2[16];
           tmem_ld16(tmem + lane_off + ST_VO + 128u * ob + 64u + uint32_t(r0), o1);
@@ -561,13 +560,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return okE;
       };
+      // Every exit from these loops follows a bar.red agreement that the
+      // issuer warp takes part in, so the two sides always leave together.
       int c = 0;
       bool ok = true;
-      for (int u = s; u < units && ok; u += p.S) {
+      for (int u = s; u < units; u += p.S) {
         const int n = u / p.H_v, h = u % p.H_v;
         int tb, te;
         seq_range(p, n, tb, te);
         const size_t state_off = (size_t(n) * p.H_v + h) * size_t(D) * D;
+        bool agreed = true;
         float H[64];
         {
           const float* h0 = (p.h0 != nullptr && jv) ? p.h0 + state_off + j : nullptr;
@@ -578,12 +580,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c_first = c;
         float dec_prev = 1.f;
         int prev_t0 = tb, prev_L = 0;
-        for (int t0 = tb; t0 < te && ok; t0 += C, ++c) {
+        for (int t0 = tb; t0 < te; t0 += C, ++c) {
           const int st = c & 1;
-          const uint32_t stg = sbase + S_STG + uint32_t(st) * STG_BYTES;
           const float* sg = reinterpret_cast<const float*>(smem + S_STG + st * STG_BYTES + STG_GATE);
           if (c > c_first) {  // dH of the previous chunk landed
-            ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u);
+            ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u) && ok;
             tc_fence_after();
           }
           ok = ok && mbar_wait(&bars[SB_STGF + st], (c >> 1) & 1, abort_flag, err, 16u);
@@ -602,20 +603,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_row64_bf16(sbase + S_HT + uint32_t(hh) * 16384, uint32_t(j), H);
           fence_proxy_async_smem();
           tc_fence_before();
-          if (!named_all(1, 256, ok)) {
-            ok = false;
+          if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts [W; Q]
+            agreed = false;
             break;
           }
-          if (issuer) {  // [Vn' | O1]^T = H^T [W; Q]^T
-            tc_fence_after();
-            for (int kk = 0; kk < ksteps_d; ++kk) {
-              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_bf16_ss(tmem + ST_VO + 128u * st, make_sdesc_sw128(sbase + S_HT + off, 16, 1024),
-                          make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_vo, kk > 0);
-            }
-            mma_commit(&bars[SB_VOFULL]);
-          }
-          if (c > c_first) ok = epilogue(c - 1, prev_t0, prev_L, h) && ok;
+          bool okE = true;
+          if (c > c_first) okE = epilogue(c - 1, 0, prev_t0, prev_L, h);
+          ok = ok && okE;
           // Vn = U - Vn'  ->  Vn^T and e^{G_C - G_r} Vn^T rows in bf16
           ok = mbar_wait(&bars[SB_VOFULL], c & 1, abort_flag, err, 16u) && ok;
           tc_fence_after();
@@ -650,30 +644,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
           tc_fence_before();
-          if (!named_all(1, 256, ok)) {
-            ok = false;
+          if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts dH, O2
+            agreed = false;
             break;
           }
-          if (issuer) {
-            tc_fence_after();
-            // dH^T = Vns^T K (fresh), then O2^T = Vn^T Aqk^T
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(tmem + ST_DH, make_sdesc_sw128(sbase + S_VNS + kk * 32, 16, 1024),
-                          make_sdesc_sw128(stg + STG_K + kk * 2048, 8192, 1024), id_dh, kk > 0);
-            mma_commit(&bars[SB_DHFULL]);
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(tmem + ST_O2 + 64u * st, make_sdesc_sw128(sbase + S_VN + kk * 32, 16, 1024),
-                          make_sdesc_sw128(stg + STG_AQK + kk * 32, 16, 1024), id_o2, kk > 0);
-            mma_commit(&bars[SB_OFULL + st]);
-            mma_commit(&bars[SB_STGE + st]);
-          }
+          if (c > c_first) ok = epilogue(c - 1, 1, prev_t0, prev_L, h) && okE && ok;
           dec_prev = dec_cur;
           prev_t0 = t0;
           prev_L = min(C, te - t0);
         }
-        if (!ok) break;
+        if (!agreed) {
+          ok = false;
+          break;
+        }
         if (te > tb) {  // the last chunk: its update and its outputs
-          ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u);
+          ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u) && ok;
           tc_fence_after();
 #pragma unroll
           for (int q2 = 0; q2 < 2; ++q2) {
@@ -683,8 +668,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) H[32 * q2 + i] = fmaf(dec_prev, H[32 * q2 + i], d[i]);
           }
-          ok = epilogue(c - 1, prev_t0, prev_L, h) && ok;
-          if (!named_all(1, 256, ok)) {
+          ok = epilogue(c - 1, 0, prev_t0, prev_L, h) && ok;
+          ok = epilogue(c - 1, 1, prev_t0, prev_L, h) && ok;
+          if (!named_all(1, kSpineSync, ok)) {  // the issuer warp takes part
             ok = false;
             break;
           }
@@ -697,10 +683,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
       }
-      if (issuer) {  // every MMA this thread issued has completed
+    } else if (warp == 9) {
+      // ---------------- issuer: joins the state warps' two barriers per chunk
+      // (bar.red: every participant gets the same outcome) and issues
+      //   after the first:  [Vn' | O1]^T = H^T [W; Q]^T              (N = 128)
+      //   after the second: dH^T = Vns^T K (fresh), O2^T = Vn^T Aqk^T
+      const uint32_t id_vo = make_idesc_bf16(128, 128, 0, 0);
+      const uint32_t id_dh = make_idesc_bf16(128, 128, 0, 1);
+      const uint32_t id_o2 = make_idesc_bf16(128, 64, 0, 0);
+      const bool leader = lane == 0;
+      int c = 0;
+      for (int u = s; u < units; u += p.S) {
+        int tb, te;
+        seq_range(p, u / p.H_v, tb, te);
+        bool agreed = true;
+        for (int t0 = tb; t0 < te; t0 += C, ++c) {
+          const int st = c & 1;
+          const uint32_t stg = sbase + S_STG + uint32_t(st) * STG_BYTES;
+          if (!named_all(1, kSpineSync, true)) {
+            agreed = false;
+            break;
+          }
+          if (leader) {
+            tc_fence_after();
+            for (int kk = 0; kk < ksteps_d; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+              mma_bf16_ss(tmem + ST_VO + 128u * st, make_sdesc_sw128(sbase + S_HT + off, 16, 1024),
+                          make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_vo, kk > 0);
+            }
+            mma_commit(&bars[SB_VOFULL]);
+          }
+          __syncwarp();
+          if (!named_all(1, kSpineSync, true)) {
+            agreed = false;
+            break;
+          }
+          if (leader) {
+            tc_fence_after();
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(tmem + ST_DH, make_sdesc_sw128(sbase + S_VNS + kk * 32, 16, 1024),
+                          make_sdesc_sw128(stg + STG_K + kk * 2048, 8192, 1024), id_dh, kk > 0);
+            mma_commit(&bars[SB_DHFULL]);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(tmem + ST_O2 + 64u * st,
+                          make_sdesc_sw128(sbase + S_VN + kk * 32, 16, 1024),
+                          make_sdesc_sw128(stg + STG_AQK + kk * 32, 16, 1024), id_o2, kk > 0);
+            mma_commit(&bars[SB_OFULL + st]);
+            mma_commit(&bars[SB_STGE + st]);
+          }
+          __syncwarp();
+        }
+        if (!agreed) break;
+        if (te > tb && !named_all(1, kSpineSync, true)) break;  // the unit-end agreement
+      }
+      if (leader) {  // every MMA this thread issued has completed
         mma_commit(&bars[SB_DRAIN]);
         mbar_wait(&bars[SB_DRAIN], 0, nullptr, err, 8u);
       }
+      __syncwarp();
     } else if (warp == 8) {
       // ---------------- feeder: the tiles of chunk c into stage c & 1 once the
       // chunk c - 2 MMAs released it: K and Q by TMA, then (when a prep has
