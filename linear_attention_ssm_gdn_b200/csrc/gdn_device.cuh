@@ -78,9 +78,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for phase `parity` of `bar` to complete.  Gives up (returns false) when
 // *abort becomes nonzero or after kSpinLimitCycles; on a timeout it sets
 // *abort and ORs `err_bit` into *err (a global error word, may be null).
-static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                       uint32_t* err, uint32_t err_bit) {
-  if (mbar_try_wait(bar, parity)) return true;
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
+                                                    volatile int* abort, uint32_t* err,
+                                                    uint32_t err_bit) {
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -91,6 +91,14 @@ static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, vo
       return false;
     }
   }
+}
+
+// The common case (the phase is already complete) stays inline: a call costs
+// the caller its live registers around the call site.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint32_t* err, uint32_t err_bit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort, err, err_bit);
 }
 
 // ---------------------------------------------------------------------------

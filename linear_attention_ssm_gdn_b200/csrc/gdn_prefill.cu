@@ -539,15 +539,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int e0 = 32 * qd;
         {
           const int r0 = 32 * hh + 16 * pc;
+          // every operand in registers first: the shared stores below carry a
+          // memory clobber, which would serialise loads placed between them
+          float egv[16];
+#pragma unroll
+          for (int i = 0; i < 16; i += 4) {
+            const float4 e4 = *reinterpret_cast<const float4*>(egp + r0 + i);
+            egv[i] = e4.x;
+            egv[i + 1] = e4.y;
+            egv[i + 2] = e4.z;
+            egv[i + 3] = e4.w;
+          }
           float o1[16], o2[16];
           tmem_ld16(tmem + lane_off + ST_VO + 128u * ob + 64u + uint32_t(r0), o1);
           tmem_ld16(tmem + lane_off + ST_O2 + 64u * ob + uint32_t(r0), o2);
           tmem_ld_wait();
+          uint32_t packed[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            packed[i] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(egv[i], o1[i], o2[i])));
           __syncwarp();  // the previous piece's reads of the buffer are done
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            st_shared_u16(ostg + uint32_t(i) * 64 + uint32_t(lane) * 2,
-                          __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(egp[r0 + i], o1[i], o2[i]))));
+            st_shared_u16(ostg + uint32_t(i) * 64 + uint32_t(lane) * 2, uint16_t(packed[i]));
           __syncwarp();
 #pragma unroll
           for (int m = 0; m < 2; ++m) {
@@ -614,18 +628,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&bars[SB_VOFULL], c & 1, abort_flag, err, 16u) && ok;
           tc_fence_after();
           {
+            // loads first (see the outputs above), then the shared stores
             const uint8_t* urow = smem + S_STG + st * STG_BYTES + STG_U;
+            uint4 uvs[4];
+            float4 eca[4], ecb[4];
+#pragma unroll
+            for (int hc = 0; hc < 4; ++hc) {
+              const int cc = 4 * hh + hc;
+              uvs[hc] = *reinterpret_cast<const uint4*>(urow + sw128_offset(j, cc * 16));
+              eca[hc] = *reinterpret_cast<const float4*>(sg + 64 + 8 * cc);
+              ecb[hc] = *reinterpret_cast<const float4*>(sg + 64 + 8 * cc + 4);
+            }
             float vn[32];
             tmem_ld32(tmem + lane_off + ST_VO + 128u * st + 32u * uint32_t(hh), vn);
             tmem_ld_wait();
 #pragma unroll
             for (int hc = 0; hc < 4; ++hc) {
               const int cc = 4 * hh + hc;
-              const uint4 uv = *reinterpret_cast<const uint4*>(urow + sw128_offset(j, cc * 16));
-              const float4 e0 = *reinterpret_cast<const float4*>(sg + 64 + 8 * cc);
-              const float4 e1 = *reinterpret_cast<const float4*>(sg + 64 + 8 * cc + 4);
+              const float4 e0 = eca[hc], e1 = ecb[hc];
               const float ec[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-              const uint32_t uw[4] = {uv.x, uv.y, uv.z, uv.w};
+              const uint32_t uw[4] = {uvs[hc].x, uvs[hc].y, uvs[hc].z, uvs[hc].w};
               float x[8], y[8];
 #pragma unroll
               for (int k2 = 0; k2 < 4; ++k2) {
