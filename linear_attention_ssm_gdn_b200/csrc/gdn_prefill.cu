@@ -72,9 +72,11 @@ constexpr uint32_t SLOT_TX = G_GATE + G_GATE_BYTES;
 constexpr uint32_t kFlagLine = 64;
 
 // ---- spine shared memory (bytes from a 1024-aligned base): two chunk stages
-// of STG_BYTES, each holding everything one chunk step reads:
-//   [box b: W rows 64x128B | Q rows 64x128B] x 2  (the N = 128 B operand [W; Q])
-//   K [box b: 64 x 128B] x 2,  U^T [128 x 128B],  Aqk [64 x 128B],  gate factors
+// of STG_BYTES, each holding everything one chunk step reads, in two parts
+// that are refilled independently:
+//   part A: [box b: W rows 64x128B | Q rows 64x128B] x 2 (the N = 128 B
+//           operand [W; Q]) and the gate factors -- read up to the [W; Q] MMA;
+//   part B: K [box b: 64 x 128B] x 2, U^T [128 x 128B], Aqk [64 x 128B].
 constexpr uint32_t STG_WQ = 0, STG_K = 32768, STG_U = 49152, STG_AQK = 65536, STG_GATE = 73728;
 constexpr uint32_t STG_BYTES = 74752;  // 73 KB
 constexpr uint32_t S_STG = 0;
@@ -82,7 +84,8 @@ constexpr uint32_t S_HT = S_STG + 2 * STG_BYTES;  // H^T bf16, [2 boxes][128 x 1
 constexpr uint32_t S_VN = S_HT + 32768;           // Vn^T bf16 [128 x 128B]
 constexpr uint32_t S_VNS = S_VN + 16384;          // e^{G_C - G_r} Vn^T bf16
 constexpr uint32_t S_EG = S_VNS + 16384;          // 2 x 64 f32: scale e^{G_r} per chunk
-constexpr uint32_t S_OSTG = S_EG + 512;           // output transpose: 8 warps x 1 KB
+constexpr uint32_t S_ECG = S_EG + 512;            // 2 x 64 f32: e^{G_C - G_r} per chunk
+constexpr uint32_t S_OSTG = S_ECG + 512;          // output transpose: 8 warps x 1 KB
 constexpr uint32_t S_BARS = S_OSTG + 8192;
 static_assert(S_HT % 1024 == 0 && STG_BYTES % 1024 == 0, "swizzled tiles are 1024-aligned");
 static_assert(STG_GATE + G_GATE_BYTES <= STG_BYTES, "stage layout");
@@ -114,13 +117,15 @@ static_assert((P_GATE + PG_EG * 4) % 16 == 0 && (P_GATE + PG_BYTES + PG_EG * 4) 
 
 // ---- barriers (spine)
 enum {
-  SB_STGF = 0,     // +stage: every tile of the chunk landed (TMA + bulk loads)
-  SB_STGE = 2,     // +stage: the chunk's MMAs are done, the stage is free (commit)
-  SB_VOFULL = 4,   // H^T [W; Q]^T done (commit)
-  SB_DHFULL = 5,   // dH = Vns^T K done (commit)
-  SB_OFULL = 6,    // +buf: O2 (and so O1) done (commit)
-  SB_DRAIN = 8,
-  SB_COUNT = 9
+  SB_AF = 0,       // +stage: part A landed: Q (TMA), W and the gate factors (bulk)
+  SB_AE = 2,       // +stage: part A free: the [W; Q] MMA is done (commit)
+  SB_BF = 4,       // +stage: part B landed: K (TMA), U^T and Aqk (bulk)
+  SB_BE = 6,       // +stage: part B free: dH and O2 are done (commit)
+  SB_VOFULL = 8,   // H^T [W; Q]^T done (commit)
+  SB_DHFULL = 9,   // dH = Vns^T K done (commit)
+  SB_OFULL = 10,   // +buf: O2 (and so O1) done (commit)
+  SB_DRAIN = 12,
+  SB_COUNT = 13
 };
 // ---- barriers (prep); per group w: base + w (GATEF / GATEE: base + 2w + b)
 enum {
@@ -526,6 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool jv = j < D;
       const uint32_t ostg = sbase + S_OSTG + uint32_t(warp) * 1024;
       float* eg_s = reinterpret_cast<float*>(smem + S_EG);
+      float* ecg_s = reinterpret_cast<float*>(smem + S_ECG);
       // Outputs of chunk cl, 16 of this warp's rows 32 hh .. + 31 per call
       // (piece pc), for the d_v lanes of its quadrant: o_r = scale e^{G_r}
       // O1[r] + O2[r], transposed through this warp's 1 KB buffer and written
@@ -601,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u) && ok;
             tc_fence_after();
           }
-          ok = ok && mbar_wait(&bars[SB_STGF + st], (c >> 1) & 1, abort_flag, err, 16u);
+          ok = ok && mbar_wait(&bars[SB_AF + st], (c >> 1) & 1, abort_flag, err, 16u);
           if (c > c_first) {  // H <- e^{G_C} H + dH
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
@@ -613,7 +619,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           const float dec_cur = sg[128];
+          // part A is released after the [W; Q] MMA: keep the gate factors
           if (tid < 64) eg_s[64 * st + tid] = sg[tid] * p.scale;
+          else if (tid < 128) ecg_s[64 * st + tid - 64] = sg[tid];
           st_row64_bf16(sbase + S_HT + uint32_t(hh) * 16384, uint32_t(j), H);
           fence_proxy_async_smem();
           tc_fence_before();
@@ -626,42 +634,47 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = ok && okE;
           // Vn = U - Vn'  ->  Vn^T and e^{G_C - G_r} Vn^T rows in bf16
           ok = mbar_wait(&bars[SB_VOFULL], c & 1, abort_flag, err, 16u) && ok;
+          ok = mbar_wait(&bars[SB_BF + st], (c >> 1) & 1, abort_flag, err, 16u) && ok;
           tc_fence_after();
           {
-            // loads first (see the outputs above), then the shared stores
             const uint8_t* urow = smem + S_STG + st * STG_BYTES + STG_U;
-            uint4 uvs[4];
-            float4 eca[4], ecb[4];
-#pragma unroll
-            for (int hc = 0; hc < 4; ++hc) {
-              const int cc = 4 * hh + hc;
-              uvs[hc] = *reinterpret_cast<const uint4*>(urow + sw128_offset(j, cc * 16));
-              eca[hc] = *reinterpret_cast<const float4*>(sg + 64 + 8 * cc);
-              ecb[hc] = *reinterpret_cast<const float4*>(sg + 64 + 8 * cc + 4);
-            }
+            const float* ecp = ecg_s + 64 * st;
             float vn[32];
             tmem_ld32(tmem + lane_off + ST_VO + 128u * st + 32u * uint32_t(hh), vn);
             tmem_ld_wait();
 #pragma unroll
-            for (int hc = 0; hc < 4; ++hc) {
-              const int cc = 4 * hh + hc;
-              const float4 e0 = eca[hc], e1 = ecb[hc];
-              const float ec[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-              const uint32_t uw[4] = {uvs[hc].x, uvs[hc].y, uvs[hc].z, uvs[hc].w};
-              float x[8], y[8];
+            for (int h2 = 0; h2 < 2; ++h2) {
+              // two 8-column chunks: loads first, then the shared stores
+              uint4 uvs[2];
+              float4 eca[2], ecb[2];
 #pragma unroll
-              for (int k2 = 0; k2 < 4; ++k2) {
-                x[2 * k2] = __uint_as_float(uw[k2] << 16) - vn[8 * hc + 2 * k2];
-                x[2 * k2 + 1] = __uint_as_float(uw[k2] & 0xFFFF0000u) - vn[8 * hc + 2 * k2 + 1];
+              for (int q = 0; q < 2; ++q) {
+                const int cc = 4 * hh + 2 * h2 + q;
+                uvs[q] = *reinterpret_cast<const uint4*>(urow + sw128_offset(j, cc * 16));
+                eca[q] = *reinterpret_cast<const float4*>(ecp + 8 * cc);
+                ecb[q] = *reinterpret_cast<const float4*>(ecp + 8 * cc + 4);
               }
 #pragma unroll
-              for (int m = 0; m < 8; ++m) y[m] = x[m] * ec[m];
-              st_shared_v4(sbase + S_VN + sw128_offset(j, cc * 16), pack_bf16x2(x[0], x[1]),
-                           pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                           pack_bf16x2(x[6], x[7]));
-              st_shared_v4(sbase + S_VNS + sw128_offset(j, cc * 16), pack_bf16x2(y[0], y[1]),
-                           pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                           pack_bf16x2(y[6], y[7]));
+              for (int q = 0; q < 2; ++q) {
+                const int hc = 2 * h2 + q, cc = 4 * hh + hc;
+                const float4 e0 = eca[q], e1 = ecb[q];
+                const float ec[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+                const uint32_t uw[4] = {uvs[q].x, uvs[q].y, uvs[q].z, uvs[q].w};
+                float x[8], y[8];
+#pragma unroll
+                for (int k2 = 0; k2 < 4; ++k2) {
+                  x[2 * k2] = __uint_as_float(uw[k2] << 16) - vn[8 * hc + 2 * k2];
+                  x[2 * k2 + 1] = __uint_as_float(uw[k2] & 0xFFFF0000u) - vn[8 * hc + 2 * k2 + 1];
+                }
+#pragma unroll
+                for (int m = 0; m < 8; ++m) y[m] = x[m] * ec[m];
+                st_shared_v4(sbase + S_VN + sw128_offset(j, cc * 16), pack_bf16x2(x[0], x[1]),
+                             pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                             pack_bf16x2(x[6], x[7]));
+                st_shared_v4(sbase + S_VNS + sw128_offset(j, cc * 16), pack_bf16x2(y[0], y[1]),
+                             pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                             pack_bf16x2(y[6], y[7]));
+              }
             }
           }
           fence_proxy_async_smem();
@@ -734,6 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_vo, kk > 0);
             }
             mma_commit(&bars[SB_VOFULL]);
+            mma_commit(&bars[SB_AE + st]);
           }
           __syncwarp();
           if (!named_all(1, kSpineSync, true)) {
@@ -751,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           make_sdesc_sw128(sbase + S_VN + kk * 32, 16, 1024),
                           make_sdesc_sw128(stg + STG_AQK + kk * 32, 16, 1024), id_o2, kk > 0);
             mma_commit(&bars[SB_OFULL + st]);
-            mma_commit(&bars[SB_STGE + st]);
+            mma_commit(&bars[SB_BE + st]);
           }
           __syncwarp();
         }
@@ -764,47 +778,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     } else if (warp == 8) {
-      // ---------------- feeder: the tiles of chunk c into stage c & 1 once the
-      // chunk c - 2 MMAs released it: K and Q by TMA, then (when a prep has
-      // published it) the ring entry: W next to Q, U^T, Aqk and the gates.
-      // It also hands chunk c - 2's ring entry back to the preps.
+      // ---------------- feeder: chunk c into stage c & 1, part by part.
+      // Part A (Q by TMA; W and the gates from the ring entry) as soon as
+      // chunk c - 2's [W; Q] MMA is done; part B (K by TMA; U^T and Aqk) once
+      // chunk c - 2's dH and O2 are done, when its ring entry also goes back
+      // to the preps.
       if (lane == 0) {
         ChunkIter fd;
         it_start(fd, p, s);
-        int issued = 0;
+        int issued_a = 0, issued_b = 0;
         bool ok = true;
         while (fd.ok && ok) {
           const int cc = fd.c, st = cc & 1;
+          uint8_t* stg = smem + S_STG + st * STG_BYTES;
+          const int hk = fd.h / vpg;
+          const uint8_t* src = ring_entry(p, s, cc % kRing);
+          // ---- part A
           if (cc >= 2) {
-            ok = mbar_wait(&bars[SB_STGE + st], ((cc >> 1) & 1) ^ 1, abort_flag, err, 1u);
+            ok = mbar_wait(&bars[SB_AE + st], ((cc >> 1) & 1) ^ 1, abort_flag, err, 1u);
+            if (!ok) break;
+          }
+          uint64_t* fa = &bars[SB_AF + st];
+          // The phase completes on the one arrival (made with the ring bytes, or
+          // bare on an abort) plus every byte announced before it.
+          mbar_expect_tx(fa, uint32_t(nbox) * 8192);
+          for (int b = 0; b < nbox; ++b)
+            tma_load_3d(stg + STG_WQ + b * 16384 + 8192, &tm_q, fa, b * 64, hk, fd.t0);
+          issued_a = cc + 1;
+          ok = poll_geq(ready_flag(p, s, cc % kRing), uint32_t(cc + 1), gabort, err, 1u);
+          if (!ok) {  // the phase still completes once the Q tiles landed
+            mbar_arrive(fa);
+            break;
+          }
+          fence_proxy_async_global();
+          mbar_arrive_expect_tx(fa, 2 * 8192 + G_GATE_BYTES);
+          bulk_load_g2s(stg + STG_WQ, src + G_W, 8192, fa);
+          bulk_load_g2s(stg + STG_WQ + 16384, src + G_W + 8192, 8192, fa);
+          bulk_load_g2s(stg + STG_GATE, src + G_GATE, G_GATE_BYTES, fa);
+          // ---- part B
+          if (cc >= 2) {
+            ok = mbar_wait(&bars[SB_BE + st], ((cc >> 1) & 1) ^ 1, abort_flag, err, 1u);
             if (!ok) break;
             // chunk cc - 2 is fully consumed: its ring entry may be reused
             st_release_gpu(free_flag(p, s, (cc - 2) % kRing), uint32_t(cc - 1));
           }
-          uint8_t* stg = smem + S_STG + st * STG_BYTES;
-          uint64_t* fb = &bars[SB_STGF + st];
-          // The phase completes on the one arrival (made with the ring bytes, or
-          // bare on an abort) plus every byte announced before it.
-          mbar_expect_tx(fb, uint32_t(nbox) * 2 * 8192);
-          const int hk = fd.h / vpg;
-          for (int b = 0; b < nbox; ++b) {
+          uint64_t* fb = &bars[SB_BF + st];
+          mbar_arrive_expect_tx(fb, uint32_t(nbox) * 8192 + 16384 + 8192);
+          for (int b = 0; b < nbox; ++b)
             tma_load_3d(stg + STG_K + b * 8192, &tm_k, fb, b * 64, hk, fd.t0);
-            tma_load_3d(stg + STG_WQ + b * 16384 + 8192, &tm_q, fb, b * 64, hk, fd.t0);
-          }
-          issued = cc + 1;
-          ok = poll_geq(ready_flag(p, s, cc % kRing), uint32_t(cc + 1), gabort, err, 1u);
-          if (!ok) {  // the phase still completes once the K/Q tiles landed
-            mbar_arrive(fb);
-            break;
-          }
-          fence_proxy_async_global();
-          mbar_arrive_expect_tx(fb, 2 * 8192 + 16384 + 8192 + G_GATE_BYTES);
-          const uint8_t* src = ring_entry(p, s, cc % kRing);
-          bulk_load_g2s(stg + STG_WQ, src + G_W, 8192, fb);
-          bulk_load_g2s(stg + STG_WQ + 16384, src + G_W + 8192, 8192, fb);
           bulk_load_g2s(stg + STG_U, src + G_U, 16384, fb);
           bulk_load_g2s(stg + STG_AQK, src + G_AQK, 8192, fb);
-          bulk_load_g2s(stg + STG_GATE, src + G_GATE, G_GATE_BYTES, fb);
+          issued_b = cc + 1;
           it_next(fd, p);
         }
         if (!ok) {
@@ -812,8 +836,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           atomicExch(const_cast<uint32_t*>(gabort), 1u);
         }
         // nothing may still be landing in shared memory at exit
-        for (int cc = issued - 2; cc < issued; ++cc)
-          if (cc >= 0) mbar_wait(&bars[SB_STGF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
+        for (int cc = issued_a - 2; cc < issued_a; ++cc)
+          if (cc >= 0) mbar_wait(&bars[SB_AF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
+        for (int cc = issued_b - 2; cc < issued_b; ++cc)
+          if (cc >= 0) mbar_wait(&bars[SB_BF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
       }
       __syncwarp();
     }
