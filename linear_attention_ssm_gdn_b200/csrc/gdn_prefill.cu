@@ -89,22 +89,24 @@ constexpr uint32_t S_OSTG = S_ECG + 512;          // output transpose: 8 warps x
 constexpr uint32_t S_BARS = S_OSTG + 8192;
 static_assert(S_HT % 1024 == 0 && STG_BYTES % 1024 == 0, "swizzled tiles are 1024-aligned");
 static_assert(STG_GATE + G_GATE_BYTES <= STG_BYTES, "stage layout");
-// ---- prep shared memory: one 256-thread worker, two tile sets (item parity)
-// so that the next item's tiles load while this one is worked on
-constexpr uint32_t P_SET = 49152;   // per set: [box b: K 8K | Q 8K] x 2, V [box b: 8K] x 2
-constexpr uint32_t P_KQ = 0;        // inside a set; after the item's W/U MMAs the set
-constexpr uint32_t P_V = 32768;     //   holds its W | U^T staging instead
-constexpr uint32_t P_AF = 2 * P_SET;            // A f32 [64][kAS]
-constexpr uint32_t P_TF = P_AF + 64 * kAS * 4;  // T f32 [64][kAS]
-constexpr uint32_t P_XS = P_TF + 64 * kAS * 4;  // inverse scratch 32x32 f32
-constexpr uint32_t P_T1B = (P_XS + 4096 + 1023) / 1024 * 1024;  // T diag(beta e^G) bf16 [64 x 128B]
-constexpr uint32_t P_T2B = P_T1B + 8192;                          // T diag(beta) bf16
-constexpr uint32_t P_AQK = P_T2B + 8192;                          // 2 x Aqk bf16 (item parity)
-constexpr uint32_t P_GATE = P_AQK + 2 * 8192;                     // 2 gate blocks (item parity)
+// ---- prep shared memory: two 128-thread item groups (item k: group k & 1)
+// and three tile sets that rotate over the items (item k: set k % 3), so that
+// one set is always being filled for the next item.  In a set, after P1 the Q
+// boxes hold T diag(beta e^G) and T diag(beta) (bf16), and after the W/U MMAs
+// [0, 32 KB) holds the item's W | U^T staging.
+constexpr uint32_t P_SET = 49152;   // [box b: K 8K | Q 8K] x 2, V [box b: 8K] x 2
+constexpr uint32_t P_KQ = 0, P_V = 32768;
+constexpr uint32_t P_T1B = 8192, P_T2B = 24576;  // in the Q boxes, inside a set
+constexpr uint32_t P_GRP = 3 * P_SET;            // the groups' own areas
+constexpr uint32_t GA_AF = 0;                     // A, then T in place: f32 [64][kAS]
+constexpr uint32_t GA_XS = GA_AF + 64 * kAS * 4;  // inverse scratch 32x32 f32
+constexpr uint32_t GA_AQK = (GA_XS + 4096 + 1023) / 1024 * 1024;  // Aqk bf16 [64 x 128B]
+constexpr uint32_t GA_GT = GA_AQK + 8192;         // 2 gate blocks
 constexpr int PG_G = 0, PG_BET = 64, PG_E1 = 128, PG_E2 = 192, PG_BEG = 448, PG_EG = 512,
               PG_ECG = 576, PG_DEC = 640;  // floats; PG_EG..PG_DEC+3 is the published block
 constexpr uint32_t PG_BYTES = 644 * 4;
-constexpr uint32_t P_BARS = (P_GATE + 2 * PG_BYTES + 15) / 16 * 16;
+constexpr uint32_t P_GS = (GA_GT + 2 * PG_BYTES + 1023) / 1024 * 1024;  // bytes per group
+constexpr uint32_t P_BARS = P_GRP + 2 * P_GS;
 constexpr uint32_t BAR_BYTES = 32 * 8;
 constexpr uint32_t kMiscBytes = 16 + 4 * kMaxSpines;  // TMEM base, abort word, chunks per spine
 constexpr uint32_t kSmemBytes =
@@ -113,9 +115,10 @@ constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 static_assert(S_BARS % 8 == 0 && P_BARS % 8 == 0, "barrier alignment");
 static_assert(P_V >= 32768, "W | U^T staging fits in a tile set");
-static_assert((P_GATE + PG_EG * 4) % 16 == 0 && (P_GATE + PG_BYTES + PG_EG * 4) % 16 == 0,
-              "gate blocks are bulk-copy sources");
-static_assert(P_SET % 1024 == 0 && P_T1B % 1024 == 0 && P_AQK % 1024 == 0, "swizzled tiles");
+static_assert((GA_GT + PG_EG * 4) % 16 == 0 && (GA_GT + PG_BYTES + PG_EG * 4) % 16 == 0 &&
+                  P_GS % 16 == 0, "gate blocks are bulk-copy sources");
+static_assert(P_SET % 1024 == 0 && P_GRP % 1024 == 0 && P_GS % 1024 == 0 && GA_AQK % 1024 == 0,
+              "swizzled tiles");
 
 // ---- barriers (spine)
 enum {
@@ -129,25 +132,25 @@ enum {
   SB_DRAIN = 12,
   SB_COUNT = 13
 };
-// ---- barriers (prep); "+b" = per item parity (tile set, TMEM buffer, Aqk and
-// gate block of items k with k & 1 == b)
+// ---- barriers (prep).  Item k: group g = k & 1, kg = k >> 1 its index in
+// the group, tile set k % 3, P1 buffer and gate block kg & 1 of group g.
 enum {
-  PB_KQVF = 0,     // +b: K, Q, V tiles landed (TMA)
-  PB_STORED = 2,   // +b: item's staging, Aqk and gates read by the bulk store (1)
-  PB_P1F = 4,      // +b: P1 = [K;Q] K^T done (commit)
-  PB_P1FREE = 6,   // +b: P1 read back (256)
-  PB_TREADY = 8,   // T1, T2 written (256)
-  PB_WUF = 9,      // +b: W^T, U^T done (commit)
-  PB_GATEF = 11,   // +b: gate block written (32, the loader warp)
-  PB_STAGED = 13,  // W | U^T staged (1)
-  PB_DRAIN = 14,
-  PB_COUNT = 15
+  PB_KQVF = 0,     // +set: K, Q, V tiles landed (TMA)
+  PB_STORED = 3,   // +set: the item's staging, Aqk and gates read by the bulk store (1)
+  PB_P1F = 6,      // +2g+buf: P1 = [K;Q] K^T done (commit)
+  PB_P1FREE = 10,  // +2g+buf: P1 read back (128)
+  PB_TREADY = 14,  // +g: T1, T2 written (128)
+  PB_WUF = 16,     // +g: W^T, U^T done (commit)
+  PB_GATEF = 18,   // +2g+buf: gate block written (32, the loader warp)
+  PB_STAGED = 22,  // +g: W | U^T staged (1)
+  PB_DRAIN = 24,
+  PB_COUNT = 25
 };
 
 // ---- TMEM columns
 // spine: [H^T W^T | O1^T] x2 (128 columns each), O2^T x2, dH^T (lane j = row j of H^T)
 constexpr uint32_t ST_VO = 0, ST_O2 = 256, ST_DH = 384;
-constexpr uint32_t PT_P1 = 0, PT_W = 64, PT_U = 128, PT_WG = 192;  // prep, per item parity
+constexpr uint32_t PT_W = 128, PT_U = 192, PT_WG = 256;  // prep, per group: P1 x2 at 0, 64
 
 struct Params {
   const float* g;
@@ -308,28 +311,30 @@ __device__ __forceinline__ bool named_all(int id, int nthreads, bool v) {
 }
 
 // ---------------------------------------------------------------------------
-// T = (I + A)^{-1} for a strictly lower triangular 64x64 A (f32, row stride
-// kAS), 256 threads (8 warps), with 16x16 blocks D_i = (I + A_ii)^{-1}:
-//   1. warps 0-3: D_w by forward substitution (lane j < 16 owns column j and
-//      pushes each new x_l into the running sums of the rows below it); lanes
-//      16-31 of warps 0 and 2 clear the upper blocks T_{0,1}, T_{2,3}, which
-//      steps 3 and 4 read as zeros (the scratch is reused between items);
-//   2. warp pair p of warps 0-3 (blocks 2p, 2p+1):
-//      T_{2p+1,2p} = -D_{2p+1} A_{2p+1,2p} D_{2p};
-//   3. X = A[32:64, 0:32] T[0:32, 0:32]       (thread: one row, four columns);
-//   4. T[32:64, 0:32] = -T[32:64, 32:64] X.
-// Named barriers: bar_all (256 threads), bar_pair and bar_pair + 1 (64 each).
-// X and the pair products use the 32x32 f32 scratch Xs.
+// T = (I + A)^{-1} in place: on entry M holds the strictly lower triangular
+// 64x64 A (f32, row stride kAS, zeros on and above the diagonal), on exit the
+// unit lower triangular T.  128 threads (4 warps), 16x16 blocks
+// D_i = (I + A_ii)^{-1}:
+//   1. warp w: D_w by forward substitution (lane j < 16 owns column j and
+//      pushes each new x_l into the running sums of the rows below it), then
+//      written over A_ww;
+//   2. warp pair p (blocks 2p, 2p+1): T_{2p+1,2p} = -D_{2p+1} A_{2p+1,2p} D_{2p},
+//      written over A_{2p+1,2p} once the pair has read it;
+//   3. X = A[32:64, 0:32] T[0:32, 0:32];
+//   4. T[32:64, 0:32] = -T[32:64, 32:64] X, written over A[32:64, 0:32].
+// The upper blocks stay the zeros of A.  Each thread of steps 2-4 owns a small
+// output tile.  bar_base: named barrier ids bar_base (128 threads),
+// bar_base+1+p (pairs).  X and the pair products use the 32x32 f32 scratch Xs.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void invert_unit_lower64(const float* Af, float* Tf, float* Xs, int p,
-                                                    int bar_all, int bar_pair) {
+__device__ __forceinline__ void invert_unit_lower64(float* M, float* Xs, int p, int bar_base) {
   const int w = p >> 5, ln = p & 31;
-  if (w < 4) {
-    // 1. diagonal blocks
+  // 1. diagonal blocks
+  {
+    float x[16];
+    const int j = ln;
     if (ln < 16) {
-      const int j = ln;
-      const float* Ab = Af + (16 * w) * kAS + 16 * w;
-      float x[16], acc[16];
+      const float* Ab = M + (16 * w) * kAS + 16 * w;
+      float acc[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) acc[i] = 0.f;
 #pragma unroll
@@ -338,30 +343,31 @@ __device__ __forceinline__ void invert_unit_lower64(const float* Af, float* Tf, 
 #pragma unroll
         for (int i = l + 1; i < 16; ++i) acc[i] = fmaf(Ab[i * kAS + l], x[l], acc[i]);
       }
-      float* Tb = Tf + (16 * w) * kAS + 16 * w + j;
+    }
+    __syncwarp();  // every lane has read A_ww
+    if (ln < 16) {
+      float* Tb = M + (16 * w) * kAS + 16 * w + j;
 #pragma unroll
       for (int i = 0; i < 16; ++i) Tb[i * kAS] = x[i];
-    } else if ((w & 1) == 0) {
-      float* Tz = Tf + (16 * w) * kAS + 16 * (w + 1) + (ln - 16);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) Tz[i * kAS] = 0.f;
     }
-    // 2. first sub-diagonal blocks: thread t of the pair owns row t>>2,
-    //    columns 4(t&3)..+3
+  }
+  // 2. first sub-diagonal blocks, one per warp pair: thread t of the pair owns
+  //    row t>>2, columns 4(t&3)..+3
+  {
     const int pr = w >> 1, t = p & 63;
     const int bi = 2 * pr + 1, bj = 2 * pr;
     const int i = t >> 2, c4 = 4 * (t & 3);
     float* Y = Xs + pr * 256;
-    named_sync(bar_pair + pr, 64);
+    named_sync(bar_base + 1 + pr, 64);
     float y[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* ar = Af + (16 * bi + i) * kAS + 16 * bj;
+    const float* ar = M + (16 * bi + i) * kAS + 16 * bj;
 #pragma unroll
     for (int l = 0; l < 16; l += 4) {
       const float4 a = *reinterpret_cast<const float4*>(ar + l);
       const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        const float4 d = *reinterpret_cast<const float4*>(Tf + (16 * bj + l + m) * kAS + 16 * bj + c4);
+        const float4 d = *reinterpret_cast<const float4*>(M + (16 * bj + l + m) * kAS + 16 * bj + c4);
         y[0] = fmaf(av[m], d.x, y[0]);
         y[1] = fmaf(av[m], d.y, y[1]);
         y[2] = fmaf(av[m], d.z, y[2]);
@@ -369,9 +375,9 @@ __device__ __forceinline__ void invert_unit_lower64(const float* Af, float* Tf, 
       }
     }
     *reinterpret_cast<float4*>(Y + i * 16 + c4) = make_float4(y[0], y[1], y[2], y[3]);
-    named_sync(bar_pair + pr, 64);
+    named_sync(bar_base + 1 + pr, 64);  // A_{2p+1,2p} read by the pair
     float z[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* dr = Tf + (16 * bi + i) * kAS + 16 * bi;
+    const float* dr = M + (16 * bi + i) * kAS + 16 * bi;
 #pragma unroll
     for (int l = 0; l < 16; l += 4) {
       const float4 a = *reinterpret_cast<const float4*>(dr + l);
@@ -385,39 +391,48 @@ __device__ __forceinline__ void invert_unit_lower64(const float* Af, float* Tf, 
         z[3] = fmaf(av[m], yv.w, z[3]);
       }
     }
-    *reinterpret_cast<float4*>(Tf + (16 * bi + i) * kAS + 16 * bj + c4) =
+    *reinterpret_cast<float4*>(M + (16 * bi + i) * kAS + 16 * bj + c4) =
         make_float4(-z[0], -z[1], -z[2], -z[3]);
   }
-  named_sync(bar_all, 256);
-  // 3. X = A[32:64, 0:32] T[0:32, 0:32]; thread p owns row p >> 3, columns 4(p&7)..+3
-  const int r0 = p >> 3, c0 = 4 * (p & 7);
+  named_sync(bar_base, 128);
+  // 3. X = A[32:64, 0:32] T[0:32, 0:32]; thread p owns rows 2(p>>3)..+1, cols 4(p&7)..+3
+  const int r0 = 2 * (p >> 3), c0 = 4 * (p & 7);
   {
-    float x0[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* a0r = Af + (32 + r0) * kAS;
-#pragma unroll 4
+    float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* a0r = M + (32 + r0) * kAS;
+    const float* a1r = a0r + kAS;
+#pragma unroll 2
     for (int k = 0; k < 32; k += 4) {
       const float4 a0 = *reinterpret_cast<const float4*>(a0r + k);
-      const float av0[4] = {a0.x, a0.y, a0.z, a0.w};
+      const float4 a1 = *reinterpret_cast<const float4*>(a1r + k);
+      const float av0[4] = {a0.x, a0.y, a0.z, a0.w}, av1[4] = {a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        const float4 tv = *reinterpret_cast<const float4*>(Tf + (k + m) * kAS + c0);
+        const float4 tv = *reinterpret_cast<const float4*>(M + (k + m) * kAS + c0);
         x0[0] = fmaf(av0[m], tv.x, x0[0]);
         x0[1] = fmaf(av0[m], tv.y, x0[1]);
         x0[2] = fmaf(av0[m], tv.z, x0[2]);
         x0[3] = fmaf(av0[m], tv.w, x0[3]);
+        x1[0] = fmaf(av1[m], tv.x, x1[0]);
+        x1[1] = fmaf(av1[m], tv.y, x1[1]);
+        x1[2] = fmaf(av1[m], tv.z, x1[2]);
+        x1[3] = fmaf(av1[m], tv.w, x1[3]);
       }
     }
     *reinterpret_cast<float4*>(Xs + r0 * 32 + c0) = make_float4(x0[0], x0[1], x0[2], x0[3]);
+    *reinterpret_cast<float4*>(Xs + (r0 + 1) * 32 + c0) = make_float4(x1[0], x1[1], x1[2], x1[3]);
   }
-  named_sync(bar_all, 256);
+  named_sync(bar_base, 128);  // A[32:64, 0:32] read, X complete
   // 4. T[32:64, 0:32] = -T[32:64, 32:64] X  (T[32+r, 32+k] = 0 for k > r)
   {
-    float z0[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* t0r = Tf + (32 + r0) * kAS + 32;
-#pragma unroll 4
+    float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* t0r = M + (32 + r0) * kAS + 32;
+    const float* t1r = t0r + kAS;
+#pragma unroll 2
     for (int k = 0; k < 32; k += 4) {
       const float4 a0 = *reinterpret_cast<const float4*>(t0r + k);
-      const float av0[4] = {a0.x, a0.y, a0.z, a0.w};
+      const float4 a1 = *reinterpret_cast<const float4*>(t1r + k);
+      const float av0[4] = {a0.x, a0.y, a0.z, a0.w}, av1[4] = {a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const float4 xv = *reinterpret_cast<const float4*>(Xs + (k + m) * 32 + c0);
@@ -425,12 +440,18 @@ __device__ __forceinline__ void invert_unit_lower64(const float* Af, float* Tf, 
         z0[1] = fmaf(av0[m], xv.y, z0[1]);
         z0[2] = fmaf(av0[m], xv.z, z0[2]);
         z0[3] = fmaf(av0[m], xv.w, z0[3]);
+        z1[0] = fmaf(av1[m], xv.x, z1[0]);
+        z1[1] = fmaf(av1[m], xv.y, z1[1]);
+        z1[2] = fmaf(av1[m], xv.z, z1[2]);
+        z1[3] = fmaf(av1[m], xv.w, z1[3]);
       }
     }
-    *reinterpret_cast<float4*>(Tf + (32 + r0) * kAS + c0) =
+    *reinterpret_cast<float4*>(M + (32 + r0) * kAS + c0) =
         make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
+    *reinterpret_cast<float4*>(M + (32 + r0 + 1) * kAS + c0) =
+        make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
   }
-  named_sync(bar_all, 256);
+  named_sync(bar_base, 128);
 }
 
 }  // namespace pf
@@ -470,8 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       for (int b = 0; b < PB_COUNT; ++b) {
         uint32_t cnt = 1;
-        if (b == PB_P1FREE || b == PB_P1FREE + 1 || b == PB_TREADY) cnt = 256;
-        if (b == PB_GATEF || b == PB_GATEF + 1) cnt = 32;
+        if ((b >= PB_P1FREE && b < PB_P1FREE + 4) || b == PB_TREADY || b == PB_TREADY + 1) cnt = 128;
+        if (b >= PB_GATEF && b < PB_GATEF + 4) cnt = 32;
         mbar_init(&bars[b], cnt);
       }
     }
@@ -836,28 +857,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // =====================================================================
-    // PREP prank = blockIdx.x - S: items k = 0, 1, ... of this CTA in order;
-    // item k uses tile set, TMEM buffer, Aqk buffer and gate block k & 1.
+    // PREP prank = blockIdx.x - S: items k = 0, 1, ... of this CTA in order.
+    // Item k: group g = k & 1 (warps 4g .. 4g+3), kg = k >> 1 its index in the
+    // group, tile set k % 3, P1 TMEM buffer and gate block kg & 1 of group g.
     // =====================================================================
     const int prank = int(blockIdx.x) - p.S;
     if (warp == 8) {
-      // ---------------- loader: the K, Q, V tiles (TMA, lane 0) and the gate
-      // factors (whole warp) of item k, once item k - 2 has been stored
+      // ---------------- loader: item k's K, Q, V tiles (TMA, lane 0) once set
+      // k % 3 is free (item k - 3 stored), and its gate factors (whole warp)
       PrepIter it;
       pi_start(it, p, sJ, iend, prank);
       int last_k = -1;
       bool ok = true;
       while (it.ok && ok) {
-        const int k = it.k, b = k & 1;
-        ok = k < 2 || mbar_wait(&bars[PB_STORED + b], ((k >> 1) & 1) ^ 1, abort_flag, err, 1u);
+        const int k = it.k, t = k % 3, g = k & 1, gb = (k >> 1) & 1;
+        ok = k < 3 || mbar_wait(&bars[PB_STORED + t], ((k / 3) & 1) ^ 1, abort_flag, err, 1u);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
         }
         if (lane == 0) {
-          uint64_t* fb = &bars[PB_KQVF + b];
+          uint64_t* fb = &bars[PB_KQVF + t];
           mbar_arrive_expect_tx(fb, uint32_t(nbox) * 3 * 8192);
-          uint8_t* set = smem + b * P_SET;
+          uint8_t* set = smem + t * P_SET;
           const int hk = it.h / vpg;
           for (int b2 = 0; b2 < nbox; ++b2) {
             tma_load_3d(set + P_KQ + b2 * 16384, &tm_k, fb, b2 * 64, hk, it.t0);
@@ -866,8 +888,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           last_k = k;
         }
-        // Gates of this item (padded rows: g = beta = 0); lane l owns rows 2l, 2l+1.
-        float* gt = reinterpret_cast<float*>(smem + P_GATE + b * PG_BYTES);
+        // Gates of this item (padded rows: g = beta = 0); lane l owns rows 2l,
+        // 2l+1.  The block was last read by the store of item k - 4.
+        float* gt = reinterpret_cast<float*>(smem + P_GRP + g * P_GS + GA_GT + gb * PG_BYTES);
         {
           const int r0 = 2 * lane;
           const float* gsrc = p.g + size_t(it.t0) * p.gb_stride + it.h;
@@ -909,7 +932,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             gt[PG_E2 + e2] = (sx < 16 * bb) ? __expf(gt[PG_G + 16 * bb] - gt[PG_G + sx]) : 0.f;
           }
         }
-        mbar_arrive(&bars[PB_GATEF + b]);  // release: this lane's gate writes
+        mbar_arrive(&bars[PB_GATEF + 2 * g + gb]);  // release: this lane's gate writes
         pi_next(it, p, sJ, iend);
       }
       if (!ok) {
@@ -917,78 +940,99 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicExch(const_cast<uint32_t*>(gabort), 1u);
       }
       if (lane == 0)  // nothing may still be landing in shared memory at exit
-        for (int k = last_k - 1; k <= last_k; ++k)
-          if (k >= 0) mbar_wait(&bars[PB_KQVF + (k & 1)], (k >> 1) & 1, nullptr, err, 32u);
+        for (int k = last_k - 2; k <= last_k; ++k)
+          if (k >= 0) mbar_wait(&bars[PB_KQVF + k % 3], (k / 3) & 1, nullptr, err, 32u);
       __syncwarp();
     } else if (warp == 9) {
-      // ---------------- MMA issue, in the order the worker needs them:
-      // P1 of item 0, then per item k: W/U of item k (once T is ready) and
-      // P1 of item k + 1 (its tiles were prefetched).  Every wait blocks in
-      // mbarrier.try_wait, so this warp takes no issue slots while idle.
+      // ---------------- MMA issue for both groups, whichever is ready: P1 of
+      // items in order (tiles landed, the group's P1 buffer read back), W/U of
+      // each group's next item once its T is ready
       if (elect_one()) {
         const uint32_t id_p1 = make_idesc_bf16(128, 64, 0, 0);
         const uint32_t id_wu = make_idesc_bf16(128, 64, 1, 0);
-        auto issue_p1 = [&](int kp) -> bool {
-          const int b = kp & 1;
-          if (!mbar_wait(&bars[PB_KQVF + b], (kp >> 1) & 1, abort_flag, err, 2u)) return false;
-          if (kp >= 2 && !mbar_wait(&bars[PB_P1FREE + b], ((kp >> 1) & 1) ^ 1, abort_flag, err, 2u))
-            return false;
-          tc_fence_after();
-          const uint32_t g = sbase + b * P_SET;
-          const uint32_t tm = tmem + PT_WG * b;
-          for (int kk = 0; kk < ksteps_d; ++kk) {
-            const uint32_t a = g + P_KQ + (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16_ss(tm + PT_P1, make_sdesc_sw128(a, 16, 1024), make_sdesc_sw128(a, 16, 1024),
-                        id_p1, kk > 0);
+        PrepIter itp;
+        pi_start(itp, p, sJ, iend, prank);
+        int kp = 0;                // next item for P1
+        int kw[2] = {0, 0};        // next in-group index for W/U
+        long long last = clock64();
+        while (true) {
+          bool prog = false;
+          if (itp.ok) {
+            const int t = kp % 3, g = kp & 1, kg = kp >> 1, pb = kg & 1;
+            if (mbar_test_wait(&bars[PB_KQVF + t], (kp / 3) & 1) &&
+                (kg < 2 || mbar_test_wait(&bars[PB_P1FREE + 2 * g + pb], ((kg >> 1) & 1) ^ 1))) {
+              tc_fence_after();
+              const uint32_t set = sbase + t * P_SET;
+              const uint32_t tm = tmem + PT_WG * g + 64u * pb;
+              for (int kk = 0; kk < ksteps_d; ++kk) {
+                const uint32_t a = set + P_KQ + (kk >> 2) * 16384 + (kk & 3) * 32;
+                mma_bf16_ss(tm, make_sdesc_sw128(a, 16, 1024), make_sdesc_sw128(a, 16, 1024), id_p1,
+                            kk > 0);
+              }
+              mma_commit(&bars[PB_P1F + 2 * g + pb]);
+              ++kp;
+              pi_next(itp, p, sJ, iend);
+              prog = true;
+            }
           }
-          mma_commit(&bars[PB_P1F + b]);
-          return true;
-        };
-        PrepIter it;
-        pi_start(it, p, sJ, iend, prank);
-        bool ok = !it.ok || issue_p1(0);
-        while (it.ok && ok) {
-          const int kw = it.k, b = kw & 1;
-          ok = mbar_wait(&bars[PB_TREADY], kw & 1, abort_flag, err, 2u);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t g = sbase + b * P_SET;
-          const uint32_t tm = tmem + PT_WG * b;
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tm + PT_W, make_sdesc_sw128(g + P_KQ + kk * 2048, 16384, 1024),
-                        make_sdesc_sw128(sbase + P_T1B + kk * 32, 16, 1024), id_wu, kk > 0);
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tm + PT_U, make_sdesc_sw128(g + P_V + kk * 2048, 8192, 1024),
-                        make_sdesc_sw128(sbase + P_T2B + kk * 32, 16, 1024), id_wu, kk > 0);
-          mma_commit(&bars[PB_WUF + b]);
-          pi_next(it, p, sJ, iend);
-          if (it.ok) ok = issue_p1(it.k);
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            const int kwg = kw[g], k = 2 * kwg + g;
+            if (k < kp && mbar_test_wait(&bars[PB_TREADY + g], kwg & 1)) {
+              tc_fence_after();
+              const uint32_t set = sbase + (k % 3) * P_SET;
+              const uint32_t tm = tmem + PT_WG * g;
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tm + PT_W, make_sdesc_sw128(set + P_KQ + kk * 2048, 16384, 1024),
+                            make_sdesc_sw128(set + P_T1B + kk * 32, 16, 1024), id_wu, kk > 0);
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tm + PT_U, make_sdesc_sw128(set + P_V + kk * 2048, 8192, 1024),
+                            make_sdesc_sw128(set + P_T2B + kk * 32, 16, 1024), id_wu, kk > 0);
+              mma_commit(&bars[PB_WUF + g]);
+              ++kw[g];
+              prog = true;
+            }
+          }
+          if ((!itp.ok && 2 * kw[0] >= kp && 2 * kw[1] + 1 >= kp) || *abort_flag) break;
+          if (prog) {
+            last = clock64();
+          } else {
+            if (clock64() - last > kSpinLimitCycles) {
+              *abort_flag = 1;
+              atomicExch(const_cast<uint32_t*>(gabort), 1u);
+              atomicOr(err, 2u);
+              break;
+            }
+            __nanosleep(32);
+          }
         }
         mma_commit(&bars[PB_DRAIN]);
         mbar_wait(&bars[PB_DRAIN], 0, nullptr, err, 8u);
       }
       __syncwarp();
     } else if (warp == 10) {
-      // ---------------- store: each staged item to its spine's ring entry
+      // ---------------- store: each staged item to its spine's ring entry, in
+      // item order
       if (lane == 0) {
         PrepIter it;
         pi_start(it, p, sJ, iend, prank);
         bool ok = true;
         while (it.ok && ok) {
-          const int k = it.k, b = k & 1;
+          const int k = it.k, t = k % 3, g = k & 1, kg = k >> 1;
           const int e = it.j % kRing;
-          ok = mbar_wait(&bars[PB_STAGED], k & 1, abort_flag, err, 4u);
+          ok = mbar_wait(&bars[PB_STAGED + g], kg & 1, abort_flag, err, 4u);
           if (ok && it.j >= kRing)  // entry e is free once the spine copied item j - kRing
             ok = poll_geq(free_flag(p, it.s, e), uint32_t(it.j - kRing + 1), gabort, err, 4u);
           if (!ok) break;
           fence_proxy_async_global();
           uint8_t* dst = ring_entry(p, it.s, e);
-          bulk_store_s2g(dst + G_W, smem + b * P_SET, 32768);
-          bulk_store_s2g(dst + G_AQK, smem + P_AQK + b * 8192, 8192);
-          bulk_store_s2g(dst + G_GATE, smem + P_GATE + b * PG_BYTES + PG_EG * 4, G_GATE_BYTES);
+          const uint8_t* ga = smem + P_GRP + g * P_GS;
+          bulk_store_s2g(dst + G_W, smem + t * P_SET, 32768);
+          bulk_store_s2g(dst + G_AQK, ga + GA_AQK, 8192);
+          bulk_store_s2g(dst + G_GATE, ga + GA_GT + (kg & 1) * PG_BYTES + PG_EG * 4, G_GATE_BYTES);
           tma_store_commit();
           tma_store_wait_read<0>();
-          mbar_arrive(&bars[PB_STORED + b]);
+          mbar_arrive(&bars[PB_STORED + t]);
           tma_store_wait_all<0>();
           fence_proxy_async_global();
           st_release_gpu(ready_flag(p, it.s, e), uint32_t(it.j + 1));
@@ -1001,44 +1045,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     } else if (warp < 8) {
-      // ---------------- worker: 256 threads, one item at a time.  Warp w
-      // reads TMEM lane quadrant q = w & 3 and column half hf = w >> 2.
-      const int q = warp & 3, hf = warp >> 2;
-      const int pt = tid;  // 0..255
-      const uint32_t lane_off = uint32_t(q * 32) << 16;
-      float* Af = reinterpret_cast<float*>(smem + P_AF);
-      float* Tf = reinterpret_cast<float*>(smem + P_TF);
-      float* Xs = reinterpret_cast<float*>(smem + P_XS);
+      // ---------------- groups: 128 threads each, items k = g, g + 2, ...
+      const int g = warp >> 2;
+      const int pt = tid & 127;
+      const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+      uint8_t* ga = smem + P_GRP + g * P_GS;
+      float* M = reinterpret_cast<float*>(ga + GA_AF);
+      float* Xs = reinterpret_cast<float*>(ga + GA_XS);
+      const int gbar = 1 + 3 * g;  // this group's named barriers: gbar (all), gbar+1, gbar+2
       PrepIter it;
       pi_start(it, p, sJ, iend, prank);
+      pi_align(it, p, sJ, iend, g);
       while (it.ok) {
-        const int k = it.k, b = k & 1;
-        const float* gt = reinterpret_cast<const float*>(smem + P_GATE + b * PG_BYTES);
-        const uint32_t tm = tmem + PT_WG * b;
-        // gates written, P1 = [K;Q] K^T done (its tiles landed after item k - 2
-        // was stored, so Aqk buffer b is free as well)
-        const bool ready = mbar_wait(&bars[PB_GATEF + b], (k >> 1) & 1, abort_flag, err, 4u) &&
-                           mbar_wait(&bars[PB_P1F + b], (k >> 1) & 1, abort_flag, err, 4u);
-        if (!named_all(1, 256, ready)) break;
+        const int k = it.k, kg = k >> 1, t = k % 3, pb = kg & 1;
+        uint8_t* set = smem + t * P_SET;
+        const float* gt = reinterpret_cast<const float*>(ga + GA_GT + pb * PG_BYTES);
+        const uint32_t tm = tmem + PT_WG * g;
+        // gates written, P1 done; the group's Aqk buffer was read by the store
+        // of its previous item k - 2
+        const bool ready =
+            mbar_wait(&bars[PB_GATEF + 2 * g + pb], (kg >> 1) & 1, abort_flag, err, 4u) &&
+            mbar_wait(&bars[PB_P1F + 2 * g + pb], (kg >> 1) & 1, abort_flag, err, 4u) &&
+            (k < 2 || mbar_wait(&bars[PB_STORED + (k - 2) % 3], ((k - 2) / 3) & 1, abort_flag, err, 4u));
+        if (!named_all(gbar, 128, ready)) break;
         tc_fence_after();
-        // ---- P1 row rr (TMEM lane): K K^T (rr < 64) or Q K^T (rr >= 64),
-        // columns 32 hf .. + 31, times e^{G_r - G_s} (s <= r): two factors <= 1
-        // for the blocks of s before r's 16-row block, a direct exponential
-        // inside it.
+        // ---- P1 row pt: K K^T (pt < 64) or Q K^T (pt >= 64), times e^{G_r - G_s}
+        // (s <= r): two factors <= 1 for the blocks of s before r's 16-row
+        // block, a direct exponential inside it.
         {
-          const int rr = 32 * q + lane, r = rr & 63, rb = r >> 4;
+          const int r = pt & 63, rb = r >> 4;
           const float Gr = gt[PG_G + r];
           const float e1 = gt[PG_E1 + r];
           const float br = gt[PG_BET + r];
           const float* e2 = gt + PG_E2 + 64 * rb;
-          float v[32];
-          tmem_ld32(tm + lane_off + PT_P1 + 32u * hf, v);
+          float v[64];
+          tmem_ld32(tm + lane_off + 64u * pb, *reinterpret_cast<float(*)[32]>(v));
+          tmem_ld32(tm + lane_off + 64u * pb + 32, *reinterpret_cast<float(*)[32]>(v + 32));
           tmem_ld_wait();
           tc_fence_before();
-          mbar_arrive(&bars[PB_P1FREE + b]);
+          mbar_arrive(&bars[PB_P1FREE + 2 * g + pb]);
 #pragma unroll
-          for (int sbl = 0; sbl < 2; ++sbl) {
-            const int sb = 2 * hf + sbl;
+          for (int sb = 0; sb < 4; ++sb) {
             float f[16];
             if (sb < rb) {
 #pragma unroll
@@ -1063,45 +1110,43 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int jj = 0; jj < 16; ++jj) f[jj] = 0.f;
             }
-            const float* vv = v + 16 * sbl;
-            if (rr < 64) {  // A[r][s] = beta_r e^{G_r-G_s} k_r.k_s, s < r
+            if (pt < 64) {  // A[r][s] = beta_r e^{G_r-G_s} k_r.k_s, s < r
 #pragma unroll
               for (int jj = 0; jj < 16; jj += 4) {
                 const int s2 = 16 * sb + jj;
-                *reinterpret_cast<float4*>(Af + r * kAS + s2) = make_float4(
-                    s2 + 0 < r ? br * f[jj] * vv[jj] : 0.f,
-                    s2 + 1 < r ? br * f[jj + 1] * vv[jj + 1] : 0.f,
-                    s2 + 2 < r ? br * f[jj + 2] * vv[jj + 2] : 0.f,
-                    s2 + 3 < r ? br * f[jj + 3] * vv[jj + 3] : 0.f);
+                *reinterpret_cast<float4*>(M + r * kAS + s2) = make_float4(
+                    s2 + 0 < r ? br * f[jj] * v[s2] : 0.f,
+                    s2 + 1 < r ? br * f[jj + 1] * v[s2 + 1] : 0.f,
+                    s2 + 2 < r ? br * f[jj + 2] * v[s2 + 2] : 0.f,
+                    s2 + 3 < r ? br * f[jj + 3] * v[s2 + 3] : 0.f);
               }
             } else {  // Aqk[r][s] = scale e^{G_r-G_s} q_r.k_s, s <= r  (bf16, swizzled)
               const float sc = p.scale;
-              uint8_t* aq = smem + P_AQK + b * 8192;
 #pragma unroll
               for (int hc = 0; hc < 2; ++hc) {
-                const int o = 8 * hc;
-                *reinterpret_cast<uint4*>(aq + sw128_offset(r, (2 * sb + hc) * 16)) = make_uint4(
-                    pack_bf16x2(sc * f[o] * vv[o], sc * f[o + 1] * vv[o + 1]),
-                    pack_bf16x2(sc * f[o + 2] * vv[o + 2], sc * f[o + 3] * vv[o + 3]),
-                    pack_bf16x2(sc * f[o + 4] * vv[o + 4], sc * f[o + 5] * vv[o + 5]),
-                    pack_bf16x2(sc * f[o + 6] * vv[o + 6], sc * f[o + 7] * vv[o + 7]));
+                const int s2 = 16 * sb + 8 * hc, o = 8 * hc;
+                *reinterpret_cast<uint4*>(ga + GA_AQK + sw128_offset(r, (2 * sb + hc) * 16)) =
+                    make_uint4(pack_bf16x2(sc * f[o] * v[s2], sc * f[o + 1] * v[s2 + 1]),
+                               pack_bf16x2(sc * f[o + 2] * v[s2 + 2], sc * f[o + 3] * v[s2 + 3]),
+                               pack_bf16x2(sc * f[o + 4] * v[s2 + 4], sc * f[o + 5] * v[s2 + 5]),
+                               pack_bf16x2(sc * f[o + 6] * v[s2 + 6], sc * f[o + 7] * v[s2 + 7]));
               }
             }
           }
         }
-        named_sync(1, 256);
-        // ---- T = (I + A)^{-1}
-        invert_unit_lower64(Af, Tf, Xs, pt, 1, 2);
-        // ---- T1 = T diag(beta e^G) (rows of task < 64), T2 = T diag(beta)
+        named_sync(gbar, 128);
+        // ---- T = (I + A)^{-1}, in place
+        invert_unit_lower64(M, Xs, pt, gbar);
+        // ---- T1 = T diag(beta e^G) (rows pt < 64), T2 = T diag(beta) (rows pt >= 64),
+        // into the item's Q boxes (Q was last read by P1)
         {
-          const int task = pt & 127, r = task & 63, half = pt >> 7;
-          const float* scv = gt + (task < 64 ? PG_BEG : PG_BET);
-          uint8_t* tile = smem + (task < 64 ? P_T1B : P_T2B);
-#pragma unroll
-          for (int c2 = 0; c2 < 4; ++c2) {
-            const int cc = 4 * half + c2;
-            const float4 ta = *reinterpret_cast<const float4*>(Tf + r * kAS + 8 * cc);
-            const float4 tb2 = *reinterpret_cast<const float4*>(Tf + r * kAS + 8 * cc + 4);
+          const int r = pt & 63;
+          const float* scv = gt + (pt < 64 ? PG_BEG : PG_BET);
+          uint8_t* tile = set + (pt < 64 ? P_T1B : P_T2B);
+#pragma unroll 1
+          for (int cc = 0; cc < 8; ++cc) {
+            const float4 ta = *reinterpret_cast<const float4*>(M + r * kAS + 8 * cc);
+            const float4 tb2 = *reinterpret_cast<const float4*>(M + r * kAS + 8 * cc + 4);
             const float4 sa = *reinterpret_cast<const float4*>(scv + 8 * cc);
             const float4 sb2 = *reinterpret_cast<const float4*>(scv + 8 * cc + 4);
             const int s0 = 8 * cc;
@@ -1113,36 +1158,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         fence_proxy_async_smem();
-        mbar_arrive(&bars[PB_TREADY]);
-        // ---- W (row-major), U^T into tile set b (its K, Q, V are no longer read)
-        if (!named_all(1, 256, mbar_wait(&bars[PB_WUF + b], (k >> 1) & 1, abort_flag, err, 4u))) break;
+        mbar_arrive(&bars[PB_TREADY + g]);
+        // ---- W (row-major), U^T into [0, 32 KB) of the item's set
+        if (!named_all(gbar, 128, mbar_wait(&bars[PB_WUF + g], kg & 1, abort_flag, err, 4u))) break;
         tc_fence_after();
         {
-          const int pq = 32 * q + lane;  // d_k (W) / d_v (U) index = TMEM lane
-          uint8_t* set = smem + b * P_SET;
-          float wv[32], uv[32];
-          tmem_ld32(tm + lane_off + PT_W + 32u * hf, wv);
-          tmem_ld32(tm + lane_off + PT_U + 32u * hf, uv);
-          tmem_ld_wait();
+          uint8_t* wcol = set + G_W + uint32_t(pt >> 6) * 8192;
+          const uint32_t wbyte = uint32_t(pt & 63) * 2;
+#pragma unroll 1
+          for (int hf = 0; hf < 2; ++hf) {
+            float wv[32], uv[32];
+            tmem_ld32(tm + lane_off + PT_W + 32u * hf, wv);
+            tmem_ld32(tm + lane_off + PT_U + 32u * hf, uv);
+            tmem_ld_wait();
 #pragma unroll
-          for (int hc = 0; hc < 4; ++hc) {
-            const uint32_t off = sw128_offset(pq, (4 * hf + hc) * 16);
-            *reinterpret_cast<uint4*>(set + G_U + off) = make_uint4(
-                pack_bf16x2(uv[8 * hc], uv[8 * hc + 1]), pack_bf16x2(uv[8 * hc + 2], uv[8 * hc + 3]),
-                pack_bf16x2(uv[8 * hc + 4], uv[8 * hc + 5]), pack_bf16x2(uv[8 * hc + 6], uv[8 * hc + 7]));
+            for (int hc = 0; hc < 4; ++hc) {
+              const uint32_t off = sw128_offset(pt, (4 * hf + hc) * 16);
+              *reinterpret_cast<uint4*>(set + G_U + off) =
+                  make_uint4(pack_bf16x2(uv[8 * hc], uv[8 * hc + 1]),
+                             pack_bf16x2(uv[8 * hc + 2], uv[8 * hc + 3]),
+                             pack_bf16x2(uv[8 * hc + 4], uv[8 * hc + 5]),
+                             pack_bf16x2(uv[8 * hc + 6], uv[8 * hc + 7]));
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              *reinterpret_cast<uint16_t*>(wcol + sw128_offset(uint32_t(32 * hf + i), wbyte)) =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(wv[i]));
           }
-          uint8_t* wcol = set + G_W + (pq >> 6) * 8192;
-          const uint32_t wbyte = uint32_t(pq & 63) * 2;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            *reinterpret_cast<uint16_t*>(wcol + sw128_offset(uint32_t(32 * hf + i), wbyte)) =
-                __bfloat16_as_ushort(__float2bfloat16_rn(wv[i]));
         }
         tc_fence_before();
         fence_proxy_async_smem();
-        named_sync(1, 256);
-        if (pt == 0) mbar_arrive(&bars[PB_STAGED]);
+        named_sync(gbar, 128);
+        if (pt == 0) mbar_arrive(&bars[PB_STAGED + g]);
         pi_next(it, p, sJ, iend);
+        pi_align(it, p, sJ, iend, g);
       }
     }
   }
