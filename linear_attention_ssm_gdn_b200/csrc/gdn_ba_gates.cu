@@ -12,12 +12,13 @@
 // (split-K, so that the 4576 x 5120 activation streams through ~all SMs).
 // TMA streams 128x64 X tiles and Nx64 W tiles (128-byte swizzle) through a
 // STAGES-deep mbarrier ring; one thread issues tcgen05.mma (M=128, N=N_pad,
-// K=16 steps) into a TMEM accumulator.  Each CTA then stages its f32 partial
-// in its own (now idle) pipeline shared memory; after a cluster barrier, rank
-// r reduces rows r*128/KS .. of all KS partials in rank order (distributed
-// shared memory reads, deterministic) and applies the gate epilogue in f32:
+// K=16 steps) into a TMEM accumulator.  Rank r owns rows r*128/KS .. of the
+// tile: every CTA pushes each of its partial rows into the owner's receive
+// buffer with distributed-shared-memory stores (no dependent remote loads),
+// one cluster barrier publishes them, and the owner sums the KS partials of
+// its rows in rank order (deterministic) from its own shared memory and
+// applies the gate epilogue in f32, one output row at a time (coalesced):
 //   beta = sigmoid(ba),  gate = -exp(A_log) * softplus(ba + dt_bias).
-// A second cluster barrier keeps every partial alive until it has been read.
 // Every activation byte is read from HBM once; W (N*K*2 bytes) stays in L2.
 // No multicast: each CTA loads its own tiles.
 #include <cuda.h>
@@ -35,7 +36,7 @@ constexpr int kBaBM = 128;       // tokens per CTA (MMA M)
 constexpr int kBaBK = 64;        // K per TMA box (one 128-byte swizzle row)
 constexpr int kBaNB = 2;         // boxes per pipeline stage: 2 x 128 contiguous bytes per row
 constexpr int kBaMaxKS = 2;      // largest K split (CTAs per cluster): measured best
-constexpr int kBaThreads = 128;  // 4 warps: TMA (warp 0), MMA (warp 1), all: epilogue
+constexpr int kBaThreads = 512;  // TMA (warp 0), MMA (warp 1); all 16 warps: epilogue
 
 struct BaParams {
   const float* a_log;
@@ -43,23 +44,21 @@ struct BaParams {
   float* out;
   int gate_stride, M, N, K, nv, vpg;
   int n_pad, stages, tmem_cols;
-  int ks;  // CTAs per cluster (K split)
+  int ks;        // CTAs per cluster (K split)
+  int overlay;   // 1: the receive buffer reuses the pipeline's shared memory
+  uint32_t recv_off, const_off, bar_off;  // shared-memory layout (bytes)
 };
 
-__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
+constexpr uint32_t kBaMaxSmem = 232448;  // dynamic shared memory per CTA
 
-// Hardware cluster barrier; every thread of every CTA of the cluster reaches
-// each call exactly once (no early exits in this kernel).
-__device__ __forceinline__ void cluster_barrier() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 __global__ void __launch_bounds__(kBaThreads, 1)
@@ -74,7 +73,12 @@ __global__ void __launch_bounds__(kBaThreads, 1)
   const uint32_t b_bytes = kBaNB * b_box;
   uint8_t* a_s = smem;
   uint8_t* b_s = a_s + stages * a_bytes;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(b_s + stages * b_bytes);
+  float* recv = reinterpret_cast<float*>(smem + p.recv_off);     // [KS][128 / KS][n_pad + 4]
+  float* coef = reinterpret_cast<float*>(smem + p.const_off);    // -exp(A_log) [nv]
+  float* dtb = coef + p.nv;                                       // dt_bias [nv]
+  // output column j -> projection column n (bits 0-15) | v-head (16-30) | gate (31)
+  uint32_t* colmap = reinterpret_cast<uint32_t*>(dtb + p.nv);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + p.bar_off);
   uint64_t* empty_bar = full_bar + stages;
   uint64_t* done_bar = empty_bar + stages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
@@ -90,6 +94,18 @@ __global__ void __launch_bounds__(kBaThreads, 1)
   const int kb_begin = kb_all * rank / p.ks, kb_end = kb_all * (rank + 1) / p.ks;
   const int nbox = kb_end - kb_begin;
   const int num_kb = (nbox + kBaNB - 1) / kBaNB;  // pipeline stages
+  // the first `stages` stages find their buffers free: issued during setup
+  const int prologue = min(stages, num_kb);
+  auto issue_stage = [&](int kb) {
+    const int s = kb % stages;
+    const int nb = min(kBaNB, nbox - kb * kBaNB);
+    mbar_arrive_expect_tx(&full_bar[s], uint32_t(nb) * (a_box + b_box));
+    for (int x = 0; x < nb; ++x) {
+      const int kx = (kb_begin + kb * kBaNB + x) * kBaBK;
+      tma_load_2d(a_s + s * a_bytes + x * a_box, &tmap_x, &full_bar[s], kx, m0);
+      tma_load_2d(b_s + s * b_bytes + x * b_box, &tmap_w, &full_bar[s], kx, 0);
+    }
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -99,27 +115,35 @@ __global__ void __launch_bounds__(kBaThreads, 1)
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    tma_prefetch_desc(&tmap_x);
-    tma_prefetch_desc(&tmap_w);
+    for (int kb = 0; kb < prologue; ++kb) issue_stage(kb);
   }
   if (warp == 0) tmem_alloc(tmem_slot, p.tmem_cols);
+  for (int i = int(threadIdx.x); i < p.nv; i += kBaThreads) {
+    coef[i] = -__expf(__ldg(&p.a_log[i]));
+    dtb[i] = __ldg(&p.dt_bias[i]);
+  }
+  // Column j < nv is the gate of v-head j, column nv + h the beta of v-head h;
+  // their projection outputs sit at n = (h / vpg) * 2 vpg + (vpg for the gate) + h % vpg.
+  for (int j = int(threadIdx.x); j < 2 * p.nv; j += kBaThreads) {
+    const bool is_gate = j < p.nv;
+    const int vh = is_gate ? j : j - p.nv;
+    const int n = (vh / p.vpg) * 2 * p.vpg + (is_gate ? p.vpg : 0) + vh % p.vpg;
+    colmap[j] = uint32_t(n) | (uint32_t(vh) << 16) | (is_gate ? 0x80000000u : 0u);
+  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // With a separate receive buffer, the cluster barrier that publishes the
+  // partials only needs every CTA of the cluster to have started: arrive now.
+  if (!p.overlay) cluster_arrive_relaxed();
 
   if (warp == 0) {
-    if (elect_one()) {  // TMA producer
-      for (int kb = 0; kb < num_kb; ++kb) {
+    if (elect_one()) {  // TMA producer (the stages after the prologue)
+      for (int kb = prologue; kb < num_kb; ++kb) {
         const int s = kb % stages;
         const uint32_t ph = (kb / stages) & 1;
         if (!mbar_wait(&empty_bar[s], ph ^ 1, abort_flag, &g_err_ba_gates, 1u)) break;
-        const int nb = min(kBaNB, nbox - kb * kBaNB);
-        mbar_arrive_expect_tx(&full_bar[s], uint32_t(nb) * (a_box + b_box));
-        for (int x = 0; x < nb; ++x) {
-          const int kx = (kb_begin + kb * kBaNB + x) * kBaBK;
-          tma_load_2d(a_s + s * a_bytes + x * a_box, &tmap_x, &full_bar[s], kx, m0);
-          tma_load_2d(b_s + s * b_bytes + x * b_box, &tmap_w, &full_bar[s], kx, 0);
-        }
+        issue_stage(kb);
       }
     }
     __syncwarp();
@@ -150,70 +174,93 @@ __global__ void __launch_bounds__(kBaThreads, 1)
     __syncwarp();
   }
 
-  // Partial sums: warp w owns TMEM lanes 32w..32w+31 (tokens m0+32w+lane);
-  // each row goes to the partial buffer P[128][n_pad + 4] f32 that reuses the
-  // pipeline's shared memory (every MMA has completed once done_bar fired).
+  // Partial sums: warp w reads TMEM lanes 32 (w % 4) .. + 31 (tile row r =
+  // 32 (w % 4) + lane), column blocks of 16 from 16 (w / 4) in steps of 64.
+  // Row r belongs to rank r / (128 / KS); this CTA's copy of it goes to slot
+  // [my rank][r % (128 / KS)] of that rank's receive buffer.  When the buffer
+  // reuses pipeline memory, every CTA of the cluster must be done with its
+  // pipeline first (the barrier below is then a full one).
   const bool ok = num_kb == 0 || mbar_wait(done_bar, 0, abort_flag, &g_err_ba_gates, 4u);
   tc_fence_after();
+  if (p.overlay) cluster_arrive_release();
+  cluster_wait_acquire();  // every CTA of the cluster is running (and idle, overlaid)
   const int pstride = p.n_pad + 4;
-  float* part = reinterpret_cast<float*>(smem);
+  const int rows = kBaBM / p.ks;
   {
-    float* prow = part + size_t(warp * 32 + lane) * pstride;
-    for (int c = 0; c < p.n_pad; c += 16) {
+    const uint32_t lq = warp & 3u;
+    const int r = int(lq) * 32 + int(lane);
+    const int owner = r / rows;
+    const uint32_t dst = mapa_shared(
+        smem_u32(recv + size_t(rank * rows + (r - owner * rows)) * pstride), uint32_t(owner));
+    const bool live = ok && num_kb > 0;
+    for (int c = 16 * int(warp >> 2); c < p.n_pad; c += 16 * (kBaThreads / 128)) {
       float acc[16];
-      tmem_ld16(tmem + ((warp * 32u) << 16) + uint32_t(c), acc);
+      tmem_ld16(tmem + ((lq * 32u) << 16) + uint32_t(c), acc);
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4*>(prow + c + j) =
-            (ok && num_kb > 0) ? make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3])
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        st_cluster_v4(dst + uint32_t(c + j) * 4, live ? __float_as_uint(acc[j]) : 0u,
+                      live ? __float_as_uint(acc[j + 1]) : 0u,
+                      live ? __float_as_uint(acc[j + 2]) : 0u,
+                      live ? __float_as_uint(acc[j + 3]) : 0u);
     }
   }
   tc_fence_before();
-  cluster_barrier();  // every partial of the cluster is written
-  // Reduction + epilogue: this CTA's rows r0 .. r0 + rows - 1; thread t takes
-  // row r0 + t / tpr and a run of 4-column groups.
+  cluster_arrive_release();  // the pushes above, before the owners read them
+  cluster_wait_acquire();
+  // Reduction + epilogue over this rank's rows, flat over (row lr, output
+  // column j) so that consecutive threads store consecutive columns; (lr, j)
+  // advance by the fixed thread stride without divisions, kEpU elements per
+  // thread at a time so that their shared-memory reads overlap.
   {
-    const int rows = kBaBM / p.ks;
-    const int tpr = kBaThreads / rows;  // threads per row
-    const int r = rank * rows + int(threadIdx.x) / tpr;
-    const int m = m0 + r;
-    const int group_dim = 2 * p.vpg;
-    const uint32_t prow = smem_u32(part + size_t(r) * pstride);
-    float* row = p.out + size_t(m) * p.gate_stride;
-    for (int c = 4 * (int(threadIdx.x) % tpr); c < p.n_pad; c += 4 * tpr) {
-      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int q = 0; q < p.ks; ++q) {  // fixed order: deterministic
-        const float4 v = ld_cluster_f4(mapa_shared(prow + uint32_t(c) * 4, uint32_t(q)));
-        sum.x += v.x;
-        sum.y += v.y;
-        sum.z += v.z;
-        sum.w += v.w;
-      }
-      const float acc[4] = {sum.x, sum.y, sum.z, sum.w};
-      if (m < p.M && ok && !*abort_flag) {
+    constexpr int kEpU = 4;
+    const int w2 = 2 * p.nv, total = rows * w2;
+    const bool write = ok && !*abort_flag;
+    const int dl = kBaThreads / w2, dj = kBaThreads - dl * w2;
+    int lr = int(threadIdx.x) / w2, j = int(threadIdx.x) - lr * w2;
+    for (int i = int(threadIdx.x); i < total; i += kEpU * kBaThreads) {
+      int lrs[kEpU], js[kEpU];
+      bool live[kEpU];
+      uint32_t cm[kEpU];
+      float sum[kEpU];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int n = c + j;
-          if (n < p.N) {
-            const int within = n % group_dim, grp = n / group_dim;
-            const float ba = acc[j];
-            if (within < p.vpg) {
-              const int vh = grp * p.vpg + within;
-              row[p.nv + vh] = 1.0f / (1.0f + __expf(-ba));
-            } else {
-              const int vh = grp * p.vpg + (within - p.vpg);
-              const float z = ba + __ldg(&p.dt_bias[vh]);
-              const float sp = fmaxf(z, 0.0f) + log1pf(__expf(-fabsf(z)));
-              row[vh] = -__expf(__ldg(&p.a_log[vh])) * sp;
-            }
-          }
+      for (int u = 0; u < kEpU; ++u) {
+        lrs[u] = lr;
+        js[u] = j;
+        live[u] = write && i + u * kBaThreads < total && m0 + rank * rows + lr < p.M;
+        lr += dl;
+        j += dj;
+        if (j >= w2) {
+          j -= w2;
+          ++lr;
         }
+      }
+#pragma unroll
+      for (int u = 0; u < kEpU; ++u) cm[u] = live[u] ? colmap[js[u]] : 0u;
+#pragma unroll
+      for (int u = 0; u < kEpU; ++u) {
+        const float* col = recv + size_t(lrs[u]) * pstride + (cm[u] & 0xffffu);
+        float acc = 0.0f;
+        for (int q = 0; q < p.ks; ++q)  // fixed order: deterministic
+          acc += live[u] ? col[size_t(q * rows) * pstride] : 0.0f;
+        sum[u] = acc;
+      }
+#pragma unroll
+      for (int u = 0; u < kEpU; ++u) {
+        if (!live[u]) continue;
+        const int vh = int((cm[u] >> 16) & 0x7fffu);
+        float val;
+        if (cm[u] & 0x80000000u) {
+          const float z = sum[u] + dtb[vh];
+          const float sp = fmaxf(z, 0.0f) + log1pf(__expf(-fabsf(z)));
+          val = coef[vh] * sp;
+        } else {
+          val = __frcp_rn(1.0f + __expf(-sum[u]));
+        }
+        p.out[size_t(m0 + rank * rows + lrs[u]) * p.gate_stride + js[u]] = val;
       }
     }
   }
-  cluster_barrier();  // no CTA leaves while its partial may still be read
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, p.tmem_cols);
@@ -242,14 +289,25 @@ cudaError_t launch_ba_gates(const uint16_t* x, int k_stride, const uint16_t* w,
   p.vpg = vpg;
   p.n_pad = (N + 15) / 16 * 16;
   p.tmem_cols = pow2_at_least(p.n_pad);
-  const int stage_bytes = kBaNB * (kBaBM * 128 + p.n_pad * 128);
-  p.stages = (200 * 1024) / stage_bytes;
-  if (p.stages > 6) p.stages = 6;
-  if (p.stages < 2) p.stages = 2;
-  // The pipeline buffers double as the f32 partial [128][n_pad + 4] afterwards.
-  const size_t part_bytes = size_t(kBaBM) * (p.n_pad + 4) * 4;
-  if (size_t(p.stages) * stage_bytes < part_bytes) return cudaErrorInvalidValue;
-  const size_t smem = 1024 + size_t(p.stages) * stage_bytes + (2 * p.stages + 1) * 8 + 16;
+  // Layout: [stages][receive buffer, f32 [128][n_pad + 4]][constants][barriers].
+  // The receive buffer gets its own space when that still leaves two or more
+  // stages, and otherwise reuses the (then idle) pipeline memory.
+  const uint32_t stage_bytes = kBaNB * (kBaBM * 128 + uint32_t(p.n_pad) * 128);
+  const uint32_t recv_bytes = uint32_t(kBaBM) * (p.n_pad + 4) * 4;
+  const uint32_t const_bytes = uint32_t(4 * nv) * 4;
+  const uint32_t tail = const_bytes + 16 + (2 * 6 + 1) * 8 + 16;
+  int stages = int((kBaMaxSmem - 1024 - recv_bytes - tail) / stage_bytes);
+  p.overlay = stages < 2;
+  if (p.overlay) stages = int((kBaMaxSmem - 1024 - tail) / stage_bytes);
+  if (stages > 6) stages = 6;
+  if (stages < 2) return cudaErrorInvalidValue;
+  if (p.overlay && uint32_t(stages) * stage_bytes < recv_bytes) return cudaErrorInvalidValue;
+  p.stages = stages;
+  p.recv_off = p.overlay ? 0u : uint32_t(stages) * stage_bytes;
+  p.const_off = (p.overlay ? uint32_t(stages) * stage_bytes : p.recv_off + recv_bytes);
+  p.bar_off = (p.const_off + const_bytes + 15) / 16 * 16;
+  const size_t smem = 1024 + p.bar_off + (2 * stages + 1) * 8 + 16;
+  if (smem > kBaMaxSmem) return cudaErrorInvalidValue;
 
   CUtensorMap tx, tw;
   {
