@@ -288,29 +288,6 @@ __device__ __forceinline__ void st_row64_bf16(uint32_t tile, uint32_t row, const
 }
 
 // ---------------------------------------------------------------------------
-// Named (hardware) barriers among a fixed set of warps.  Used only
-// where every thread of the group is guaranteed to arrive (no early exits in
-// between); after a bounded wait that may fail, named_all() first agrees on
-// the outcome so that all threads leave together.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-__device__ __forceinline__ bool named_all(int id, int nthreads, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(uint32_t(v)), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
-
-// ---------------------------------------------------------------------------
 // T = (I + A)^{-1} in place: on entry M holds the strictly lower triangular
 // 64x64 A (f32, row stride kAS, zeros on and above the diagonal), on exit the
 // unit lower triangular T.  128 threads (4 warps), 16x16 blocks

@@ -49,133 +49,304 @@ __global__ void flag_clear_kernel(uint32_t* flag) {
   if (threadIdx.x == 0) *flag = 0u;
 }
 
-constexpr int kVThreads = 256;
+constexpr int kVThreads = 256;  // fold block; verify compute threads
 
-// grid = (H_v, batch); block = 256 threads = GROUPS row groups x QUADS column
-// quads.  Every thread issues all of its state loads (16 x 16 bytes at
-// d = 128) before it needs any of them, so a CTA waits for memory about once;
-// four CTAs per SM (64 registers) keep the loads of one CTA overlapping the
-// recurrence of another (measured: 55.6 us against 75.4 us at two per SM).
+// ---------------------------------------------------------------------------
+// Verify: one persistent CTA per SM walks the (sequence, v-head) items
+// blockIdx.x, blockIdx.x + gridDim.x, ...  Warp roles:
+//   warps 0-7 (256 threads)  compute: thread = (row group, column quad); the
+//       FMA phase reads its rows of the item's state from shared memory and
+//       accumulates a_r and b_r for its four columns; warps 0 .. D/32 - 1 then
+//       reduce the row groups and run the per-column 4-step recurrence.
+//   warp 8   copies: each item's state, as two contiguous halves (rows
+//       0 .. D/2 - 1 and D/2 .. D - 1), into a ring of shared-memory slots
+//       with cp.async.bulk, as far ahead as the ring allows.
+//   warps 9, 10  item descriptors (even / odd items): k and q transposed to
+//       4-row vectors, v, the dot products k_s.k_r and k_s.q_r, the cumulative
+//       gates and the decay factors, prepared while earlier items compute.
+// Warps 0-3 read the first half of the state, warps 4-7 the second.
+// ---------------------------------------------------------------------------
+constexpr int kVCompute = 256;
+constexpr int kVCopyWarp = 8;
+constexpr int kVBlock = kVCompute + 3 * 32;
+constexpr uint32_t kVRingBytes = 160 * 1024;
+
 template <int D>
-__global__ void __launch_bounds__(kVThreads, 4) verify_kernel(
+struct VerifyDesc {
+  float4 kq4[D];        // (k_0[i], k_1[i], k_2[i], k_3[i])
+  float4 qq4[D];        // (q_0[i], .., q_3[i])
+  float vv[kRows][D];   // v rows
+  float eG[kRows];      // e^{G_r}
+  float cK[kRows][kRows];  // [s][r] = e^{G_r - G_s} k_s.k_r   (s < r)
+  float cQ[kRows][kRows];  // [s][r] = e^{G_r - G_s} k_s.q_r   (s <= r)
+  float bt[kRows];      // beta_r
+  float Gc[kRows];      // G_r (stashed for the fold)
+  int pad;              // 1: the sequence has no state (zero outputs only)
+  int pad_[3];
+};
+
+template <int D>
+struct VerifySmem {
+  static constexpr int QUADS = D / 4;
+  static constexpr int GROUPS = kVCompute / QUADS;  // 8 (D=128) / 16 (D=64)
+  static constexpr int RPG = D / GROUPS;            // rows per group: 16 / 4
+  static constexpr uint32_t HALF = uint32_t(D) * D * 4 / 2;
+  static constexpr int NSLOT = int(kVRingBytes / HALF);
+  static constexpr uint32_t PART = 0 + kVRingBytes;  // float4 [GROUPS][2*kRows][QUADS]
+  static constexpr uint32_t DESC = PART + uint32_t(GROUPS) * 2 * kRows * QUADS * 16;
+  static constexpr uint32_t BARS = DESC + 2 * uint32_t(sizeof(VerifyDesc<D>));
+  // full[NSLOT], empty[NSLOT], dfull[2], dempty[2], abort word
+  static constexpr uint32_t TOTAL = BARS + (2 * NSLOT + 4) * 8 + 16;
+};
+static_assert(VerifySmem<128>::TOTAL + 128 <= 232448, "verify shared memory");
+static_assert(VerifySmem<64>::TOTAL + 128 <= 232448, "verify shared memory");
+
+template <int D>
+__global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
     float* const* __restrict__ h_table, const uint16_t* __restrict__ q,
     const uint16_t* __restrict__ k, int qk_stride, const uint16_t* __restrict__ v, int v_stride,
     const float* __restrict__ g, const float* __restrict__ beta, int gb_stride,
-    uint16_t* __restrict__ o, float* __restrict__ stash, int stash_seq_floats, int H_k, int H_v,
-    float scale, uint32_t* flag) {
-  constexpr int QUADS = D / 4;              // column quads per row
-  constexpr int GROUPS = kVThreads / QUADS;  // row groups (8 for D=128, 16 for D=64)
-  constexpr int RPG = D / GROUPS;            // rows per group (16 resp. 4)
-  __shared__ float ks[kRows][D], qs[kRows][D];
-  __shared__ float4 part[GROUPS][2 * kRows][QUADS];  // partial a_r, b_r per row group
-  __shared__ float kk[kRows][kRows], kq[kRows][kRows], G[kRows], bt[kRows];
+    uint16_t* __restrict__ o, float* __restrict__ stash, int stash_seq_floats, int batch, int H_k,
+    int H_v, float scale, uint32_t* flag) {
+  using L = VerifySmem<D>;
+  constexpr int QUADS = L::QUADS, GROUPS = L::GROUPS, RPG = L::RPG, NSLOT = L::NSLOT;
+  constexpr int EPL = D / 32;  // elements of a row per lane (descriptor warps)
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                             ~uintptr_t(127));
+  float4* part = reinterpret_cast<float4*>(smem + L::PART);
+  VerifyDesc<D>* desc = reinterpret_cast<VerifyDesc<D>*>(smem + L::DESC);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BARS);
+  uint64_t* empty = full + NSLOT;
+  uint64_t* dfull = empty + NSLOT;
+  uint64_t* dempty = dfull + 2;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(dempty + 2);
 
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int hk = h / (H_v / H_k);
-  const int tid = threadIdx.x;
-  const int quad = tid % QUADS, grp = tid / QUADS;
-  const float* H0 = h_table[b];
-  if (b == 0 && h == 0 && tid == 0) atomicOr(flag, kFlagEngaged);
-
-  const size_t row0 = size_t(b) * kRows;
-  if (H0 == nullptr) {  // padding sequence: zero outputs, nothing else
-    for (int idx = tid; idx < kRows * D; idx += kVThreads) {
-      const int r = idx / D, j = idx % D;
-      o[((row0 + r) * H_v + h) * D + j] = 0;
-    }
-    return;
-  }
-  // This thread's rows of the state, all loads in flight at once.
-  const float4* H4 = reinterpret_cast<const float4*>(H0 + size_t(h) * D * D);
-  float4 hv[RPG];
-#pragma unroll
-  for (int ii = 0; ii < RPG; ++ii) hv[ii] = __ldg(&H4[(grp * RPG + ii) * QUADS + quad]);
-  // v for the recurrence (thread j < D owns column j)
-  float vr[kRows];
-#pragma unroll
-  for (int r = 0; r < kRows; ++r)
-    vr[r] = tid < D ? bf16_at(v + (row0 + r) * v_stride + size_t(h) * D + tid) : 0.f;
-  for (int idx = tid; idx < kRows * D; idx += kVThreads) {
-    const int r = idx / D, i = idx % D;
-    ks[r][i] = bf16_at(k + (row0 + r) * qk_stride + size_t(hk) * D + i);
-    qs[r][i] = bf16_at(q + (row0 + r) * qk_stride + size_t(hk) * D + i);
-  }
-  if (tid < kRows) {
-    G[tid] = g[(row0 + tid) * gb_stride + h];
-    bt[tid] = beta[(row0 + tid) * gb_stride + h];
-  }
-  __syncthreads();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int items = batch * H_v;
+  const int vpg = H_v / H_k;
   if (tid == 0) {
-    float run = 0.f;
-    for (int r = 0; r < kRows; ++r) {
-      run += G[r];
-      G[r] = run;
+    for (int i = 0; i < NSLOT; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 4);  // the four warps that read a half
     }
-  }
-  if (tid >= 64 && tid < 64 + 2 * kRows * kRows) {  // 16 k.k and 16 k.q dot products
-    const int t = tid - 64;
-    const int which = t / (kRows * kRows), s = (t / kRows) % kRows, r = t % kRows;
-    float acc = 0.f;
-    const float* other = which == 0 ? ks[r] : qs[r];
-    for (int i = 0; i < D; ++i) acc = fmaf(ks[s][i], other[i], acc);
-    if (which == 0)
-      kk[s][r] = acc;
-    else
-      kq[s][r] = acc;
-  }
-  // a_r, b_r partial sums over this thread's rows for its 4 columns.
-  float4 acc[2 * kRows];
-#pragma unroll
-  for (int r = 0; r < 2 * kRows; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int ii = 0; ii < RPG; ++ii) {
-    const int i = grp * RPG + ii;
-#pragma unroll
-    for (int r = 0; r < kRows; ++r) {
-      const float kv = ks[r][i], qv = qs[r][i];
-      acc[r].x = fmaf(hv[ii].x, kv, acc[r].x);
-      acc[r].y = fmaf(hv[ii].y, kv, acc[r].y);
-      acc[r].z = fmaf(hv[ii].z, kv, acc[r].z);
-      acc[r].w = fmaf(hv[ii].w, kv, acc[r].w);
-      acc[kRows + r].x = fmaf(hv[ii].x, qv, acc[kRows + r].x);
-      acc[kRows + r].y = fmaf(hv[ii].y, qv, acc[kRows + r].y);
-      acc[kRows + r].z = fmaf(hv[ii].z, qv, acc[kRows + r].z);
-      acc[kRows + r].w = fmaf(hv[ii].w, qv, acc[kRows + r].w);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&dfull[i], 32);
+      mbar_init(&dempty[i], kVCompute / 32);
     }
+    *abort_flag = 0;
+    fence_barrier_init();
+    if (blockIdx.x == 0) atomicOr(flag, kFlagEngaged);
   }
-#pragma unroll
-  for (int r = 0; r < 2 * kRows; ++r) part[grp][r][quad] = acc[r];
   __syncthreads();
-  // One thread per column: reduce the row groups, run the 4-step recurrence.
-  if (tid < D) {
-    const int j = tid;
-    float a[kRows], bq[kRows], delta[kRows];
-#pragma unroll
-    for (int r = 0; r < 2 * kRows; ++r) {
-      float s = 0.f;
-#pragma unroll
-      for (int gg = 0; gg < GROUPS; ++gg) {
-        const float* pp = reinterpret_cast<const float*>(&part[gg][r][j / 4]);
-        s += pp[j % 4];
+
+  if (warp == kVCopyWarp) {
+    // ---------------- state copies: two halves per item with a state
+    if (lane == 0) {
+      int sc = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
+        const int b = it / H_v, h = it - b * H_v;
+        const float* H0 = h_table[b];
+        if (H0 == nullptr) continue;
+        for (int hf = 0; hf < 2 && ok; ++hf, ++sc) {
+          const int slot = sc % NSLOT, use = sc / NSLOT;
+          if (use > 0) ok = mbar_wait(&empty[slot], (use - 1) & 1, abort_flag, &g_err_verify, 1u);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&full[slot], L::HALF);
+          bulk_load_g2s(smem + size_t(slot) * L::HALF,
+                        H0 + size_t(h) * D * D + size_t(hf) * (D / 2) * D, L::HALF, &full[slot]);
+        }
       }
-      if (r < kRows)
-        a[r] = s;
-      else
-        bq[r - kRows] = s;
+      if (!ok) *abort_flag = 1;
+      // nothing may still be landing in shared memory at exit
+      for (int c = max(0, sc - NSLOT); c < sc; ++c)
+        mbar_wait(&full[c % NSLOT], (c / NSLOT) & 1, nullptr, &g_err_verify, 1u);
     }
+    __syncwarp();
+  } else if (warp > kVCopyWarp) {
+    // ---------------- item descriptors: warp 9 the even, warp 10 the odd items
+    const int ds = warp - kVCopyWarp - 1;
+    int n = ds;
+    for (int it = blockIdx.x + ds * gridDim.x; it < items; it += 2 * gridDim.x, n += 2) {
+      const int b = it / H_v, h = it - b * H_v;
+      const int hk = h / vpg;
+      const bool pad = h_table[b] == nullptr;
+      // raw rows into registers before the slot is free: lane l takes i = l + 32 e
+      float kr[kRows][EPL], qr[kRows][EPL], vr[kRows][EPL], gr[kRows], br[kRows];
+      if (!pad) {
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) {
-      float pred = __expf(G[r]) * a[r];
-      for (int s2 = 0; s2 < r; ++s2) pred += __expf(G[r] - G[s2]) * kk[s2][r] * delta[s2];
-      delta[r] = bt[r] * (vr[r] - pred);
-      float out = __expf(G[r]) * bq[r];
-      for (int s2 = 0; s2 <= r; ++s2) out += __expf(G[r] - G[s2]) * kq[s2][r] * delta[s2];
-      o[((row0 + r) * H_v + h) * D + j] = __bfloat16_as_ushort(__float2bfloat16_rn(scale * out));
-      stash[size_t(b) * stash_seq_floats + size_t(h) * kRows * (D + 4) + r * D + j] = delta[r];
+        for (int r = 0; r < kRows; ++r) {
+          const size_t row = size_t(b) * kRows + r;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            const int i = lane + 32 * e;
+            kr[r][e] = bf16_at(k + row * qk_stride + size_t(hk) * D + i);
+            qr[r][e] = bf16_at(q + row * qk_stride + size_t(hk) * D + i);
+            vr[r][e] = bf16_at(v + row * v_stride + size_t(h) * D + i);
+          }
+          gr[r] = g[row * gb_stride + h];
+          br[r] = beta[row * gb_stride + h];
+        }
+      }
+      const int use = n >> 1;
+      bool ok = use == 0 || mbar_wait(&dempty[ds], (use - 1) & 1, abort_flag, &g_err_verify, 2u);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      VerifyDesc<D>& d = desc[ds];
+      if (!pad) {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          const int i = lane + 32 * e;
+          d.kq4[i] = make_float4(kr[0][e], kr[1][e], kr[2][e], kr[3][e]);
+          d.qq4[i] = make_float4(qr[0][e], qr[1][e], qr[2][e], qr[3][e]);
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) d.vv[r][i] = vr[r][e];
+        }
+        // k_s.k_r and k_s.q_r: lane partials, then a butterfly over the warp
+        float dk[kRows][kRows], dq[kRows][kRows];
+#pragma unroll
+        for (int s2 = 0; s2 < kRows; ++s2)
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            float a = 0.f, c = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+              a = fmaf(kr[s2][e], kr[r][e], a);
+              c = fmaf(kr[s2][e], qr[r][e], c);
+            }
+            dk[s2][r] = a;
+            dq[s2][r] = c;
+          }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+          for (int s2 = 0; s2 < kRows; ++s2)
+#pragma unroll
+            for (int r = 0; r < kRows; ++r) {
+              dk[s2][r] += __shfl_xor_sync(0xffffffffu, dk[s2][r], off);
+              dq[s2][r] += __shfl_xor_sync(0xffffffffu, dq[s2][r], off);
+            }
+        if (lane == 0) {
+          float Gc[kRows];
+          float run = 0.f;
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            run += gr[r];
+            Gc[r] = run;
+          }
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            d.eG[r] = __expf(Gc[r]);
+            d.bt[r] = br[r];
+            d.Gc[r] = Gc[r];
+#pragma unroll
+            for (int s2 = 0; s2 < kRows; ++s2) {
+              const float e = __expf(Gc[r] - Gc[s2]);
+              d.cK[s2][r] = s2 < r ? e * dk[s2][r] : 0.f;
+              d.cQ[s2][r] = s2 <= r ? e * dq[s2][r] : 0.f;
+            }
+          }
+        }
+      }
+      if (lane == 0) d.pad = pad ? 1 : 0;
+      mbar_arrive(&dfull[ds]);  // every lane, after its own writes
+    }
+  } else {
+    // ---------------- compute (256 threads)
+    const int quad = tid % QUADS, grp = tid / QUADS;
+    const int half = grp / (GROUPS / 2);
+    const int lrow0 = (grp - half * (GROUPS / 2)) * RPG;  // first row within the half
+    int sc = 0, n = 0;
+    for (int it = blockIdx.x; it < items; it += gridDim.x, ++n) {
+      const int b = it / H_v, h = it - b * H_v;
+      const int ds = n & 1;
+      bool ok = mbar_wait(&dfull[ds], (n >> 1) & 1, abort_flag, &g_err_verify, 4u);
+      const VerifyDesc<D>& d = desc[ds];
+      const bool pad = ok && d.pad != 0;
+      float4 acc[2 * kRows];
+#pragma unroll
+      for (int r = 0; r < 2 * kRows; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (ok && !pad) {
+        const int c = sc + half;
+        const int slot = c % NSLOT;
+        ok = mbar_wait(&full[slot], (c / NSLOT) & 1, abort_flag, &g_err_verify, 4u);
+        if (ok) {
+          const float4* S4 = reinterpret_cast<const float4*>(smem + size_t(slot) * L::HALF);
+#pragma unroll 4
+          for (int ii = 0; ii < RPG; ++ii) {
+            const int i = grp * RPG + ii;
+            const float4 hv = S4[(lrow0 + ii) * QUADS + quad];
+            const float4 kv = d.kq4[i], qv = d.qq4[i];
+            const float kk4[kRows] = {kv.x, kv.y, kv.z, kv.w};
+            const float qq4[kRows] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+            for (int r = 0; r < kRows; ++r) {
+              acc[r].x = fmaf(hv.x, kk4[r], acc[r].x);
+              acc[r].y = fmaf(hv.y, kk4[r], acc[r].y);
+              acc[r].z = fmaf(hv.z, kk4[r], acc[r].z);
+              acc[r].w = fmaf(hv.w, kk4[r], acc[r].w);
+              acc[kRows + r].x = fmaf(hv.x, qq4[r], acc[kRows + r].x);
+              acc[kRows + r].y = fmaf(hv.y, qq4[r], acc[kRows + r].y);
+              acc[kRows + r].z = fmaf(hv.z, qq4[r], acc[kRows + r].z);
+              acc[kRows + r].w = fmaf(hv.w, qq4[r], acc[kRows + r].w);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);  // this warp is done with the slot
+        sc += 2;
+      }
+      // every compute thread agrees before going on (the previous item's
+      // reduction has also finished reading part[])
+      if (!named_all(1, kVCompute, ok)) {
+        *abort_flag = 1;
+        break;
+      }
+      if (!pad) {
+#pragma unroll
+        for (int r = 0; r < 2 * kRows; ++r) part[(grp * 2 * kRows + r) * QUADS + quad] = acc[r];
+      }
+      named_sync(2, kVCompute);
+      if (tid < D) {
+        const int j = tid;
+        const size_t row0 = size_t(b) * kRows;
+        if (pad) {
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) o[((row0 + r) * H_v + h) * D + j] = 0;
+        } else {
+          const float* pf = reinterpret_cast<const float*>(part);
+          float a[kRows], bq[kRows], delta[kRows];
+#pragma unroll
+          for (int r = 0; r < 2 * kRows; ++r) {
+            float s2 = 0.f;
+#pragma unroll
+            for (int gg = 0; gg < GROUPS; ++gg) s2 += pf[(gg * 2 * kRows + r) * D + j];
+            if (r < kRows)
+              a[r] = s2;
+            else
+              bq[r - kRows] = s2;
+          }
+          float* st = stash + size_t(b) * stash_seq_floats + size_t(h) * kRows * (D + 4);
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            float pred = d.eG[r] * a[r];
+#pragma unroll
+            for (int s2 = 0; s2 < r; ++s2) pred += d.cK[s2][r] * delta[s2];
+            delta[r] = d.bt[r] * (d.vv[r][j] - pred);
+            float out = d.eG[r] * bq[r];
+#pragma unroll
+            for (int s2 = 0; s2 <= r; ++s2) out += d.cQ[s2][r] * delta[s2];
+            o[((row0 + r) * H_v + h) * D + j] = __bfloat16_as_ushort(__float2bfloat16_rn(scale * out));
+            st[r * D + j] = delta[r];
+          }
+          if (j < kRows) st[kRows * D + j] = d.Gc[j];
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dempty[ds]);  // this warp is done with the descriptor
     }
   }
-  if (tid < kRows)
-    stash[size_t(b) * stash_seq_floats + size_t(h) * kRows * (D + 4) + kRows * D + tid] = G[tid];
+  __syncthreads();
 }
 
 // grid = (H_v, batch); block = 256.  Each thread loads all of its 16-byte
@@ -248,15 +419,25 @@ cudaError_t launch_verify(float* const* h_table, const uint16_t* q, const uint16
                           int stash_seq_floats, int batch, int H_k, int H_v, int D, float scale,
                           uint32_t* flag, cudaStream_t s) {
   if (batch == 0) return cudaSuccess;
-  dim3 grid(H_v, batch);
-  if (D == 128)
-    verify_kernel<128><<<grid, kVThreads, 0, s>>>(h_table, q, k, qk_stride, v, v_stride, g, beta,
-                                            gb_stride, o, stash, stash_seq_floats, H_k, H_v,
-                                            scale, flag);
-  else
-    verify_kernel<64><<<grid, kVThreads, 0, s>>>(h_table, q, k, qk_stride, v, v_stride, g, beta,
-                                           gb_stride, o, stash, stash_seq_floats, H_k, H_v,
-                                           scale, flag);
+  const int items = batch * H_v;
+  const int grid = items < sm_count() ? items : sm_count();
+  if (D == 128) {
+    const int smem = int(VerifySmem<128>::TOTAL) + 128;
+    cudaError_t e = cudaFuncSetAttribute(verify_kernel<128>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    verify_kernel<128><<<grid, kVBlock, smem, s>>>(h_table, q, k, qk_stride, v, v_stride, g,
+                                                   beta, gb_stride, o, stash, stash_seq_floats,
+                                                   batch, H_k, H_v, scale, flag);
+  } else {
+    const int smem = int(VerifySmem<64>::TOTAL) + 128;
+    cudaError_t e = cudaFuncSetAttribute(verify_kernel<64>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    verify_kernel<64><<<grid, kVBlock, smem, s>>>(h_table, q, k, qk_stride, v, v_stride, g,
+                                                  beta, gb_stride, o, stash, stash_seq_floats,
+                                                  batch, H_k, H_v, scale, flag);
+  }
   return cudaGetLastError();
 }
 
