@@ -53,28 +53,50 @@ constexpr int kVThreads = 256;  // fold block; verify compute threads
 
 // ---------------------------------------------------------------------------
 // Verify: one persistent CTA per SM walks the (sequence, v-head) items
-// blockIdx.x, blockIdx.x + gridDim.x, ...  Warp roles:
-//   warps 0-7 (256 threads)  compute: thread = (row group, column quad); the
-//       FMA phase reads its rows of the item's state from shared memory and
-//       accumulates a_r and b_r for its four columns; warps 0 .. D/32 - 1 then
-//       reduce the row groups and run the per-column 4-step recurrence.
+// blockIdx.x, blockIdx.x + gridDim.x, ...  Warp roles, each warp running at
+// its own pace (mbarriers only, no block-wide barrier inside the loop):
+//   warps 0-7 (256 threads)  FMA: thread = (row group, column quad); reads
+//       its rows of the item's state from shared memory and accumulates the
+//       row-group partials of a_r and b_r for its four columns into part[];
+//       warps 0-3 read the first half of the state, warps 4-7 the second.
 //   warp 8   copies: each item's state, as two contiguous halves (rows
 //       0 .. D/2 - 1 and D/2 .. D - 1), into a ring of shared-memory slots
 //       with cp.async.bulk, as far ahead as the ring allows.
-//   warps 9, 10  item descriptors (even / odd items): k and q transposed to
-//       4-row vectors, v, the dot products k_s.k_r and k_s.q_r, the cumulative
-//       gates and the decay factors, prepared while earlier items compute.
-// Warps 0-3 read the first half of the state, warps 4-7 the second.
+//   warps 9-11  item descriptors (warp 9 + m takes the items n = m mod 3 into
+//       descriptor slot m): k and q transposed to 4-row vectors, v, the dot
+//       products k_s.k_r and k_s.q_r, the cumulative gates and the decay
+//       factors, prepared while earlier items compute (their global loads
+//       take microseconds while the state copies saturate HBM, hence three).
+//   warps 12-15  epilogue: thread j < D reduces the row groups of column j
+//       and runs its 4-step recurrence, while the FMA warps go on with the
+//       next item (part[] is double-buffered).
 // ---------------------------------------------------------------------------
+// Packed f32x2 arithmetic (two IEEE f32 FMAs per instruction): a pair lives
+// in one 64-bit register, low half first.
+__device__ __forceinline__ uint64_t dup_f32x2(float x) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(d) : "f"(x));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float lo_f32x2(uint64_t d) { return __uint_as_float(uint32_t(d)); }
+__device__ __forceinline__ float hi_f32x2(uint64_t d) { return __uint_as_float(uint32_t(d >> 32)); }
+
 constexpr int kVCompute = 256;
 constexpr int kVCopyWarp = 8;
-constexpr int kVBlock = kVCompute + 3 * 32;
-constexpr uint32_t kVRingBytes = 160 * 1024;
+constexpr int kVDesc = 3;  // descriptor slots = descriptor warps (16 warps in all)
+constexpr int kVEpiWarp = kVCopyWarp + 1 + kVDesc;
+constexpr int kVEpi = 128;
+constexpr int kVBlock = kVCompute + 32 * (1 + kVDesc) + kVEpi;
+constexpr uint32_t kVRingBytes = 128 * 1024;
 
 template <int D>
 struct VerifyDesc {
-  float4 kq4[D];        // (k_0[i], k_1[i], k_2[i], k_3[i])
-  float4 qq4[D];        // (q_0[i], .., q_3[i])
+  float4 kq[D][2];      // (k_0[i], q_0[i], k_1[i], q_1[i]), (k_2[i], q_2[i], k_3[i], q_3[i])
   float vv[kRows][D];   // v rows
   float eG[kRows];      // e^{G_r}
   float cK[kRows][kRows];  // [s][r] = e^{G_r - G_s} k_s.k_r   (s < r)
@@ -92,11 +114,12 @@ struct VerifySmem {
   static constexpr int RPG = D / GROUPS;            // rows per group: 16 / 4
   static constexpr uint32_t HALF = uint32_t(D) * D * 4 / 2;
   static constexpr int NSLOT = int(kVRingBytes / HALF);
-  static constexpr uint32_t PART = 0 + kVRingBytes;  // float4 [GROUPS][2*kRows][QUADS]
-  static constexpr uint32_t DESC = PART + uint32_t(GROUPS) * 2 * kRows * QUADS * 16;
-  static constexpr uint32_t BARS = DESC + 2 * uint32_t(sizeof(VerifyDesc<D>));
-  // full[NSLOT], empty[NSLOT], dfull[2], dempty[2], abort word
-  static constexpr uint32_t TOTAL = BARS + (2 * NSLOT + 4) * 8 + 16;
+  static constexpr uint32_t PART_BYTES = uint32_t(GROUPS) * 2 * kRows * QUADS * 16;
+  static constexpr uint32_t PART = 0 + kVRingBytes;  // 2 x float4 [GROUPS][2*kRows][QUADS]
+  static constexpr uint32_t DESC = PART + 2 * PART_BYTES;
+  static constexpr uint32_t BARS = DESC + kVDesc * uint32_t(sizeof(VerifyDesc<D>));
+  // full[NSLOT], empty[NSLOT], dfull[kVDesc], dempty[kVDesc], pfull[2], pempty[2], abort word
+  static constexpr uint32_t TOTAL = BARS + (2 * NSLOT + 2 * kVDesc + 4) * 8 + 16;
 };
 static_assert(VerifySmem<128>::TOTAL + 128 <= 232448, "verify shared memory");
 static_assert(VerifySmem<64>::TOTAL + 128 <= 232448, "verify shared memory");
@@ -114,13 +137,14 @@ __global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                              ~uintptr_t(127));
-  float4* part = reinterpret_cast<float4*>(smem + L::PART);
   VerifyDesc<D>* desc = reinterpret_cast<VerifyDesc<D>*>(smem + L::DESC);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BARS);
   uint64_t* empty = full + NSLOT;
   uint64_t* dfull = empty + NSLOT;
-  uint64_t* dempty = dfull + 2;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(dempty + 2);
+  uint64_t* dempty = dfull + kVDesc;
+  uint64_t* pfull = dempty + kVDesc;
+  uint64_t* pempty = pfull + 2;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(pempty + 2);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int items = batch * H_v;
@@ -130,9 +154,13 @@ __global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 4);  // the four warps that read a half
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kVDesc; ++i) {
       mbar_init(&dfull[i], 32);
-      mbar_init(&dempty[i], kVCompute / 32);
+      mbar_init(&dempty[i], (kVCompute + kVEpi) / 32);  // FMA and epilogue warps
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&pfull[i], kVCompute / 32);
+      mbar_init(&pempty[i], kVEpi / 32);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -164,11 +192,11 @@ __global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
         mbar_wait(&full[c % NSLOT], (c / NSLOT) & 1, nullptr, &g_err_verify, 1u);
     }
     __syncwarp();
-  } else if (warp > kVCopyWarp) {
-    // ---------------- item descriptors: warp 9 the even, warp 10 the odd items
+  } else if (warp > kVCopyWarp && warp < kVEpiWarp) {
+    // ---------------- item descriptors: warp 9 + m the items n = m (mod kVDesc)
     const int ds = warp - kVCopyWarp - 1;
     int n = ds;
-    for (int it = blockIdx.x + ds * gridDim.x; it < items; it += 2 * gridDim.x, n += 2) {
+    for (int it = blockIdx.x + ds * gridDim.x; it < items; it += kVDesc * gridDim.x, n += kVDesc) {
       const int b = it / H_v, h = it - b * H_v;
       const int hk = h / vpg;
       const bool pad = h_table[b] == nullptr;
@@ -189,7 +217,7 @@ __global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
           br[r] = beta[row * gb_stride + h];
         }
       }
-      const int use = n >> 1;
+      const int use = n / kVDesc;
       bool ok = use == 0 || mbar_wait(&dempty[ds], (use - 1) & 1, abort_flag, &g_err_verify, 2u);
       if (!__all_sync(0xffffffffu, ok)) break;
       VerifyDesc<D>& d = desc[ds];
@@ -197,8 +225,8 @@ __global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
           const int i = lane + 32 * e;
-          d.kq4[i] = make_float4(kr[0][e], kr[1][e], kr[2][e], kr[3][e]);
-          d.qq4[i] = make_float4(qr[0][e], qr[1][e], qr[2][e], qr[3][e]);
+          d.kq[i][0] = make_float4(kr[0][e], qr[0][e], kr[1][e], qr[1][e]);
+          d.kq[i][1] = make_float4(kr[2][e], qr[2][e], kr[3][e], qr[3][e]);
 #pragma unroll
           for (int r = 0; r < kRows; ++r) d.vv[r][i] = vr[r][e];
         }
@@ -226,47 +254,69 @@ __global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
               dk[s2][r] += __shfl_xor_sync(0xffffffffu, dk[s2][r], off);
               dq[s2][r] += __shfl_xor_sync(0xffffffffu, dq[s2][r], off);
             }
-        if (lane == 0) {
-          float Gc[kRows];
-          float run = 0.f;
+        // every lane holds the totals and the cumulative gates; lane
+        // 4 s + r writes the [s][r] factors, lanes r < 4 the per-row ones
+        float Gc[kRows];
+        float run = 0.f;
 #pragma unroll
-          for (int r = 0; r < kRows; ++r) {
-            run += gr[r];
-            Gc[r] = run;
+        for (int r = 0; r < kRows; ++r) {
+          run += gr[r];
+          Gc[r] = run;
+        }
+        if (lane < kRows * kRows) {
+          const int s2 = lane >> 2, r = lane & 3;
+          float gs = Gc[0], grr = Gc[0], kkv = dk[0][0], kqv = dq[0][0];
+#pragma unroll
+          for (int x = 0; x < kRows; ++x) {
+            if (x == s2) gs = Gc[x];
+            if (x == r) grr = Gc[x];
+#pragma unroll
+            for (int y = 0; y < kRows; ++y)
+              if (x == s2 && y == r) {
+                kkv = dk[x][y];
+                kqv = dq[x][y];
+              }
           }
+          const float e = __expf(grr - gs);
+          d.cK[s2][r] = s2 < r ? e * kkv : 0.f;
+          d.cQ[s2][r] = s2 <= r ? e * kqv : 0.f;
+          if (lane < kRows) {
+            float gl = Gc[0], bl = br[0];
 #pragma unroll
-          for (int r = 0; r < kRows; ++r) {
-            d.eG[r] = __expf(Gc[r]);
-            d.bt[r] = br[r];
-            d.Gc[r] = Gc[r];
-#pragma unroll
-            for (int s2 = 0; s2 < kRows; ++s2) {
-              const float e = __expf(Gc[r] - Gc[s2]);
-              d.cK[s2][r] = s2 < r ? e * dk[s2][r] : 0.f;
-              d.cQ[s2][r] = s2 <= r ? e * dq[s2][r] : 0.f;
-            }
+            for (int x = 1; x < kRows; ++x)
+              if (x == lane) {
+                gl = Gc[x];
+                bl = br[x];
+              }
+            d.eG[lane] = __expf(gl);
+            d.bt[lane] = bl;
+            d.Gc[lane] = gl;
           }
         }
       }
       if (lane == 0) d.pad = pad ? 1 : 0;
       mbar_arrive(&dfull[ds]);  // every lane, after its own writes
     }
-  } else {
-    // ---------------- compute (256 threads)
+  } else if (warp < kVCopyWarp) {
+    // ---------------- FMA warps (256 threads)
     const int quad = tid % QUADS, grp = tid / QUADS;
     const int half = grp / (GROUPS / 2);
     const int lrow0 = (grp - half * (GROUPS / 2)) * RPG;  // first row within the half
     int sc = 0, n = 0;
-    for (int it = blockIdx.x; it < items; it += gridDim.x, ++n) {
-      const int b = it / H_v, h = it - b * H_v;
-      const int ds = n & 1;
-      bool ok = mbar_wait(&dfull[ds], (n >> 1) & 1, abort_flag, &g_err_verify, 4u);
+    bool ok = true;
+    for (int it = blockIdx.x; it < items && ok; it += gridDim.x, ++n) {
+      const int ds = n % kVDesc, pb = n & 1, pu = n >> 1;
+      ok = mbar_wait(&dfull[ds], (n / kVDesc) & 1, abort_flag, &g_err_verify, 4u);
+      if (!__all_sync(0xffffffffu, ok)) break;
       const VerifyDesc<D>& d = desc[ds];
-      const bool pad = ok && d.pad != 0;
-      float4 acc[2 * kRows];
+      const bool pad = d.pad != 0;
+      // acc[c][r] = (a_r, b_r) partials of column 4 quad + c
+      uint64_t acc[4][kRows];
 #pragma unroll
-      for (int r = 0; r < 2 * kRows; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (ok && !pad) {
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) acc[c][r] = 0ull;
+      if (!pad) {
         const int c = sc + half;
         const int slot = c % NSLOT;
         ok = mbar_wait(&full[slot], (c / NSLOT) & 1, abort_flag, &g_err_verify, 4u);
@@ -276,45 +326,65 @@ __global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
           for (int ii = 0; ii < RPG; ++ii) {
             const int i = grp * RPG + ii;
             const float4 hv = S4[(lrow0 + ii) * QUADS + quad];
-            const float4 kv = d.kq4[i], qv = d.qq4[i];
-            const float kk4[kRows] = {kv.x, kv.y, kv.z, kv.w};
-            const float qq4[kRows] = {qv.x, qv.y, qv.z, qv.w};
+            const ulonglong2 p01 = *reinterpret_cast<const ulonglong2*>(&d.kq[i][0]);
+            const ulonglong2 p23 = *reinterpret_cast<const ulonglong2*>(&d.kq[i][1]);
+            const uint64_t kq2[kRows] = {p01.x, p01.y, p23.x, p23.y};  // (k_r[i], q_r[i])
+            const float hs[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
-            for (int r = 0; r < kRows; ++r) {
-              acc[r].x = fmaf(hv.x, kk4[r], acc[r].x);
-              acc[r].y = fmaf(hv.y, kk4[r], acc[r].y);
-              acc[r].z = fmaf(hv.z, kk4[r], acc[r].z);
-              acc[r].w = fmaf(hv.w, kk4[r], acc[r].w);
-              acc[kRows + r].x = fmaf(hv.x, qq4[r], acc[kRows + r].x);
-              acc[kRows + r].y = fmaf(hv.y, qq4[r], acc[kRows + r].y);
-              acc[kRows + r].z = fmaf(hv.z, qq4[r], acc[kRows + r].z);
-              acc[kRows + r].w = fmaf(hv.w, qq4[r], acc[kRows + r].w);
+            for (int cc = 0; cc < 4; ++cc) {
+              const uint64_t s2 = dup_f32x2(hs[cc]);
+#pragma unroll
+              for (int r = 0; r < kRows; ++r) acc[cc][r] = fma_f32x2(s2, kq2[r], acc[cc][r]);
             }
           }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);  // this warp is done with the slot
         sc += 2;
+        if (!__all_sync(0xffffffffu, ok)) break;
       }
-      // every compute thread agrees before going on (the previous item's
-      // reduction has also finished reading part[])
-      if (!named_all(1, kVCompute, ok)) {
-        *abort_flag = 1;
-        break;
-      }
+      // part[pb] is free once the epilogue finished item n - 2
+      ok = pu == 0 || mbar_wait(&pempty[pb], (pu - 1) & 1, abort_flag, &g_err_verify, 4u);
+      if (!__all_sync(0xffffffffu, ok)) break;
       if (!pad) {
+        float4* part = reinterpret_cast<float4*>(smem + L::PART + pb * L::PART_BYTES);
 #pragma unroll
-        for (int r = 0; r < 2 * kRows; ++r) part[(grp * 2 * kRows + r) * QUADS + quad] = acc[r];
+        for (int r = 0; r < kRows; ++r) {
+          part[(grp * 2 * kRows + r) * QUADS + quad] =
+              make_float4(lo_f32x2(acc[0][r]), lo_f32x2(acc[1][r]), lo_f32x2(acc[2][r]),
+                          lo_f32x2(acc[3][r]));
+          part[(grp * 2 * kRows + kRows + r) * QUADS + quad] =
+              make_float4(hi_f32x2(acc[0][r]), hi_f32x2(acc[1][r]), hi_f32x2(acc[2][r]),
+                          hi_f32x2(acc[3][r]));
+        }
       }
-      named_sync(2, kVCompute);
-      if (tid < D) {
-        const int j = tid;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&pfull[pb]);
+        mbar_arrive(&dempty[ds]);  // the FMA warps are done with the descriptor
+      }
+    }
+    if (!ok) *abort_flag = 1;
+  } else {
+    // ---------------- epilogue warps (128 threads): reduction + recurrence
+    const int et = tid - kVEpiWarp * 32;
+    int n = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < items && ok; it += gridDim.x, ++n) {
+      const int b = it / H_v, h = it - b * H_v;
+      const int ds = n % kVDesc, pb = n & 1;
+      ok = mbar_wait(&dfull[ds], (n / kVDesc) & 1, abort_flag, &g_err_verify, 8u) &&
+           mbar_wait(&pfull[pb], (n >> 1) & 1, abort_flag, &g_err_verify, 8u);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const VerifyDesc<D>& d = desc[ds];
+      if (et < D) {
+        const int j = et;
         const size_t row0 = size_t(b) * kRows;
-        if (pad) {
+        if (d.pad != 0) {
 #pragma unroll
           for (int r = 0; r < kRows; ++r) o[((row0 + r) * H_v + h) * D + j] = 0;
         } else {
-          const float* pf = reinterpret_cast<const float*>(part);
+          const float* pf = reinterpret_cast<const float*>(smem + L::PART + pb * L::PART_BYTES);
           float a[kRows], bq[kRows], delta[kRows];
 #pragma unroll
           for (int r = 0; r < 2 * kRows; ++r) {
@@ -343,8 +413,12 @@ __global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&dempty[ds]);  // this warp is done with the descriptor
+      if (lane == 0) {
+        mbar_arrive(&pempty[pb]);
+        mbar_arrive(&dempty[ds]);  // the epilogue warps are done with the descriptor
+      }
     }
+    if (!ok) *abort_flag = 1;
   }
   __syncthreads();
 }
