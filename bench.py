@@ -191,28 +191,30 @@ def make_inputs(dev):
 
 
 def step_calls(d, meta, ev=None):
-    """Queue one step on the current stream; ev: optional list of 6 events."""
+    """Queue one step on the current stream.  ev: optional list of 6 events
+    (None entries are skipped) recorded before BA, prefill, flag clear,
+    verify, fold and after fold."""
     from linear_attention_ssm_gdn_b200 import (gdn_ba_gates, gdn_chunk_prefill, gdn_flag_clear,
                                                gdn_fold, gdn_verify_woa)
     nv = meta["nv"]
-    if ev:
+    if ev and ev[0] is not None:
         ev[0].record()
     gdn_ba_gates(d["x"], d["w"], d["a_log"], d["dt_bias"], meta["vpg"], gate_out=d["gates"])
-    if ev:
+    if ev and ev[1] is not None:
         ev[1].record()
     gdn_chunk_prefill(d["q"], d["k"], d["v"], d["gates"][:, :nv], d["gates"][:, nv:], d["cu"],
                       h0=d["h0"], hT=d["hT"], o=d["o"], workspace=d["ws"])
-    if ev:
+    if ev and ev[2] is not None:
         ev[2].record()
     gdn_flag_clear(d["flag"])
-    if ev:
+    if ev and ev[3] is not None:
         ev[3].record()
     gdn_verify_woa(d["table"], d["vq"], d["vk"], d["vv"], d["vg"], d["vb"], d["flag"], o=d["vo"],
                    stash=d["stash"])
-    if ev:
+    if ev and ev[4] is not None:
         ev[4].record()
     gdn_fold(d["table"], d["stash"], d["na"], d["vk"], d["flag"], meta["H_v"])
-    if ev:
+    if ev and ev[5] is not None:
         ev[5].record()
 
 
@@ -231,9 +233,13 @@ def run_ours(args, rank, world, dist):
         step_calls(d, meta)
     torch.cuda.synchronize()
 
-    # ---- timed region: exactly K steps, per-kernel events on the launch stream
+    # ---- timed region: exactly K steps.  Only the prefill kernel (the
+    # roofline kernel) is bracketed by events here: every event record costs
+    # the stream about 2.7 us, so the split of the other kernels comes from a
+    # separate, untimed pass below.
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    evs = [[None, torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            None, None, None] for _ in range(K)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(dev.index).start()
@@ -249,9 +255,17 @@ def run_ours(args, rank, world, dist):
         dist.barrier()
     clk = clocks.stop()
     total_ms = t_start.elapsed_time(t_end)
-    per = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
-           for j, name in enumerate(["ba_gates", "prefill", "flag_clear", "verify", "fold"])}
+    t_prefill_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     total_ms = max_over_ranks(total_ms, dist, dev)
+
+    # ---- untimed split: per-kernel events on every kernel of a few steps
+    ks = max(1, min(K, 50))
+    evs2 = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(ks)]
+    for i in range(ks):
+        step_calls(d, meta, evs2[i])
+    torch.cuda.synchronize()
+    per = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs2)
+           for j, name in enumerate(["ba_gates", "prefill", "flag_clear", "verify", "fold"])}
 
     # ---- end to end through the public API: H2D inputs, the calls, D2H results
     pinned = {k: v.pin_memory() for k, v in host.items()}
@@ -286,7 +300,7 @@ def run_ours(args, rank, world, dist):
     hbm, tf_burst, tf_sust, src = peaks()
     B = prefill_alg_bytes(T, meta["N"], meta["H_k"], meta["H_v"], meta["d_k"], meta["d_v"])
     F = prefill_alg_flops(T, meta["H_v"], meta["d_k"], meta["d_v"])
-    t_pf = per["prefill"] / 1e3
+    t_pf = t_prefill_ms / 1e3
     achieved = B / t_pf / 1e9
     t_roof = max(B / (hbm * 1e9), F / (tf_burst * 1e12))
     line = {
@@ -303,6 +317,8 @@ def run_ours(args, rank, world, dist):
                      "roofline_time_us": t_roof * 1e6,
                      "frac_of_roofline_time": t_roof / t_pf},
         "kernels_us": {k: v * 1e3 for k, v in per.items()},
+        "kernels_us_note": "separate untimed pass with events around every kernel "
+                           "(each event record adds about 2.7 us to its interval)",
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": LAUNCHES_PER_STEP * K,

@@ -61,6 +61,16 @@ __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// log(1 + t) for t in [0, 1], relative error below 1e-5: the Taylor series
+// t - t^2/2 + t^3/3 - ... through t^6 below t = 1/16 (truncation < t^6 / 7),
+// and the fast logarithm of 1 + t above it (its absolute error over a result
+// of at least log(17/16) = 0.06).
+__device__ __forceinline__ float log1p_unit(float t) {
+  if (t < 0.0625f)
+    return t * (1.0f - t * (0.5f - t * (1.0f / 3.0f - t * (0.25f - t * (0.2f - t * (1.0f / 6.0f))))));
+  return __logf(1.0f + t);
+}
+
 __global__ void __launch_bounds__(kBaThreads, 1)
     ba_gates_kernel(const __grid_constant__ CUtensorMap tmap_x,
                     const __grid_constant__ CUtensorMap tmap_w, const BaParams p) {
@@ -208,56 +218,38 @@ __global__ void __launch_bounds__(kBaThreads, 1)
   tc_fence_before();
   cluster_arrive_release();  // the pushes above, before the owners read them
   cluster_wait_acquire();
-  // Reduction + epilogue over this rank's rows, flat over (row lr, output
-  // column j) so that consecutive threads store consecutive columns; (lr, j)
-  // advance by the fixed thread stride without divisions, kEpU elements per
-  // thread at a time so that their shared-memory reads overlap.
-  {
-    constexpr int kEpU = 4;
-    const int w2 = 2 * p.nv, total = rows * w2;
-    const bool write = ok && !*abort_flag;
-    const int dl = kBaThreads / w2, dj = kBaThreads - dl * w2;
-    int lr = int(threadIdx.x) / w2, j = int(threadIdx.x) - lr * w2;
-    for (int i = int(threadIdx.x); i < total; i += kEpU * kBaThreads) {
-      int lrs[kEpU], js[kEpU];
-      bool live[kEpU];
-      uint32_t cm[kEpU];
-      float sum[kEpU];
-#pragma unroll
-      for (int u = 0; u < kEpU; ++u) {
-        lrs[u] = lr;
-        js[u] = j;
-        live[u] = write && i + u * kBaThreads < total && m0 + rank * rows + lr < p.M;
+  // Reduction + epilogue over this rank's valid rows: a pass over the gate
+  // columns (j < nv: the gate of v-head j) and one over the beta columns
+  // (nv + j), each flat over (row lr, column j) so that consecutive threads
+  // store consecutive columns of a row and no warp mixes the two paths;
+  // (lr, j) advance by the fixed thread stride without divisions.
+  if (ok && !*abort_flag) {
+    const int nv = p.nv;
+    const int row0 = m0 + rank * rows;
+    const int total = max(0, min(rows, p.M - row0)) * nv;
+    const int dl = kBaThreads / nv, dj = kBaThreads - dl * nv;
+    const uint32_t qstride = uint32_t(rows * pstride);
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+      int lr = int(threadIdx.x) / nv, j = int(threadIdx.x) - lr * nv;
+      for (int i = int(threadIdx.x); i < total; i += kBaThreads) {
+        const float* col = recv + uint32_t(lr * pstride) + (colmap[pass * nv + j] & 0xffffu);
+        float sum = 0.0f;
+        for (int q = 0; q < p.ks; ++q) sum += col[uint32_t(q) * qstride];  // rank order
+        float val;
+        if (pass == 0) {
+          const float z = sum + dtb[j];
+          val = coef[j] * (fmaxf(z, 0.0f) + log1p_unit(__expf(-fabsf(z))));
+        } else {
+          val = __frcp_rn(1.0f + __expf(-sum));
+        }
+        p.out[size_t(row0 + lr) * p.gate_stride + pass * nv + j] = val;
         lr += dl;
         j += dj;
-        if (j >= w2) {
-          j -= w2;
+        if (j >= nv) {
+          j -= nv;
           ++lr;
         }
-      }
-#pragma unroll
-      for (int u = 0; u < kEpU; ++u) cm[u] = live[u] ? colmap[js[u]] : 0u;
-#pragma unroll
-      for (int u = 0; u < kEpU; ++u) {
-        const float* col = recv + size_t(lrs[u]) * pstride + (cm[u] & 0xffffu);
-        float acc = 0.0f;
-        for (int q = 0; q < p.ks; ++q)  // fixed order: deterministic
-          acc += live[u] ? col[size_t(q * rows) * pstride] : 0.0f;
-        sum[u] = acc;
-      }
-#pragma unroll
-      for (int u = 0; u < kEpU; ++u) {
-        if (!live[u]) continue;
-        const int vh = int((cm[u] >> 16) & 0x7fffu);
-        float val;
-        if (cm[u] & 0x80000000u) {
-          const float z = sum[u] + dtb[vh];
-          const float sp = fmaxf(z, 0.0f) + log1pf(__expf(-fabsf(z)));
-          val = coef[vh] * sp;
-        } else {
-          val = __frcp_rn(1.0f + __expf(-sum[u]));
-        }
-        p.out[size_t(m0 + rank * rows + lrs[u]) * p.gate_stride + js[u]] = val;
       }
     }
   }
