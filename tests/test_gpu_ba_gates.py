@@ -58,3 +58,13 @@ def test_ba_gates_zero_weight_closed_form():
     want_g = -np.exp(f64(ba.a_log)) * np.log1p(np.exp(f64(ba.dt_bias)))
     np.testing.assert_allclose(got[:, :6], np.broadcast_to(want_g, (130, 6)), rtol=1e-5)
     np.testing.assert_allclose(got[:, 6:], 0.5, rtol=1e-6)
+
+
+def test_ba_gates_wide_range():
+    """Weights scaled so that |ba| reaches about 60: softplus runs through both
+    of its branches (series for e^{-|z|} < 1/16, logarithm above) and the
+    sigmoid through its tails; every output within the elementwise bound."""
+    ba = I.ba_inputs(512, 1024, 48, 3, seed=5)
+    ba.w = (ba.w.float() * 20.0).to(torch.bfloat16)
+    got = _check(ba)
+    assert float(np.abs(got[:, :48]).min()) < 1e-6 < float(np.abs(got[:, :48]).max())

@@ -132,3 +132,32 @@ def test_d64_heads():
     o_ref, h_ref = oracle.gdn_verify_fold(f64(vi.pool)[slots], f64(vi.q), f64(vi.k), f64(vi.v),
                                           f64(vi.g), f64(vi.beta), vi.na.numpy())
     assert_prefill_close(o, pool.numpy()[slots], o_ref, h_ref, "d=64")
+
+
+@pytest.mark.parametrize("batch,H_k,H_v,d", [(150, 2, 4, 128), (240, 2, 6, 64)])
+def test_many_items_per_cta_with_padding(batch, H_k, H_v, d):
+    """More (sequence, v-head) items than SMs, every third sequence a padding
+    entry: each persistent CTA walks several items, and its half-state ring
+    (4 slots at d = 128, 16 at d = 64) wraps across padding items, which
+    take no slot.  Outputs and folded states of the present sequences match
+    the oracle; padding rows are zero and their states bit-identical."""
+    vi = I.verify_inputs(batch, 4, H_k, H_v, d, d, slots_total=batch + 3, seed=46 + d)
+    pool, table, dd, flag = _setup(vi)
+    present = np.ones(batch, dtype=np.int32)
+    present[::3] = 0
+    for b in np.nonzero(present == 0)[0]:
+        table[int(b)] = 0
+    gdn_flag_clear(flag)
+    o, stash = gdn_verify_woa(table, dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], flag)
+    gdn_fold(table, stash, dd["na"], dd["k"], flag, vi.H_v)
+    torch.cuda.synchronize()
+    assert debug_device_errors() == [0, 0, 0, 0]
+    slots = vi.slots.numpy()
+    o_ref, h_ref = oracle.gdn_verify_fold(f64(vi.pool)[slots], f64(vi.q), f64(vi.k), f64(vi.v),
+                                          f64(vi.g), f64(vi.beta), vi.na.numpy(), present=present)
+    o_np = o.float().cpu().numpy()
+    pool_after = pool.cpu()
+    assert_prefill_close(o_np, pool_after.numpy()[slots], o_ref, h_ref, f"padded d={d}")
+    for b in np.nonzero(present == 0)[0]:
+        assert np.all(o_np[4 * b:4 * b + 4] == 0)
+        assert torch.equal(pool_after[slots[b]], vi.pool[slots[b]])
