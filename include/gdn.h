@@ -131,8 +131,11 @@ int gdn_chunk_prefill(const uint16_t* q, const uint16_t* k, int qk_stride, const
  *   gates, padded to a multiple of 4 floats.
  *
  *   h_table  [batch] device array of device pointers; entry b points at the
- *            state of sequence b, [H_v, d_k, d_v] f32; a NULL entry marks a
- *            padding sequence (its o rows are written as zeros, nothing else)
+ *            state of sequence b, [H_v, d_k, d_v] f32, 16-byte aligned (the
+ *            verify streams each state with bulk copies, the fold uses 16-byte
+ *            accesses; entries live on the device, so this is not checked);
+ *            a NULL entry marks a padding sequence (its o rows are written as
+ *            zeros, nothing else)
  *   q, k     [batch*4, qk_stride] bf16; rows b*4 .. b*4+3 belong to sequence b
  *   v        [batch*4, v_stride] bf16; g, beta [batch*4, gb_stride] f32
  *   o        [batch*4, H_v, d_v] bf16
@@ -140,6 +143,8 @@ int gdn_chunk_prefill(const uint16_t* q, const uint16_t* k, int qk_stride, const
  *            read by gdn_fold; stash_seq_floats >= gdn_stash_seq_floats(...)
  *   engaged_flag  u32: bit 0 is OR-ed in by every launched verify
  * No state is written.  Supported: d_k == d_v in {64, 128}, H_v % H_k == 0.
+ * Launch: min(batch * H_v, SM count) persistent CTAs of 512 threads walk the
+ * (sequence, v-head) items; 211 KB (d = 128) of dynamic shared memory each.
  * Errors: GDN_ERR_NULL (h_table, stash, engaged_flag, q, k, v, g, beta or o
  * NULL -- the null guard of the page's launcher), GDN_ERR_SHAPE,
  * GDN_ERR_STRIDE, GDN_ERR_ALIGN, GDN_ERR_CUDA.  batch == 0 launches nothing.

@@ -10,10 +10,9 @@
 //   delta_r[j] = beta_r (v_r[j] - e^{G_r} a_r[j]
 //                          - sum_{s<r} e^{G_r - G_s} kk[s][r] delta_s[j])
 //   o_r[j] = scale (e^{G_r} b_r[j] + sum_{s<=r} e^{G_r - G_s} kq[s][r] delta_s[j])
-// which is the token recurrence unrolled over four rows.  H0 is read once
-// (16-byte loads, 4 columns per thread, 8 row groups per CTA, every load of a
-// thread in flight at once); nothing is written to it.  delta_r and G_r go to
-// the stash for the fold.
+// which is the token recurrence unrolled over four rows.  H0 is read once,
+// streamed into shared memory by bulk copies (persistent kernel below);
+// nothing is written to it.  delta_r and G_r go to the stash for the fold.
 //
 // Fold.  With na = na_tab[b] in 1..4 (and the engaged bit set):
 //   H[i][j] <- e^{G_{na-1}} H[i][j] + sum_{r<na} e^{G_{na-1} - G_r} k_r[i] delta_r[j]
@@ -49,7 +48,7 @@ __global__ void flag_clear_kernel(uint32_t* flag) {
   if (threadIdx.x == 0) *flag = 0u;
 }
 
-constexpr int kVThreads = 256;  // fold block; verify compute threads
+constexpr int kVThreads = 256;  // fold block
 
 // ---------------------------------------------------------------------------
 // Verify: one persistent CTA per SM walks the (sequence, v-head) items
