@@ -83,6 +83,27 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
   return d;
 }
 __device__ __forceinline__ float lo_f32x2(uint64_t d) { return __uint_as_float(uint32_t(d)); }
+
+// Shared-space loads by 32-bit shared address (the block's dynamic shared
+// memory is addressed through a realigned generic pointer, which the
+// compiler would otherwise access with generic loads).
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ ulonglong2 lds_u64x2(uint32_t addr) {
+  ulonglong2 v;
+  asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
 __device__ __forceinline__ float hi_f32x2(uint64_t d) { return __uint_as_float(uint32_t(d >> 32)); }
 
 constexpr int kVCompute = 256;
@@ -320,13 +341,14 @@ __global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
         const int slot = c % NSLOT;
         ok = mbar_wait(&full[slot], (c / NSLOT) & 1, abort_flag, &g_err_verify, 4u);
         if (ok) {
-          const float4* S4 = reinterpret_cast<const float4*>(smem + size_t(slot) * L::HALF);
+          const uint32_t s_row = smem_u32(smem + size_t(slot) * L::HALF) +
+                                 uint32_t((lrow0 * QUADS + quad) * 16);
+          const uint32_t kq_row = smem_u32(&d.kq[grp * RPG][0]);
 #pragma unroll 4
           for (int ii = 0; ii < RPG; ++ii) {
-            const int i = grp * RPG + ii;
-            const float4 hv = S4[(lrow0 + ii) * QUADS + quad];
-            const ulonglong2 p01 = *reinterpret_cast<const ulonglong2*>(&d.kq[i][0]);
-            const ulonglong2 p23 = *reinterpret_cast<const ulonglong2*>(&d.kq[i][1]);
+            const float4 hv = lds_f4(s_row + uint32_t(ii * QUADS * 16));
+            const ulonglong2 p01 = lds_u64x2(kq_row + uint32_t(ii * 32));
+            const ulonglong2 p23 = lds_u64x2(kq_row + uint32_t(ii * 32 + 16));
             const uint64_t kq2[kRows] = {p01.x, p01.y, p23.x, p23.y};  // (k_r[i], q_r[i])
             const float hs[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
@@ -346,15 +368,15 @@ __global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
       ok = pu == 0 || mbar_wait(&pempty[pb], (pu - 1) & 1, abort_flag, &g_err_verify, 4u);
       if (!__all_sync(0xffffffffu, ok)) break;
       if (!pad) {
-        float4* part = reinterpret_cast<float4*>(smem + L::PART + pb * L::PART_BYTES);
+        const uint32_t part = smem_u32(smem + L::PART + pb * L::PART_BYTES);
 #pragma unroll
         for (int r = 0; r < kRows; ++r) {
-          part[(grp * 2 * kRows + r) * QUADS + quad] =
-              make_float4(lo_f32x2(acc[0][r]), lo_f32x2(acc[1][r]), lo_f32x2(acc[2][r]),
-                          lo_f32x2(acc[3][r]));
-          part[(grp * 2 * kRows + kRows + r) * QUADS + quad] =
-              make_float4(hi_f32x2(acc[0][r]), hi_f32x2(acc[1][r]), hi_f32x2(acc[2][r]),
-                          hi_f32x2(acc[3][r]));
+          st_shared_v4(part + uint32_t(((grp * 2 * kRows + r) * QUADS + quad) * 16),
+                       uint32_t(acc[0][r]), uint32_t(acc[1][r]), uint32_t(acc[2][r]),
+                       uint32_t(acc[3][r]));
+          st_shared_v4(part + uint32_t(((grp * 2 * kRows + kRows + r) * QUADS + quad) * 16),
+                       uint32_t(acc[0][r] >> 32), uint32_t(acc[1][r] >> 32),
+                       uint32_t(acc[2][r] >> 32), uint32_t(acc[3][r] >> 32));
         }
       }
       __syncwarp();
@@ -383,13 +405,13 @@ __global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
 #pragma unroll
           for (int r = 0; r < kRows; ++r) o[((row0 + r) * H_v + h) * D + j] = 0;
         } else {
-          const float* pf = reinterpret_cast<const float*>(smem + L::PART + pb * L::PART_BYTES);
+          const uint32_t pf = smem_u32(smem + L::PART + pb * L::PART_BYTES) + uint32_t(j * 4);
           float a[kRows], bq[kRows], delta[kRows];
 #pragma unroll
           for (int r = 0; r < 2 * kRows; ++r) {
             float s2 = 0.f;
 #pragma unroll
-            for (int gg = 0; gg < GROUPS; ++gg) s2 += pf[(gg * 2 * kRows + r) * D + j];
+            for (int gg = 0; gg < GROUPS; ++gg) s2 += lds_f32(pf + uint32_t((gg * 2 * kRows + r) * D * 4));
             if (r < kRows)
               a[r] = s2;
             else
