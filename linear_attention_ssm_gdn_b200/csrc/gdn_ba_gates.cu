@@ -75,8 +75,9 @@ __global__ void __launch_bounds__(kBaThreads, 1)
     ba_gates_kernel(const __grid_constant__ CUtensorMap tmap_x,
                     const __grid_constant__ CUtensorMap tmap_w, const BaParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  // 1024-byte aligned start, kept as an offset from the __shared__ array so
+  // that accesses through it stay shared-space (not generic) loads and stores
+  uint8_t* smem = smem_raw + ((uint32_t(1024) - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int stages = p.stages;
   const uint32_t a_box = kBaBM * 128, b_box = uint32_t(p.n_pad) * 128;
   const uint32_t a_bytes = kBaNB * a_box;

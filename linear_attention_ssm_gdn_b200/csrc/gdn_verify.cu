@@ -155,8 +155,9 @@ __global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
   constexpr int QUADS = L::QUADS, GROUPS = L::GROUPS, RPG = L::RPG, NSLOT = L::NSLOT;
   constexpr int EPL = D / 32;  // elements of a row per lane (descriptor warps)
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
-                                             ~uintptr_t(127));
+  // 128-byte aligned start, kept as an offset from the __shared__ array so
+  // that accesses through it stay shared-space (not generic) loads and stores
+  uint8_t* smem = smem_raw + ((uint32_t(128) - (smem_u32(smem_raw) & 127u)) & 127u);
   VerifyDesc<D>* desc = reinterpret_cast<VerifyDesc<D>*>(smem + L::DESC);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BARS);
   uint64_t* empty = full + NSLOT;
