@@ -126,3 +126,44 @@ def test_python_binding_rejects_wrong_dtypes():
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(ImportError):
         _lib.load(str(tmp_path / "libgdn.so"))
+
+
+def test_verify_static_guards(lib):
+    """The no-allocation verify refuses bad arguments before it looks up its
+    static stash (so no CUDA call is made here)."""
+    ssf = lib.gdn_stash_seq_floats(48, 128, 128)
+    assert ssf == 48 * 4 * (128 + 4)
+    out = ctypes.c_void_p()
+
+    def call(batch=64, qks=2048, vs=6144, gbs=48, Hv=48, dk=128, dv=128, stash_out=True,
+             table=P, q=P):
+        return lib.gdn_verify_woa_static(table, q, P, qks, P, vs, P, P, gbs, P, batch, 16, Hv, dk,
+                                         dv, 1.0, P, ctypes.byref(out) if stash_out else NULL,
+                                         None)
+
+    assert call(stash_out=False) == _lib.GDN_ERR_NULL and "stash_out" in _err(lib)
+    assert call(table=NULL) == _lib.GDN_ERR_NULL
+    assert call(q=NULL) == _lib.GDN_ERR_NULL
+    assert call(Hv=47) == _lib.GDN_ERR_SHAPE
+    assert call(dk=128, dv=64) == _lib.GDN_ERR_SHAPE
+    assert call(batch=-1) == _lib.GDN_ERR_SHAPE
+    assert call(qks=2047) == _lib.GDN_ERR_STRIDE
+    assert call(vs=6143) == _lib.GDN_ERR_STRIDE
+    assert call(gbs=47) == _lib.GDN_ERR_STRIDE
+    limit = (2 * 1024 * 1024) // ssf
+    assert call(batch=limit + 1) == _lib.GDN_ERR_SHAPE and "exceeds the static stash" in _err(lib)
+
+
+def test_verify_stride_and_shape_guards(lib):
+    def call(qks=2048, vs=6144, gbs=48, batch=64, Hk=16, Hv=48, dk=128, dv=128, ssf=25344,
+             stash=P):
+        return lib.gdn_verify_woa(P, P, P, qks, P, vs, P, P, gbs, P, stash, ssf, batch, Hk, Hv,
+                                  dk, dv, 1.0, P, None)
+
+    assert call(qks=2047) == _lib.GDN_ERR_STRIDE
+    assert call(vs=6143) == _lib.GDN_ERR_STRIDE
+    assert call(gbs=47) == _lib.GDN_ERR_STRIDE
+    assert call(batch=-1) == _lib.GDN_ERR_SHAPE
+    assert call(Hv=40) == _lib.GDN_ERR_SHAPE  # not a multiple of H_k
+    assert call(dk=96, dv=96) == _lib.GDN_ERR_SHAPE
+    assert call(stash=P + 4) == _lib.GDN_ERR_ALIGN
