@@ -48,6 +48,30 @@ def _need(t: torch.Tensor, dtype, name: str):
         raise ValueError(f"{name}: must be a CUDA tensor")
 
 
+def _dense(t: torch.Tensor, dtype, shape, name: str):
+    """A CUDA tensor of this dtype and shape, dense in memory (the C ABI takes
+    no strides for it)."""
+    _need(t, dtype, name)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+def _gates(g: torch.Tensor, beta: torch.Tensor, rows: int, H_v: int) -> int:
+    """g, beta [rows, H_v] f32 with unit head stride and one shared row stride;
+    returns that stride."""
+    _need(g, torch.float32, "g")
+    _need(beta, torch.float32, "beta")
+    if tuple(g.shape) != (rows, H_v) or tuple(beta.shape) != (rows, H_v):
+        raise ValueError(f"g, beta: expected [{rows}, {H_v}]")
+    if H_v > 1 and (g.stride(1) != 1 or beta.stride(1) != 1):
+        raise ValueError("g, beta: the head dimension must be contiguous")
+    if rows > 1 and beta.stride(0) != g.stride(0):
+        raise ValueError("g and beta must share one row stride")
+    return int(g.stride(0)) if rows > 1 else H_v
+
+
 def version() -> str:
     return _lib.load().gdn_version().decode()
 
@@ -63,8 +87,14 @@ def gdn_ba_gates(x, w_ba, a_log, dt_bias, vheads_per_group, gate_out=None, strea
     nv = a_log.shape[0]
     if x.stride(1) != 1 or not w_ba.is_contiguous():
         raise ValueError("x rows and w_ba must be dense along K")
+    _dense(a_log, torch.float32, (nv,), "a_log")
+    _dense(dt_bias, torch.float32, (nv,), "dt_bias")
     if gate_out is None:
         gate_out = torch.empty(M, 2 * nv, dtype=torch.float32, device=x.device)
+    _need(gate_out, torch.float32, "gate_out")
+    if gate_out.dim() != 2 or gate_out.shape[0] != M or gate_out.shape[1] < 2 * nv or \
+            (2 * nv > 1 and gate_out.stride(1) != 1):
+        raise ValueError(f"gate_out: expected [{M}, >= {2 * nv}] with contiguous rows")
     k_stride = int(x.stride(0)) if M > 1 else K
     rc = lib.gdn_ba_gates(_ptr(x), k_stride, _ptr(w_ba), _ptr(a_log), _ptr(dt_bias),
                           _ptr(gate_out), int(gate_out.stride(0)), M, N, K, nv,
@@ -92,21 +122,22 @@ def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens, h0=None, hT=None, o=None, sc
     if _rows(k, "k", H_k, d_k) != qk_stride:
         raise ValueError("q and k must share one token stride")
     v_stride = _rows(v, "v", H_v, d_v)
-    if g.shape != (T, H_v) or beta.shape != (T, H_v) or g.stride(1) != 1 or beta.stride(1) != 1:
-        raise ValueError("g, beta: expected [T, H_v] with unit head stride")
-    gb_stride = int(g.stride(0)) if T > 1 else H_v
-    if T > 1 and beta.stride(0) != g.stride(0):
-        raise ValueError("g and beta must share one token stride")
+    gb_stride = _gates(g, beta, T, H_v)
+    _need(cu_seqlens, torch.int32, "cu_seqlens")
     num_seqs = cu_seqlens.shape[0] - 1
-    if cu_seqlens.dtype != torch.int32:
-        raise TypeError("cu_seqlens must be int32")
     if o is None:
         o = torch.empty(T, H_v, d_v, dtype=torch.bfloat16, device=q.device)
+    _dense(o, torch.bfloat16, (T, H_v, d_v), "o")
     if hT is None and store_final_state:
         hT = torch.empty(num_seqs, H_v, d_k, d_v, dtype=torch.float32, device=q.device)
+    for t, n in ((h0, "h0"), (hT, "hT")):
+        if t is not None:
+            _dense(t, torch.float32, (num_seqs, H_v, d_k, d_v), n)
     need = int(lib.gdn_chunk_prefill_workspace_bytes(T, num_seqs, H_k, H_v, d_k, d_v))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is not None and not workspace.is_cuda:
+        raise ValueError("workspace: must be a CUDA tensor")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = lib.gdn_chunk_prefill(_ptr(q), _ptr(k), qk_stride, _ptr(v), v_stride, _ptr(g),
                                _ptr(beta), gb_stride, _ptr(cu_seqlens), num_seqs, T, _ptr(h0),
@@ -125,19 +156,30 @@ def gdn_verify_woa(h_table, q, k, v, g, beta, engaged_flag, o=None, stash=None, 
     """K=4 verify. h_table: int64 CUDA tensor [batch] of state pointers.
     Returns (o [batch*4, H_v, d] bf16, stash f32 [batch, stash_seq_floats])."""
     lib = _lib.load()
+    _need(h_table, torch.int64, "h_table")
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    _need(engaged_flag, torch.int32, "engaged_flag")
     R, H_k, d_k = q.shape
     H_v, d_v = v.shape[1], v.shape[2]
     batch = h_table.shape[0]
     if R != 4 * batch:
         raise ValueError("q/k/v must hold 4 rows per sequence")
     qk_stride = _rows(q, "q", H_k, d_k)
+    if _rows(k, "k", H_k, d_k) != qk_stride:
+        raise ValueError("q and k must share one row stride")
     v_stride = _rows(v, "v", H_v, d_v)
-    gb_stride = int(g.stride(0)) if R > 1 else H_v
+    gb_stride = _gates(g, beta, R, H_v)
     ssf = gdn_stash_seq_floats(H_v, d_k, d_v)
     if o is None:
         o = torch.empty(R, H_v, d_v, dtype=torch.bfloat16, device=q.device)
+    _dense(o, torch.bfloat16, (R, H_v, d_v), "o")
     if stash is None:
         stash = torch.empty(batch, ssf, dtype=torch.float32, device=q.device)
+    _need(stash, torch.float32, "stash")
+    if stash.dim() != 2 or stash.shape[0] != batch or stash.shape[1] < ssf or \
+            (ssf > 1 and stash.stride(1) != 1):
+        raise ValueError(f"stash: expected [{batch}, >= {ssf}] with contiguous rows")
     rc = lib.gdn_verify_woa(_ptr(h_table), _ptr(q), _ptr(k), qk_stride, _ptr(v), v_stride,
                             _ptr(g), _ptr(beta), gb_stride, _ptr(o), _ptr(stash),
                             int(stash.stride(0)) if batch > 1 else ssf, batch, H_k, H_v, d_k,
@@ -149,7 +191,12 @@ def gdn_verify_woa(h_table, q, k, v, g, beta, engaged_flag, o=None, stash=None, 
 def gdn_fold(h_table, stash, na_tab, k, engaged_flag, H_v, k_rows=4, stream=None):
     """Apply the first na_tab[b] verified rows to each state (in place)."""
     lib = _lib.load()
+    _need(h_table, torch.int64, "h_table")
+    _need(stash, torch.float32, "stash")
+    _need(k, torch.bfloat16, "k")
+    _need(engaged_flag, torch.int32, "engaged_flag")
     batch = h_table.shape[0]
+    _dense(na_tab, torch.int32, (batch,), "na_tab")
     _, H_k, d = k.shape
     qk_stride = _rows(k, "k", H_k, d)
     ssf = int(stash.stride(0)) if batch > 1 else gdn_stash_seq_floats(H_v, d, d)
@@ -160,6 +207,7 @@ def gdn_fold(h_table, stash, na_tab, k, engaged_flag, H_v, k_rows=4, stream=None
 
 
 def gdn_flag_clear(engaged_flag, stream=None):
+    _need(engaged_flag, torch.int32, "engaged_flag")
     rc = _lib.load().gdn_flag_clear(_ptr(engaged_flag), _stream(stream))
     _lib.check("gdn_flag_clear", rc)
 

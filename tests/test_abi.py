@@ -167,3 +167,20 @@ def test_verify_stride_and_shape_guards(lib):
     assert call(Hv=40) == _lib.GDN_ERR_SHAPE  # not a multiple of H_k
     assert call(dk=96, dv=96) == _lib.GDN_ERR_SHAPE
     assert call(stash=P + 4) == _lib.GDN_ERR_ALIGN
+
+
+def test_python_binding_rejects_wrong_table_and_flag_dtypes():
+    """The binding checks dtypes before anything reaches the library: a float
+    pointer table or engaged word is refused on the host."""
+    import torch
+    from linear_attention_ssm_gdn_b200 import gdn_flag_clear, gdn_fold, gdn_verify_woa
+    bf = torch.zeros(4, 1, 64, dtype=torch.bfloat16)
+    f = torch.zeros(4, 1, dtype=torch.float32)
+    with pytest.raises(TypeError, match="h_table"):
+        gdn_verify_woa(torch.zeros(1, dtype=torch.float32), bf, bf, bf, f, f,
+                       torch.zeros(1, dtype=torch.int32))
+    with pytest.raises(TypeError, match="h_table"):
+        gdn_fold(torch.zeros(1, dtype=torch.int32), f, torch.zeros(1, dtype=torch.int32), bf,
+                 torch.zeros(1, dtype=torch.int32), 1)
+    with pytest.raises(TypeError, match="engaged_flag"):
+        gdn_flag_clear(torch.zeros(1, dtype=torch.float32))
