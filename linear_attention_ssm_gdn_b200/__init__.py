@@ -13,6 +13,7 @@ from .gdn import (  # noqa: F401
     gdn_flag_clear,
     gdn_fold,
     gdn_stash_seq_floats,
+    gdn_verify_parent,
     gdn_verify_woa,
     version,
 )

@@ -22,6 +22,7 @@ GDN_ERR_CUDA = 5
 GDN_ERR_ALIGN = 6
 GDN_FLAG_ENGAGED = 1
 GDN_FLAG_ERROR = 2
+GDN_FLAG_STASH_BAD = 4
 
 ERROR_NAMES = {1: "GDN_ERR_NULL", 2: "GDN_ERR_SHAPE", 3: "GDN_ERR_STRIDE",
                4: "GDN_ERR_WORKSPACE", 5: "GDN_ERR_CUDA", 6: "GDN_ERR_ALIGN"}
@@ -38,12 +39,19 @@ SIGNATURES = {
     "gdn_chunk_prefill_workspace_bytes": (_S, [_I, _I, _I, _I, _I, _I]),
     "gdn_chunk_prefill": (_I, [_P, _P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _P, _P, _P, _I, _I,
                                _I, _I, _F, _P, _S, _P]),
+    "gdn_chunk_prefill_x2": (_I, [_P, _P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _P, _P, _P, _I, _I,
+                                  _I, _I, _F, _P, _S, _P]),
+    "gdn_chunk_prefill_segmented_workspace_bytes": (_S, [_I, _I, _I, _I, _I, _I, _I]),
+    "gdn_chunk_prefill_segmented": (_I, [_P, _P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _P, _P, _P,
+                                         _I, _I, _I, _I, _F, _I, _I, _P, _S, _P]),
     "gdn_stash_seq_floats": (_I, [_I, _I, _I]),
     "gdn_verify_woa": (_I, [_P, _P, _P, _I, _P, _I, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I,
                             _F, _P, _P]),
     "gdn_verify_woa_static": (_I, [_P, _P, _P, _I, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I,
                                    _F, _P, _P, _P]),
-    "gdn_fold": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "gdn_verify_parent": (_I, [_P, _P, _P, _I, _P, _I, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I,
+                               _I, _F, _P]),
+    "gdn_fold": (_I, [_P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     "gdn_flag_clear": (_I, [_P, _P]),
     "gdn_debug_device_errors": (_I, [_P]),
 }

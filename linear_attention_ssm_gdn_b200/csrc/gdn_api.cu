@@ -151,38 +151,65 @@ int gdn_ba_gates(const uint16_t* x, int k_stride, const uint16_t* w_ba, const fl
                      "gdn_ba_gates");
 }
 
-size_t gdn_chunk_prefill_workspace_bytes(int total_tokens, int num_seqs, int H_k, int H_v,
-                                         int d_k, int d_v) {
-  (void)d_v;
-  return gdn::prefill_workspace_bytes(total_tokens, num_seqs, H_k, H_v, d_k);
+// Workspace of a prefill call with `segments` segments per sequence
+// (1: single level; the segmented path also needs the per-segment states).
+static size_t prefill_need(int total_tokens, int num_seqs, int H_v, int d_k, int segments) {
+  if (segments <= 1) return gdn::prefill_ring_bytes(num_seqs * H_v);
+  return gdn::prefill_segmented_workspace_bytes(total_tokens, num_seqs, H_v, d_k, segments);
 }
 
-int gdn_chunk_prefill(const uint16_t* q, const uint16_t* k, int qk_stride, const uint16_t* v,
-                      int v_stride, const float* g, const float* beta, int gb_stride,
-                      const int32_t* cu_seqlens, int num_seqs, int total_tokens,
-                      const float* h0, float* hT, uint16_t* o, int H_k, int H_v, int d_k,
-                      int d_v, float scale, void* workspace, size_t workspace_bytes,
-                      gdn_stream_t stream) {
-  const char* fn = "gdn_chunk_prefill";
+static int auto_segments(int total_tokens, int num_seqs, int H_v) {
+  if (num_seqs <= 0 || H_v <= 0 || total_tokens <= 0) return 1;
+  return gdn::prefill_auto_segments(total_tokens, num_seqs, H_v);
+}
+
+size_t gdn_chunk_prefill_workspace_bytes(int total_tokens, int num_seqs, int H_k, int H_v,
+                                         int d_k, int d_v) {
+  (void)H_k;
+  (void)d_v;
+  if (num_seqs <= 0 || H_v <= 0) return 0;
+  return prefill_need(total_tokens, num_seqs, H_v, d_k,
+                      auto_segments(total_tokens, num_seqs, H_v));
+}
+
+size_t gdn_chunk_prefill_segmented_workspace_bytes(int total_tokens, int num_seqs, int H_k,
+                                                   int H_v, int d_k, int d_v, int segments) {
+  (void)H_k;
+  (void)d_v;
+  if (num_seqs <= 0 || H_v <= 0 || segments < 1) return 0;
+  return prefill_need(total_tokens, num_seqs, H_v, d_k, segments);
+}
+
+// segments: >= 1 as given, 0 = the library's choice.
+static int chunk_prefill(const char* fn, int limbs, int segments, const uint16_t* q,
+                         const uint16_t* k, int qk_stride, const uint16_t* v, int v_stride,
+                         const float* g, const float* beta, int gb_stride,
+                         const int32_t* cu_seqlens, int num_seqs, int total_tokens,
+                         const float* h0, float* hT, uint16_t* o, int H_k, int H_v, int d_k,
+                         int d_v, float scale, void* workspace, size_t workspace_bytes,
+                         gdn_stream_t stream) {
+  const std::string f(fn);
   if (!q || !k || !v || !g || !beta || !cu_seqlens || !o)
-    return fail(GDN_ERR_NULL, "gdn_chunk_prefill: null q/k/v/g/beta/cu_seqlens/o");
+    return fail(GDN_ERR_NULL, f + ": null q/k/v/g/beta/cu_seqlens/o");
   int rc = check_heads(fn, H_k, H_v, d_k, d_v);
   if (rc != GDN_OK) return rc;
-  if (num_seqs <= 0) return fail(GDN_ERR_SHAPE, "gdn_chunk_prefill: num_seqs must be >= 1");
-  if (total_tokens < 0) return fail(GDN_ERR_SHAPE, "gdn_chunk_prefill: total_tokens < 0");
-  if (qk_stride < H_k * d_k) return fail(GDN_ERR_STRIDE, "gdn_chunk_prefill: qk_stride < H_k*d_k");
-  if (v_stride < H_v * d_v) return fail(GDN_ERR_STRIDE, "gdn_chunk_prefill: v_stride < H_v*d_v");
-  if (gb_stride < H_v) return fail(GDN_ERR_STRIDE, "gdn_chunk_prefill: gb_stride < H_v");
+  if (num_seqs <= 0) return fail(GDN_ERR_SHAPE, f + ": num_seqs must be >= 1");
+  if (total_tokens < 0) return fail(GDN_ERR_SHAPE, f + ": total_tokens < 0");
+  if (segments < 0 || segments > 64)
+    return fail(GDN_ERR_SHAPE, f + ": segments must be in 0..64");
+  if (qk_stride < H_k * d_k) return fail(GDN_ERR_STRIDE, f + ": qk_stride < H_k*d_k");
+  if (v_stride < H_v * d_v) return fail(GDN_ERR_STRIDE, f + ": v_stride < H_v*d_v");
+  if (gb_stride < H_v) return fail(GDN_ERR_STRIDE, f + ": gb_stride < H_v");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (h0 && !aligned16(h0)) || (hT && !aligned16(hT)))
-    return fail(GDN_ERR_ALIGN, "gdn_chunk_prefill: q/k/v/o/h0/hT not 16-byte aligned");
+    return fail(GDN_ERR_ALIGN, f + ": q/k/v/o/h0/hT not 16-byte aligned");
   if (qk_stride % 8 != 0 || v_stride % 8 != 0)
-    return fail(GDN_ERR_ALIGN, "gdn_chunk_prefill: qk_stride and v_stride must be multiples of 8");
-  const size_t need =
-      gdn::prefill_workspace_bytes(total_tokens, num_seqs, H_k, H_v, d_k);
+    return fail(GDN_ERR_ALIGN, f + ": qk_stride and v_stride must be multiples of 8");
+  const int S = segments == 0 ? auto_segments(total_tokens, num_seqs, H_v) : segments;
+  const size_t need = prefill_need(total_tokens, num_seqs, H_v, d_k, S);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need ||
                    (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
-    return fail(GDN_ERR_WORKSPACE, "gdn_chunk_prefill: workspace missing, small or unaligned");
+    return fail(GDN_ERR_WORKSPACE, f + ": workspace missing, small or unaligned");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (total_tokens == 0) {
     if (hT != nullptr && hT != h0) {
@@ -194,10 +221,67 @@ int gdn_chunk_prefill(const uint16_t* q, const uint16_t* k, int qk_stride, const
     gdn::clear_error();
     return GDN_OK;
   }
-  return cuda_status(gdn::launch_prefill(q, k, qk_stride, v, v_stride, g, beta, gb_stride,
-                                         cu_seqlens, num_seqs, total_tokens, h0, hT, o, H_k, H_v,
-                                         d_k, scale, workspace, s),
-                     fn);
+  gdn::PrefillCall c = {};
+  c.q = q;
+  c.k = k;
+  c.v = v;
+  c.qk_stride = qk_stride;
+  c.v_stride = v_stride;
+  c.g = g;
+  c.beta = beta;
+  c.gb_stride = gb_stride;
+  c.cu_seqlens = cu_seqlens;
+  c.num_seqs = num_seqs;
+  c.total_tokens = total_tokens;
+  c.h0 = h0;
+  c.hT = hT;
+  c.o = o;
+  c.H_k = H_k;
+  c.H_v = H_v;
+  c.D = d_k;
+  c.scale = scale;
+  c.limbs = limbs;
+  c.workspace = workspace;
+  if (S >= 2) return cuda_status(gdn::launch_prefill_segmented(c, S, workspace, s), fn);
+  return cuda_status(gdn::launch_prefill_call(c, s), fn);
+}
+
+int gdn_chunk_prefill(const uint16_t* q, const uint16_t* k, int qk_stride, const uint16_t* v,
+                      int v_stride, const float* g, const float* beta, int gb_stride,
+                      const int32_t* cu_seqlens, int num_seqs, int total_tokens,
+                      const float* h0, float* hT, uint16_t* o, int H_k, int H_v, int d_k,
+                      int d_v, float scale, void* workspace, size_t workspace_bytes,
+                      gdn_stream_t stream) {
+  return chunk_prefill("gdn_chunk_prefill", 1, 0, q, k, qk_stride, v, v_stride, g, beta,
+                       gb_stride, cu_seqlens, num_seqs, total_tokens, h0, hT, o, H_k, H_v, d_k,
+                       d_v, scale, workspace, workspace_bytes, stream);
+}
+
+int gdn_chunk_prefill_x2(const uint16_t* q, const uint16_t* k, int qk_stride, const uint16_t* v,
+                         int v_stride, const float* g, const float* beta, int gb_stride,
+                         const int32_t* cu_seqlens, int num_seqs, int total_tokens,
+                         const float* h0, float* hT, uint16_t* o, int H_k, int H_v, int d_k,
+                         int d_v, float scale, void* workspace, size_t workspace_bytes,
+                         gdn_stream_t stream) {
+  return chunk_prefill("gdn_chunk_prefill_x2", 2, 0, q, k, qk_stride, v, v_stride, g, beta,
+                       gb_stride, cu_seqlens, num_seqs, total_tokens, h0, hT, o, H_k, H_v, d_k,
+                       d_v, scale, workspace, workspace_bytes, stream);
+}
+
+int gdn_chunk_prefill_segmented(const uint16_t* q, const uint16_t* k, int qk_stride,
+                                const uint16_t* v, int v_stride, const float* g,
+                                const float* beta, int gb_stride, const int32_t* cu_seqlens,
+                                int num_seqs, int total_tokens, const float* h0, float* hT,
+                                uint16_t* o, int H_k, int H_v, int d_k, int d_v, float scale,
+                                int segments, int limbs, void* workspace,
+                                size_t workspace_bytes, gdn_stream_t stream) {
+  if (segments < 1)
+    return fail(GDN_ERR_SHAPE, "gdn_chunk_prefill_segmented: segments must be >= 1");
+  if (limbs != 1 && limbs != 2)
+    return fail(GDN_ERR_SHAPE, "gdn_chunk_prefill_segmented: limbs must be 1 or 2");
+  return chunk_prefill("gdn_chunk_prefill_segmented", limbs, segments, q, k, qk_stride, v,
+                       v_stride, g, beta, gb_stride, cu_seqlens, num_seqs, total_tokens, h0, hT,
+                       o, H_k, H_v, d_k, d_v, scale, workspace, workspace_bytes, stream);
 }
 
 int gdn_stash_seq_floats(int H_v, int d_k, int d_v) {
@@ -268,27 +352,63 @@ int gdn_verify_woa_static(float* const* h_table, const uint16_t* q, const uint16
                      fn);
 }
 
-int gdn_fold(float* const* h_table, const float* stash, const int32_t* na_tab,
-             const uint16_t* k, int qk_stride, uint32_t* engaged_flag, int k_rows, int batch,
-             int H_k, int H_v, int d_k, int d_v, int stash_seq_floats, gdn_stream_t stream) {
-  const char* fn = "gdn_fold";
-  if (!h_table || !stash || !na_tab || !k || !engaged_flag)
-    return fail(GDN_ERR_NULL, "gdn_fold: null table/stash/na_tab/k/flag");
+int gdn_verify_parent(float* const* h_table, const uint16_t* q, const uint16_t* k,
+                      int qk_stride, const uint16_t* v, int v_stride, const float* g,
+                      const float* beta, int gb_stride, uint16_t* o, float* const* hi_tables,
+                      int slab_entries, int batch, int H_k, int H_v, int d_k, int d_v,
+                      float scale, gdn_stream_t stream) {
+  const char* fn = "gdn_verify_parent";
+  if (!h_table) return fail(GDN_ERR_NULL, "gdn_verify_parent: null table");
+  if (!q || !k || !v || !g || !beta || !o)
+    return fail(GDN_ERR_NULL, "gdn_verify_parent: null q/k/v/g/beta/o");
   int rc = check_heads(fn, H_k, H_v, d_k, d_v);
   if (rc != GDN_OK) return rc;
-  if (k_rows != 4) return fail(GDN_ERR_SHAPE, "gdn_fold: k_rows must be 4");
-  if (batch < 0) return fail(GDN_ERR_SHAPE, "gdn_fold: batch < 0");
-  if (qk_stride < H_k * d_k) return fail(GDN_ERR_STRIDE, "gdn_fold: qk_stride < H_k*d_k");
-  if (stash_seq_floats < gdn_stash_seq_floats(H_v, d_k, d_v))
-    return fail(GDN_ERR_SHAPE, "gdn_fold: stash_seq_floats < gdn_stash_seq_floats()");
-  if (!aligned16(stash)) return fail(GDN_ERR_ALIGN, "gdn_fold: stash not 16-byte aligned");
+  if (batch < 0) return fail(GDN_ERR_SHAPE, "gdn_verify_parent: batch < 0");
+  if (hi_tables != nullptr && slab_entries < 3)
+    return fail(GDN_ERR_SHAPE, "gdn_verify_parent: slab_entries < k_rows - 1 = 3");
+  if (qk_stride < H_k * d_k || v_stride < H_v * d_v || gb_stride < H_v)
+    return fail(GDN_ERR_STRIDE, "gdn_verify_parent: a stride is shorter than its row");
   if (batch == 0) {
     gdn::clear_error();
     return GDN_OK;
   }
-  return cuda_status(gdn::launch_fold(h_table, stash, na_tab, k, qk_stride, engaged_flag, k_rows,
-                                      batch, H_k, H_v, d_k, stash_seq_floats,
-                                      reinterpret_cast<cudaStream_t>(stream)),
+  return cuda_status(gdn::launch_verify_parent(h_table, q, k, qk_stride, v, v_stride, g, beta,
+                                               gb_stride, o, hi_tables, slab_entries, batch, H_k,
+                                               H_v, d_k, scale,
+                                               reinterpret_cast<cudaStream_t>(stream)),
+                     fn);
+}
+
+int gdn_fold(float* const* h_table, const float* stash, const int32_t* na_tab,
+             const uint16_t* k, int qk_stride, float* const* hi_tables, int slab_entries,
+             uint32_t* engaged_flag, int k_rows, int batch, int H_k, int H_v, int d_k, int d_v,
+             int stash_seq_floats, gdn_stream_t stream) {
+  const char* fn = "gdn_fold";
+  if (!h_table || !na_tab || !engaged_flag)
+    return fail(GDN_ERR_NULL, "gdn_fold: null table/na_tab/flag");
+  if ((stash == nullptr) != (k == nullptr))
+    return fail(GDN_ERR_NULL, "gdn_fold: stash and k must both be given or both be NULL");
+  if (stash == nullptr && hi_tables == nullptr)
+    return fail(GDN_ERR_NULL, "gdn_fold: neither a stash (write-on-accept) nor hi_tables (parent)");
+  int rc = check_heads(fn, H_k, H_v, d_k, d_v);
+  if (rc != GDN_OK) return rc;
+  if (k_rows != 4) return fail(GDN_ERR_SHAPE, "gdn_fold: k_rows must be 4");
+  if (batch < 0) return fail(GDN_ERR_SHAPE, "gdn_fold: batch < 0");
+  if (hi_tables != nullptr && slab_entries < k_rows - 1)
+    return fail(GDN_ERR_SHAPE, "gdn_fold: slab_entries < k_rows - 1");
+  if (stash != nullptr) {
+    if (qk_stride < H_k * d_k) return fail(GDN_ERR_STRIDE, "gdn_fold: qk_stride < H_k*d_k");
+    if (stash_seq_floats < gdn_stash_seq_floats(H_v, d_k, d_v))
+      return fail(GDN_ERR_SHAPE, "gdn_fold: stash_seq_floats < gdn_stash_seq_floats()");
+    if (!aligned16(stash)) return fail(GDN_ERR_ALIGN, "gdn_fold: stash not 16-byte aligned");
+  }
+  if (batch == 0) {
+    gdn::clear_error();
+    return GDN_OK;
+  }
+  return cuda_status(gdn::launch_fold(h_table, stash, na_tab, k, qk_stride, hi_tables,
+                                      slab_entries, engaged_flag, k_rows, batch, H_k, H_v, d_k,
+                                      stash_seq_floats, reinterpret_cast<cudaStream_t>(stream)),
                      fn);
 }
 

@@ -259,6 +259,166 @@ __global__ void __launch_bounds__(kBaThreads, 1)
   if (warp == 0) tmem_dealloc(tmem, p.tmem_cols);
 }
 
+// ---------------------------------------------------------------------------
+// Few tokens (the batched decode step: M = 1 .. kBaSmallM rows).
+//
+// Page "ssm_ba_gates_hopper.rs", module doc: one CTA per token starves the
+// device when the step has few tokens (16 rows put 16 CTAs on the machine),
+// hence its token-count guard.  With M <= kBaSmallM the 128-row tensor-core
+// tile above would leave the GPU just as empty, so these shapes split the
+// OUTPUTS and the REDUCTION across CTAs instead of the tokens:
+//   grid = NG output groups of kBaSmallNPB outputs x KS K slices, as clusters
+//   of KS CTAs along K (one cluster per output group);
+//   warp w of a CTA computes output n0 + w for every token of the chunk: each
+//   lane holds 8 weights at a time and sweeps the token rows' matching 8
+//   activations (16-byte loads; the activation slice is shared by the
+//   group's 8 warps through L1), then a warp butterfly per token;
+//   rank r of the cluster stores its [M_chunk x 8] partial sums into rank 0's
+//   receive buffer (distributed shared memory), one cluster barrier publishes
+//   them, and rank 0 adds the KS partials in rank order (deterministic) and
+//   applies the gate epilogue of the large-M kernel.
+// Tokens beyond kBaSmallMB per CTA go to further grid rows (blockIdx.y).  CUDA
+// cores, f32 accumulation: at these sizes the weight read and the launch, not
+// the arithmetic, set the time.
+// ---------------------------------------------------------------------------
+constexpr int kBaSmallM = 64;     // largest M sent to the few-token kernel
+constexpr int kBaSmallMB = 64;    // tokens per CTA row
+constexpr int kBaSmallNPB = 8;    // outputs per CTA (one per warp)
+constexpr int kBaSmallKS = 8;     // CTAs per cluster along K (portable cluster size)
+
+struct BaSmallParams {
+  const uint16_t* x;
+  const uint16_t* w;
+  const float* a_log;
+  const float* dt_bias;
+  float* out;
+  int k_stride, gate_stride, M, N, K, nv, vpg, ks;
+};
+
+__global__ void __launch_bounds__(32 * kBaSmallNPB, 1)
+    ba_gates_small_kernel(const BaSmallParams p) {
+  __shared__ float recv[kBaSmallKS][kBaSmallMB][kBaSmallNPB];
+  const int rank = int(cluster_ctarank());
+  const int grp = int(cluster_id_x());
+  const int warp = int(threadIdx.x >> 5), lane = int(threadIdx.x & 31);
+  const int m0 = int(blockIdx.y) * kBaSmallMB;
+  const int mb = min(kBaSmallMB, p.M - m0);
+  const int n = grp * kBaSmallNPB + warp;
+  // K slice of this rank, in whole 8-column (16-byte) units
+  const int units = p.K / 8;
+  const int u0 = units * rank / p.ks, u1 = units * (rank + 1) / p.ks;
+  // every CTA of the cluster is running before any remote store lands
+  cluster_arrive_relaxed();
+  cluster_wait_acquire();
+  float acc[kBaSmallMB];
+#pragma unroll
+  for (int m = 0; m < kBaSmallMB; ++m) acc[m] = 0.0f;
+  if (n < p.N) {
+    const uint16_t* wrow = p.w + size_t(n) * p.K;
+    for (int u = u0 + lane; u < u1; u += 32) {
+      const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wrow) + u);
+      const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+      float wf[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        wf[2 * e] = __uint_as_float(ww[e] << 16);
+        wf[2 * e + 1] = __uint_as_float(ww[e] & 0xffff0000u);
+      }
+#pragma unroll
+      for (int m = 0; m < kBaSmallMB; ++m) {
+        if (m < mb) {
+          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(
+                                     p.x + size_t(m0 + m) * p.k_stride) + u);
+          const uint32_t xx[4] = {xv.x, xv.y, xv.z, xv.w};
+          float a = acc[m];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            a = fmaf(wf[2 * e], __uint_as_float(xx[e] << 16), a);
+            a = fmaf(wf[2 * e + 1], __uint_as_float(xx[e] & 0xffff0000u), a);
+          }
+          acc[m] = a;
+        }
+      }
+    }
+  }
+  // per-token butterfly; lane 0 pushes the warp's column into rank 0
+  const uint32_t base = mapa_shared(smem_u32(&recv[rank][0][warp]), 0u);
+#pragma unroll
+  for (int m = 0; m < kBaSmallMB; ++m) {
+    if (m < mb) {
+      float v = acc[m];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (lane == 0)
+        asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(base + uint32_t(m * kBaSmallNPB) * 4),
+                     "f"(v)
+                     : "memory");
+    }
+  }
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  if (rank != 0) return;
+  const int ng = min(kBaSmallNPB, p.N - grp * kBaSmallNPB);
+  for (int i = int(threadIdx.x); i < mb * ng; i += 32 * kBaSmallNPB) {
+    const int m = i / ng, j = i - m * ng;
+    float sum = 0.0f;
+    for (int q = 0; q < p.ks; ++q) sum += recv[q][m][j];  // rank order
+    const int nn = grp * kBaSmallNPB + j;
+    const int within = nn % (2 * p.vpg), g2 = nn / (2 * p.vpg);
+    float val;
+    int col;
+    if (within < p.vpg) {  // beta of v-head g2 * vpg + within
+      val = __frcp_rn(1.0f + __expf(-sum));
+      col = p.nv + g2 * p.vpg + within;
+    } else {               // gate of v-head g2 * vpg + within - vpg
+      const int vh = g2 * p.vpg + within - p.vpg;
+      const float z = sum + __ldg(&p.dt_bias[vh]);
+      val = -__expf(__ldg(&p.a_log[vh])) * (fmaxf(z, 0.0f) + log1p_unit(__expf(-fabsf(z))));
+      col = vh;
+    }
+    p.out[size_t(m0 + m) * p.gate_stride + col] = val;
+  }
+}
+
+static cudaError_t launch_ba_gates_small(const uint16_t* x, int k_stride, const uint16_t* w,
+                                         const float* a_log, const float* dt_bias, float* out,
+                                         int gate_stride, int M, int N, int K, int nv, int vpg,
+                                         cudaStream_t s) {
+  BaSmallParams p;
+  p.x = x;
+  p.w = w;
+  p.a_log = a_log;
+  p.dt_bias = dt_bias;
+  p.out = out;
+  p.k_stride = k_stride;
+  p.gate_stride = gate_stride;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.nv = nv;
+  p.vpg = vpg;
+  // K split: up to kBaSmallKS slices of at least 32 16-byte units each
+  int ks = K / 8 / 32;
+  ks = ks < 1 ? 1 : (ks > kBaSmallKS ? kBaSmallKS : ks);
+  p.ks = ks;
+  const int ngroups = (N + kBaSmallNPB - 1) / kBaSmallNPB;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ngroups * ks, (M + kBaSmallMB - 1) / kBaSmallMB);
+  cfg.blockDim = dim3(32 * kBaSmallNPB);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = ks;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 static int pow2_at_least(int x) {
   int c = 32;
   while (c < x) c <<= 1;
@@ -270,6 +430,9 @@ cudaError_t launch_ba_gates(const uint16_t* x, int k_stride, const uint16_t* w,
                             int gate_stride, int M, int N, int K, int nv, int vpg,
                             cudaStream_t s) {
   if (M == 0) return cudaSuccess;
+  if (M <= kBaSmallM)
+    return launch_ba_gates_small(x, k_stride, w, a_log, dt_bias, out, gate_stride, M, N, K, nv,
+                                 vpg, s);
   BaParams p;
   p.a_log = a_log;
   p.dt_bias = dt_bias;

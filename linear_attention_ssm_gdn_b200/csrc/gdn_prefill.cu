@@ -61,6 +61,11 @@ constexpr int kAS = 68;        // f32 row stride of the A / T scratch (16-byte r
 constexpr int kRing = 4;       // ring entries per spine
 constexpr int kMaxSpines = 256;
 constexpr int kSpineSync = 288;  // the spine's per-chunk barriers: 8 state warps + the issuer warp
+// Largest rise of the cumulative gate within a chunk (G_r - G_s, s <= r) that
+// keeps every decay factor finite in f32 (e^88 overflows); a rise above it
+// sets kErrGateRise in the prefill's device error word.
+constexpr float kGateRise = 80.f;
+constexpr uint32_t kErrGateRise = 64u;
 
 // ---- ring entry (workspace): W (rows r, two 64-column d_k boxes) | U^T | Aqk | gate factors
 constexpr uint32_t G_W = 0, G_U = 16384, G_AQK = 32768, G_GATE = 40960;
@@ -158,7 +163,15 @@ struct Params {
   const int32_t* cu_seqlens;
   const float* h0;
   float* hT;
-  uint16_t* o;
+  uint16_t* o;  // NULL: outputs not stored
+  // Optional per-sequence overrides (the segment-parallel scan runs the
+  // kernel over segments of the caller's sequences): token ranges [x, y),
+  // initial-state and final-state pointers ([H_v, D, D] each; NULL entry =
+  // zeros / not stored), and v read as zeros.
+  const int2* seg;
+  const float* const* h0_tab;
+  float* const* hT_tab;
+  int v_zero;
   uint32_t* flags;  // abort line + S * kRing flag lines
   uint8_t* ring;    // S * kRing entries of SLOT_G bytes
   int gb_stride, num_seqs, total_tokens, H_k, H_v, D;
@@ -177,6 +190,12 @@ __device__ __forceinline__ uint8_t* ring_entry(const Params& p, int s, int e) {
 }
 
 __device__ __forceinline__ void seq_range(const Params& p, int n, int& b, int& e) {
+  if (p.seg != nullptr) {
+    const int2 r = p.seg[n];
+    b = min(max(r.x, 0), p.total_tokens);
+    e = min(max(r.y, b), p.total_tokens);
+    return;
+  }
   b = min(max(p.cu_seqlens[n], 0), p.total_tokens);
   e = min(max(p.cu_seqlens[n + 1], b), p.total_tokens);
 }
@@ -285,6 +304,20 @@ __device__ __forceinline__ void st_row64_bf16(uint32_t tile, uint32_t row, const
     st_shared_v4(tile + sw128_offset(row, c * 16), pack_bf16x2(x[8 * c + 0], x[8 * c + 1]),
                  pack_bf16x2(x[8 * c + 2], x[8 * c + 3]), pack_bf16x2(x[8 * c + 4], x[8 * c + 5]),
                  pack_bf16x2(x[8 * c + 6], x[8 * c + 7]));
+}
+
+// The low bf16 limb of 64 f32 values: x - bf16(x), rounded to bf16, as one
+// 128-byte row of a 128B-swizzled tile (the second limb of the state copy).
+__device__ __forceinline__ void st_row64_bf16_lo(uint32_t tile, uint32_t row, const float* x) {
+  float r[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      r[e] = x[8 * c + e] - __bfloat162float(__float2bfloat16_rn(x[8 * c + e]));
+    st_shared_v4(tile + sw128_offset(row, c * 16), pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]),
+                 pack_bf16x2(r[4], r[5]), pack_bf16x2(r[6], r[7]));
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -435,6 +468,11 @@ __device__ __forceinline__ void invert_unit_lower64(float* M, float* Xs, int p, 
 
 using namespace pf;
 
+// kLimbs = 1: the state enters the H-dependent MMA as one bf16 copy; 2: as
+// two bf16 limbs hi + lo (page "ssm_gdn_tc_route.rs": the _tcfuse spine uses
+// one limb of S_c, the _tcfuse_x2 spine two), the low limb staged in the Vn
+// buffers, which that MMA does not read.
+template <int kLimbs>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -564,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int id = lane + 32 * m, i = id >> 2, seg = id & 3;
             const int r = r0 + i;
             const uint4 val = ld_shared_v4(ostg + uint32_t(i) * 64 + uint32_t(seg) * 16);
-            if (okE && r < Ll && e0 < D)
+            if (okE && r < Ll && e0 < D && p.o != nullptr)
               *reinterpret_cast<uint4*>(p.o + (size_t(t0l + r) * p.H_v + hl) * D + e0 + seg * 8) = val;
           }
         }
@@ -578,11 +616,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = u / p.H_v, h = u % p.H_v;
         int tb, te;
         seq_range(p, n, tb, te);
-        const size_t state_off = (size_t(n) * p.H_v + h) * size_t(D) * D;
+        const size_t seq_off = size_t(n) * p.H_v * size_t(D) * D, head_off = size_t(h) * D * D;
+        const float* h0b = p.h0_tab != nullptr ? p.h0_tab[n]
+                                               : (p.h0 != nullptr ? p.h0 + seq_off : nullptr);
+        float* hTb = p.hT_tab != nullptr ? p.hT_tab[n] : (p.hT != nullptr ? p.hT + seq_off : nullptr);
         bool agreed = true;
         float H[64];
         {
-          const float* h0 = (p.h0 != nullptr && jv) ? p.h0 + state_off + j : nullptr;
+          const float* h0 = (h0b != nullptr && jv) ? h0b + head_off + j : nullptr;
 #pragma unroll
           for (int i = 0; i < 64; ++i)
             H[i] = (h0 != nullptr && 64 * hh + i < D) ? h0[size_t(64 * hh + i) * D] : 0.f;
@@ -613,6 +654,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (tid < 64) eg_s[64 * st + tid] = sg[tid] * p.scale;
           else if (tid < 128) ecg_s[64 * st + tid - 64] = sg[tid];
           st_row64_bf16(sbase + S_HT + uint32_t(hh) * 16384, uint32_t(j), H);
+          if constexpr (kLimbs == 2) {
+            // the previous chunk's O2 MMA reads the Vn buffers: done first
+            if (c > c_first)
+              ok = mbar_wait(&bars[SB_OFULL + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag, err,
+                             16u) && ok;
+            st_row64_bf16_lo(sbase + S_VN + uint32_t(hh) * 16384, uint32_t(j), H);
+          }
           fence_proxy_async_smem();
           tc_fence_before();
           if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts [W; Q]
@@ -700,8 +748,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
         }
-        if (p.hT != nullptr && jv) {
-          float* hT = p.hT + state_off + j;
+        if (hTb != nullptr && jv) {
+          float* hT = hTb + head_off + j;
 #pragma unroll
           for (int i = 0; i < 64; ++i)
             if (64 * hh + i < D) hT[size_t(64 * hh + i) * D] = H[i];
@@ -735,6 +783,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
               mma_bf16_ss(tmem + ST_VO + 128u * st, make_sdesc_sw128(sbase + S_HT + off, 16, 1024),
                           make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_vo, kk > 0);
+            }
+            if constexpr (kLimbs == 2) {
+              for (int kk = 0; kk < ksteps_d; ++kk) {
+                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                mma_bf16_ss(tmem + ST_VO + 128u * st, make_sdesc_sw128(sbase + S_VN + off, 16, 1024),
+                            make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_vo, 1u);
+              }
             }
             mma_commit(&bars[SB_VOFULL]);
             mma_commit(&bars[SB_AE + st]);
@@ -856,13 +911,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (lane == 0) {
           uint64_t* fb = &bars[PB_KQVF + t];
-          mbar_arrive_expect_tx(fb, uint32_t(nbox) * 3 * 8192);
+          mbar_arrive_expect_tx(fb, uint32_t(nbox) * (p.v_zero ? 2 : 3) * 8192);
           uint8_t* set = smem + t * P_SET;
           const int hk = it.h / vpg;
           for (int b2 = 0; b2 < nbox; ++b2) {
             tma_load_3d(set + P_KQ + b2 * 16384, &tm_k, fb, b2 * 64, hk, it.t0);
             tma_load_3d(set + P_KQ + b2 * 16384 + 8192, &tm_q, fb, b2 * 64, hk, it.t0);
-            tma_load_3d(set + P_V + b2 * 8192, &tm_v, fb, b2 * 64, it.h, it.t0);
+            // v read as zeros: the V boxes keep the zeros of the start-up clear
+            if (!p.v_zero) tma_load_3d(set + P_V + b2 * 8192, &tm_v, fb, b2 * 64, it.h, it.t0);
           }
           last_k = k;
         }
@@ -885,6 +941,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float G1 = s2, G0 = s2 - a1;       // G_{r0+1}, G_{r0}
           const float GC = __shfl_sync(0xffffffffu, G1, 31);
+          {
+            // Every decay factor is e^{G_r - G_s} for some s <= r (G_{-1} = 0):
+            // finite while the gates rise by at most kGateRise after any row
+            // of the chunk.  A larger rise (positive gates) is flagged.
+            float mn = fminf(fminf(G0, G1), 0.f);
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+              const float y = __shfl_up_sync(0xffffffffu, mn, off);
+              if (lane >= off) mn = fminf(mn, y);
+            }
+            float before = __shfl_up_sync(0xffffffffu, mn, 1);  // min over rows < r0
+            if (lane == 0) before = 0.f;
+            const float m0 = fminf(before, G0), m1 = fminf(m0, G1);
+            float rise = fmaxf(G0 - m0, G1 - m1);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+              rise = fmaxf(rise, __shfl_xor_sync(0xffffffffu, rise, off));
+            if (lane == 0 && !(rise <= kGateRise)) atomicOr(err, kErrGateRise);
+          }
           // G at the start of this pair's 16-row block: row r0 & ~15 is the
           // first row of lane (r0 & ~15) / 2
           const float Gb = __shfl_sync(0xffffffffu, G0, (r0 & ~15) >> 1);
@@ -1195,9 +1270,9 @@ int resident_ctas() {
   int* slot = (dev >= 0 && dev < 64) ? &cache[dev] : nullptr;
   if (slot != nullptr && *slot > 0) return *slot;
   int per_sm = 0;
-  cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaFuncSetAttribute(prefill_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        int(kSmemAlloc));
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prefill_kernel, kThreads,
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prefill_kernel<1>, kThreads,
                                                     kSmemAlloc) != cudaSuccess) {
     cudaGetLastError();
     per_sm = 0;
@@ -1224,59 +1299,64 @@ size_t flag_bytes(int S) { return (size_t(1 + S * kRing) * kFlagLine + 1023) / 1
 
 }  // namespace
 
-size_t prefill_workspace_bytes(int total_tokens, int num_seqs, int H_k, int H_v, int D) {
-  (void)total_tokens;
-  (void)H_k;
-  (void)D;
+size_t prefill_ring_bytes(int units) {
   int G = 0, S = 0;
-  plan(num_seqs * H_v, &G, &S);
+  plan(units, &G, &S);
   return flag_bytes(S) + size_t(S) * kRing * SLOT_G;
 }
 
-cudaError_t launch_prefill(const uint16_t* q, const uint16_t* k, int qk_stride,
-                           const uint16_t* v, int v_stride, const float* g, const float* beta,
-                           int gb_stride, const int32_t* cu_seqlens, int num_seqs,
-                           int total_tokens, const float* h0, float* hT, uint16_t* o, int H_k,
-                           int H_v, int D, float scale, void* workspace, cudaStream_t s) {
+int prefill_spine_budget() {
+  int G = 0, S = 0;
+  plan(1 << 20, &G, &S);
+  return S;
+}
+
+cudaError_t launch_prefill_call(const PrefillCall& c, cudaStream_t s) {
+  const int D = c.D;
   CUtensorMap tq, tk, tv;
   {
-    uint64_t dims[3] = {uint64_t(D), uint64_t(H_k), uint64_t(total_tokens)};
-    uint64_t strides[2] = {uint64_t(D) * 2, uint64_t(qk_stride) * 2};
+    uint64_t dims[3] = {uint64_t(D), uint64_t(c.H_k), uint64_t(c.total_tokens)};
+    uint64_t strides[2] = {uint64_t(D) * 2, uint64_t(c.qk_stride) * 2};
     uint32_t box[3] = {64, 1, 64};
-    if (!encode_tmap_bf16(&tq, q, 3, dims, strides, box, true)) return cudaErrorInvalidValue;
-    if (!encode_tmap_bf16(&tk, k, 3, dims, strides, box, true)) return cudaErrorInvalidValue;
+    if (!encode_tmap_bf16(&tq, c.q, 3, dims, strides, box, true)) return cudaErrorInvalidValue;
+    if (!encode_tmap_bf16(&tk, c.k, 3, dims, strides, box, true)) return cudaErrorInvalidValue;
   }
   {
-    uint64_t dims[3] = {uint64_t(D), uint64_t(H_v), uint64_t(total_tokens)};
-    uint64_t strides[2] = {uint64_t(D) * 2, uint64_t(v_stride) * 2};
+    uint64_t dims[3] = {uint64_t(D), uint64_t(c.H_v), uint64_t(c.total_tokens)};
+    uint64_t strides[2] = {uint64_t(D) * 2, uint64_t(c.v_stride) * 2};
     uint32_t box[3] = {64, 1, 64};
-    if (!encode_tmap_bf16(&tv, v, 3, dims, strides, box, true)) return cudaErrorInvalidValue;
+    if (!encode_tmap_bf16(&tv, c.v, 3, dims, strides, box, true)) return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kernel = c.limbs == 2 ? prefill_kernel<2> : prefill_kernel<1>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(kSmemAlloc));
   if (e != cudaSuccess) return e;
   int G = 0, S = 0;
-  plan(num_seqs * H_v, &G, &S);
+  plan(c.num_seqs * c.H_v, &G, &S);
   if (G < 2) return cudaErrorCooperativeLaunchTooLarge;
   Params p;
-  p.g = g;
-  p.beta = beta;
-  p.cu_seqlens = cu_seqlens;
-  p.h0 = h0;
-  p.hT = hT;
-  p.o = o;
-  p.flags = static_cast<uint32_t*>(workspace);
-  p.ring = static_cast<uint8_t*>(workspace) + flag_bytes(S);
-  p.gb_stride = gb_stride;
-  p.num_seqs = num_seqs;
-  p.total_tokens = total_tokens;
-  p.H_k = H_k;
-  p.H_v = H_v;
+  p.g = c.g;
+  p.beta = c.beta;
+  p.cu_seqlens = c.cu_seqlens;
+  p.h0 = c.h0;
+  p.hT = c.hT;
+  p.o = c.o;
+  p.seg = c.seg;
+  p.h0_tab = c.h0_tab;
+  p.hT_tab = c.hT_tab;
+  p.v_zero = c.v_zero;
+  p.flags = static_cast<uint32_t*>(c.workspace);
+  p.ring = static_cast<uint8_t*>(c.workspace) + flag_bytes(S);
+  p.gb_stride = c.gb_stride;
+  p.num_seqs = c.num_seqs;
+  p.total_tokens = c.total_tokens;
+  p.H_k = c.H_k;
+  p.H_v = c.H_v;
   p.D = D;
   p.S = S;
-  p.scale = scale;
+  p.scale = c.scale;
   // The hand-off counters start from zero on every launch.
-  e = cudaMemsetAsync(workspace, 0, flag_bytes(S), s);
+  e = cudaMemsetAsync(c.workspace, 0, flag_bytes(S), s);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G);
@@ -1288,7 +1368,7 @@ cudaError_t launch_prefill(const uint16_t* q, const uint16_t* k, int qk_stride,
   attr.val.cooperative = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, prefill_kernel, tq, tk, tv, p);
+  e = cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

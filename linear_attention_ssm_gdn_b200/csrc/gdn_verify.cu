@@ -17,6 +17,12 @@
 // Fold.  With na = na_tab[b] in 1..4 (and the engaged bit set):
 //   H[i][j] <- e^{G_{na-1}} H[i][j] + sum_{r<na} e^{G_{na-1} - G_r} k_r[i] delta_r[j]
 // reading and writing each state element once; na = 0 touches nothing.
+// Parent (non write-on-accept) verify.  The same four rows, but the states are
+// written: the state after row r, Hi(r), goes to the intermediate slab
+// hi_tables[b * slab_entries + r] for r < 3 and the state after all four rows
+// replaces the live state.  With the engaged word clear the fold then
+// restores Hi(na - 1) into the live state on a partial accept (1 <= na < 4).
+//
 // All of this is HBM-bound CUDA-core work: 4 rows give 8 flops per state
 // element, far below the tensor-core ridge.
 #include <cuda_bf16.h>
@@ -38,6 +44,7 @@ static __device__ __align__(256) float g_static_stash[kStaticStashFloats];
 
 constexpr uint32_t kFlagEngaged = 1u;
 constexpr uint32_t kFlagError = 2u;
+constexpr uint32_t kFlagStashBad = 4u;  // a verify gave up before its whole stash was written
 constexpr int kRows = 4;
 
 __device__ __forceinline__ float bf16_at(const uint16_t* p) {
@@ -443,6 +450,9 @@ __global__ void __launch_bounds__(kVBlock, 1) verify_kernel(
     if (!ok) *abort_flag = 1;
   }
   __syncthreads();
+  // A CTA that gave up (a bounded wait ran out) left part of its stash
+  // unwritten: say so in the engaged word, so that the fold applies nothing.
+  if (tid == 0 && *abort_flag) atomicOr(flag, kFlagError | kFlagStashBad);
 }
 
 // grid = (H_v, batch); block = 256.  Each thread loads all of its 16-byte
@@ -452,18 +462,40 @@ __global__ void __launch_bounds__(kVThreads) fold_kernel(float* const* __restric
                                                          const float* __restrict__ stash,
                                                          const int32_t* __restrict__ na_tab,
                                                          const uint16_t* __restrict__ k,
-                                                         int qk_stride, uint32_t* flag, int H_k,
-                                                         int H_v, int stash_seq_floats) {
+                                                         int qk_stride,
+                                                         float* const* __restrict__ hi_tables,
+                                                         int slab_entries, uint32_t* flag,
+                                                         int H_k, int H_v, int stash_seq_floats) {
   constexpr int QUADS = D / 4;
   constexpr int PER = D * QUADS / kVThreads;  // quads per thread (16 resp. 4)
   __shared__ float ks[kRows][D], dl[kRows][D], coef[kRows], cdecay;
   const int h = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x;
-  if ((*(volatile uint32_t*)flag & kFlagEngaged) == 0u) return;
+  const uint32_t fw = *(volatile uint32_t*)flag;
   const int na = na_tab[b];
   float* H = h_table[b];
+  if ((fw & kFlagEngaged) == 0u) {
+    // The parent verify ran: the live state holds the state after all four
+    // rows; a partial accept restores the kept intermediate Hi(na - 1).
+    if (hi_tables == nullptr || H == nullptr || na == kRows) return;
+    const float* src =
+        (na >= 1 && na < kRows) ? hi_tables[size_t(b) * slab_entries + (na - 1)] : nullptr;
+    if (src == nullptr) {  // na out of range (0 included: the pre-verify state is gone)
+      if (h == 0 && tid == 0) atomicOr(flag, kFlagError);
+      return;
+    }
+    const float4* s4 = reinterpret_cast<const float4*>(src + size_t(h) * D * D);
+    float4* d4 = reinterpret_cast<float4*>(H + size_t(h) * D * D);
+    float4 hv[PER];
+#pragma unroll
+    for (int m = 0; m < PER; ++m) hv[m] = s4[tid + kVThreads * m];
+#pragma unroll
+    for (int m = 0; m < PER; ++m) d4[tid + kVThreads * m] = hv[m];
+    return;
+  }
+  if ((fw & kFlagStashBad) != 0u) return;
   if (na == 0 || H == nullptr) return;
-  if (na < 0 || na > kRows) {
+  if (na < 0 || na > kRows || stash == nullptr || k == nullptr) {
     if (h == 0 && tid == 0) atomicOr(flag, kFlagError);
     return;
   }
@@ -504,6 +536,182 @@ __global__ void __launch_bounds__(kVThreads) fold_kernel(float* const* __restric
   }
 }
 
+// ---------------------------------------------------------------------------
+// Parent verify: grid = (H_v, batch), 256 threads, one (sequence, v-head) item
+// per CTA.  Pass 1 reduces the state columns against the four k and q rows
+// (thread = (column j, row slice)); thread j < D then runs the 4-step column
+// recurrence of the header (o rows and delta rows); pass 2 writes Hi(0..2) to
+// the slabs and Hi(3) over the live state, each element
+//   Hi(r)[i][j] = e^{G_r} H0[i][j] + sum_{s<=r} e^{G_r - G_s} k_s[i] delta_s[j],
+// re-reading H0 (from L2) as 16-byte quads.  No waits: nothing can hang.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) verify_parent_kernel(
+    float* const* __restrict__ h_table, const uint16_t* __restrict__ q,
+    const uint16_t* __restrict__ k, int qk_stride, const uint16_t* __restrict__ v, int v_stride,
+    const float* __restrict__ g, const float* __restrict__ beta, int gb_stride,
+    uint16_t* __restrict__ o, float* const* __restrict__ hi_tables, int slab_entries, int H_k,
+    int H_v, float scale) {
+  constexpr int NT = 256, QUADS = D / 4, SLICES = NT / D, RPS = D / SLICES;
+  __shared__ float ks[kRows][D], qs[kRows][D], dl[kRows][D];
+  __shared__ float part[SLICES][2 * kRows][D];
+  __shared__ float cK[kRows][kRows], cQ[kRows][kRows], cf[kRows][kRows];
+  __shared__ float eG[kRows], bt[kRows], Gc[kRows];
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int hk = h / (H_v / H_k);
+  float* live = h_table[b];
+  const size_t row0 = size_t(b) * kRows;
+  if (live == nullptr) {  // padding sequence: zero outputs, no state
+    for (int idx = tid; idx < kRows * D; idx += NT) {
+      const int r = idx / D, j = idx % D;
+      o[((row0 + r) * H_v + h) * D + j] = 0;
+    }
+    return;
+  }
+  const float* H0 = live + size_t(h) * D * D;
+  for (int idx = tid; idx < kRows * D; idx += NT) {
+    const int r = idx / D, i = idx % D;
+    ks[r][i] = bf16_at(k + (row0 + r) * qk_stride + size_t(hk) * D + i);
+    qs[r][i] = bf16_at(q + (row0 + r) * qk_stride + size_t(hk) * D + i);
+  }
+  __syncthreads();
+  // k_s . k_r and k_s . q_r: warp w takes the four products 4 w .. 4 w + 3
+  // (the first 16 are k.k, the next 16 k.q); the gates on the side
+  for (int m = 0; m < 4; ++m) {
+    const int pidx = 4 * warp + m, sr = pidx & 15, s2 = sr >> 2, r = sr & 3;
+    const float* other = pidx < 16 ? ks[r] : qs[r];
+    float acc = 0.f;
+    for (int i = lane; i < D; i += 32) acc = fmaf(ks[s2][i], other[i], acc);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+      if (pidx < 16)
+        cK[s2][r] = acc;
+      else
+        cQ[s2][r] = acc;
+    }
+  }
+  if (tid == 0) {
+    float run = 0.f;
+    for (int r = 0; r < kRows; ++r) {
+      run += g[(row0 + r) * gb_stride + h];
+      Gc[r] = run;
+      bt[r] = beta[(row0 + r) * gb_stride + h];
+      eG[r] = __expf(run);
+    }
+  }
+  // pass 1: column partials a_r[j] = sum_i H0[i][j] k_r[i], b_r[j] likewise with q_r
+  {
+    const int j = tid % D, sl = tid / D;
+    float a[kRows] = {0.f, 0.f, 0.f, 0.f}, bq[kRows] = {0.f, 0.f, 0.f, 0.f};
+    for (int ii = 0; ii < RPS; ++ii) {
+      const int i = sl * RPS + ii;
+      const float hv = H0[size_t(i) * D + j];
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) {
+        a[r] = fmaf(hv, ks[r][i], a[r]);
+        bq[r] = fmaf(hv, qs[r][i], bq[r]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      part[sl][r][j] = a[r];
+      part[sl][kRows + r][j] = bq[r];
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {  // decay factors of the pair products (scalars, once)
+    for (int s2 = 0; s2 < kRows; ++s2)
+      for (int r = 0; r < kRows; ++r) {
+        const float e = __expf(Gc[r] - Gc[s2]);
+        cK[s2][r] = s2 < r ? e * cK[s2][r] : 0.f;
+        cQ[s2][r] = s2 <= r ? e * cQ[s2][r] : 0.f;
+        cf[r][s2] = s2 <= r ? e : 0.f;
+      }
+  }
+  __syncthreads();
+  if (tid < D) {
+    const int j = tid;
+    float a[kRows], bq[kRows], delta[kRows];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      float x = 0.f, y = 0.f;
+#pragma unroll
+      for (int sl = 0; sl < SLICES; ++sl) {
+        x += part[sl][r][j];
+        y += part[sl][kRows + r][j];
+      }
+      a[r] = x;
+      bq[r] = y;
+    }
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      float pred = eG[r] * a[r];
+#pragma unroll
+      for (int s2 = 0; s2 < r; ++s2) pred += cK[s2][r] * delta[s2];
+      delta[r] = bt[r] * (bf16_at(v + (row0 + r) * v_stride + size_t(h) * D + j) - pred);
+      float out = eG[r] * bq[r];
+#pragma unroll
+      for (int s2 = 0; s2 <= r; ++s2) out += cQ[s2][r] * delta[s2];
+      o[((row0 + r) * H_v + h) * D + j] = __bfloat16_as_ushort(__float2bfloat16_rn(scale * out));
+      dl[r][j] = delta[r];
+    }
+  }
+  __syncthreads();
+  // pass 2: the four states; the live state is written last (H0 is re-read
+  // from it until then, and every read of a quad precedes its own write)
+  float* dst[kRows];
+#pragma unroll
+  for (int r = 0; r < kRows - 1; ++r)
+    dst[r] = hi_tables != nullptr ? hi_tables[size_t(b) * slab_entries + r] : nullptr;
+  dst[kRows - 1] = live;
+  const float4* H04 = reinterpret_cast<const float4*>(H0);
+  for (int idx = tid; idx < D * QUADS; idx += NT) {
+    const int i = idx / QUADS, j4 = idx % QUADS;
+    const float4 h0v = H04[idx];
+    float kv[kRows];
+#pragma unroll
+    for (int s2 = 0; s2 < kRows; ++s2) kv[s2] = ks[s2][i];
+    float4 out[kRows];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      float x0 = eG[r] * h0v.x, x1 = eG[r] * h0v.y, x2 = eG[r] * h0v.z, x3 = eG[r] * h0v.w;
+#pragma unroll
+      for (int s2 = 0; s2 <= r; ++s2) {
+        const float c = cf[r][s2] * kv[s2];
+        x0 = fmaf(c, dl[s2][4 * j4 + 0], x0);
+        x1 = fmaf(c, dl[s2][4 * j4 + 1], x1);
+        x2 = fmaf(c, dl[s2][4 * j4 + 2], x2);
+        x3 = fmaf(c, dl[s2][4 * j4 + 3], x3);
+      }
+      out[r] = make_float4(x0, x1, x2, x3);
+    }
+#pragma unroll
+    for (int r = 0; r < kRows; ++r)
+      if (dst[r] != nullptr)
+        reinterpret_cast<float4*>(dst[r] + size_t(h) * D * D)[idx] = out[r];
+  }
+}
+
+cudaError_t launch_verify_parent(float* const* h_table, const uint16_t* q, const uint16_t* k,
+                                 int qk_stride, const uint16_t* v, int v_stride, const float* g,
+                                 const float* beta, int gb_stride, uint16_t* o,
+                                 float* const* hi_tables, int slab_entries, int batch, int H_k,
+                                 int H_v, int D, float scale, cudaStream_t s) {
+  if (batch == 0) return cudaSuccess;
+  dim3 grid(H_v, batch);
+  if (D == 128)
+    verify_parent_kernel<128><<<grid, 256, 0, s>>>(h_table, q, k, qk_stride, v, v_stride, g,
+                                                   beta, gb_stride, o, hi_tables, slab_entries,
+                                                   H_k, H_v, scale);
+  else
+    verify_parent_kernel<64><<<grid, 256, 0, s>>>(h_table, q, k, qk_stride, v, v_stride, g, beta,
+                                                  gb_stride, o, hi_tables, slab_entries, H_k,
+                                                  H_v, scale);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_flag_clear(uint32_t* flag, cudaStream_t s) {
   flag_clear_kernel<<<1, 32, 0, s>>>(flag);
   return cudaGetLastError();
@@ -538,17 +746,18 @@ cudaError_t launch_verify(float* const* h_table, const uint16_t* q, const uint16
 }
 
 cudaError_t launch_fold(float* const* h_table, const float* stash, const int32_t* na_tab,
-                        const uint16_t* k, int qk_stride, uint32_t* flag, int k_rows, int batch,
-                        int H_k, int H_v, int D, int stash_seq_floats, cudaStream_t s) {
+                        const uint16_t* k, int qk_stride, float* const* hi_tables,
+                        int slab_entries, uint32_t* flag, int k_rows, int batch, int H_k, int H_v,
+                        int D, int stash_seq_floats, cudaStream_t s) {
   (void)k_rows;
   if (batch == 0) return cudaSuccess;
   dim3 grid(H_v, batch);
   if (D == 128)
-    fold_kernel<128><<<grid, kVThreads, 0, s>>>(h_table, stash, na_tab, k, qk_stride, flag, H_k, H_v,
-                                          stash_seq_floats);
+    fold_kernel<128><<<grid, kVThreads, 0, s>>>(h_table, stash, na_tab, k, qk_stride, hi_tables,
+                                                slab_entries, flag, H_k, H_v, stash_seq_floats);
   else
-    fold_kernel<64><<<grid, kVThreads, 0, s>>>(h_table, stash, na_tab, k, qk_stride, flag, H_k, H_v,
-                                         stash_seq_floats);
+    fold_kernel<64><<<grid, kVThreads, 0, s>>>(h_table, stash, na_tab, k, qk_stride, hi_tables,
+                                               slab_entries, flag, H_k, H_v, stash_seq_floats);
   return cudaGetLastError();
 }
 

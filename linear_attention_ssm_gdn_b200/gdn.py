@@ -109,8 +109,12 @@ def gdn_chunk_prefill_workspace_bytes(total_tokens, num_seqs, H_k, H_v, d_k, d_v
 
 
 def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens, h0=None, hT=None, o=None, scale=1.0,
-                      workspace=None, store_final_state=True, stream=None):
-    """Chunked prefill over packed sequences. Returns (o, hT)."""
+                      workspace=None, store_final_state=True, stream=None, limbs=1,
+                      segments=None):
+    """Chunked prefill over packed sequences. Returns (o, hT).  limbs=2 calls
+    gdn_chunk_prefill_x2 (the state enters the MMAs as two bf16 limbs);
+    segments=S calls gdn_chunk_prefill_segmented (two-level scan with S
+    segments per sequence; None lets the library choose)."""
     lib = _lib.load()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, n)
@@ -133,17 +137,29 @@ def gdn_chunk_prefill(q, k, v, g, beta, cu_seqlens, h0=None, hT=None, o=None, sc
     for t, n in ((h0, "h0"), (hT, "hT")):
         if t is not None:
             _dense(t, torch.float32, (num_seqs, H_v, d_k, d_v), n)
-    need = int(lib.gdn_chunk_prefill_workspace_bytes(T, num_seqs, H_k, H_v, d_k, d_v))
+    if segments is None:
+        need = int(lib.gdn_chunk_prefill_workspace_bytes(T, num_seqs, H_k, H_v, d_k, d_v))
+    else:
+        need = int(lib.gdn_chunk_prefill_segmented_workspace_bytes(T, num_seqs, H_k, H_v, d_k,
+                                                                   d_v, int(segments)))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     if workspace is not None and not workspace.is_cuda:
         raise ValueError("workspace: must be a CUDA tensor")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = lib.gdn_chunk_prefill(_ptr(q), _ptr(k), qk_stride, _ptr(v), v_stride, _ptr(g),
-                               _ptr(beta), gb_stride, _ptr(cu_seqlens), num_seqs, T, _ptr(h0),
-                               _ptr(hT), _ptr(o), H_k, H_v, d_k, d_v, float(scale),
-                               _ptr(workspace), ws_bytes, _stream(stream))
-    _lib.check("gdn_chunk_prefill", rc)
+    if limbs not in (1, 2):
+        raise ValueError("limbs must be 1 or 2")
+    args = (_ptr(q), _ptr(k), qk_stride, _ptr(v), v_stride, _ptr(g), _ptr(beta), gb_stride,
+            _ptr(cu_seqlens), num_seqs, T, _ptr(h0), _ptr(hT), _ptr(o), H_k, H_v, d_k, d_v,
+            float(scale))
+    if segments is None:
+        name = "gdn_chunk_prefill" if limbs == 1 else "gdn_chunk_prefill_x2"
+        rc = getattr(lib, name)(*args, _ptr(workspace), ws_bytes, _stream(stream))
+    else:
+        name = "gdn_chunk_prefill_segmented"
+        rc = lib.gdn_chunk_prefill_segmented(*args, int(segments), int(limbs), _ptr(workspace),
+                                             ws_bytes, _stream(stream))
+    _lib.check(name, rc)
     return o, hT
 
 
@@ -188,19 +204,69 @@ def gdn_verify_woa(h_table, q, k, v, g, beta, engaged_flag, o=None, stash=None, 
     return o, stash
 
 
-def gdn_fold(h_table, stash, na_tab, k, engaged_flag, H_v, k_rows=4, stream=None):
-    """Apply the first na_tab[b] verified rows to each state (in place)."""
+def _slab_table(hi_tables, batch):
+    """hi_tables: int64 CUDA tensor [batch, slab_entries] of state pointers (or None)."""
+    if hi_tables is None:
+        return None, 0
+    _need(hi_tables, torch.int64, "hi_tables")
+    if hi_tables.dim() != 2 or hi_tables.shape[0] != batch or not hi_tables.is_contiguous():
+        raise ValueError(f"hi_tables: expected a contiguous [{batch}, slab_entries] table")
+    return _ptr(hi_tables), int(hi_tables.shape[1])
+
+
+def gdn_verify_parent(h_table, q, k, v, g, beta, hi_tables=None, o=None, scale=1.0,
+                      stream=None):
+    """Parent K=4 verify: outputs as gdn_verify_woa; the states after rows 0..2
+    go to the slabs hi_tables[b, r] (int64 [batch, slab_entries] table of state
+    pointers), the state after row 3 replaces the live state.  Returns o."""
     lib = _lib.load()
     _need(h_table, torch.int64, "h_table")
-    _need(stash, torch.float32, "stash")
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    R, H_k, d_k = q.shape
+    H_v, d_v = v.shape[1], v.shape[2]
+    batch = h_table.shape[0]
+    if R != 4 * batch:
+        raise ValueError("q/k/v must hold 4 rows per sequence")
+    qk_stride = _rows(q, "q", H_k, d_k)
+    if _rows(k, "k", H_k, d_k) != qk_stride:
+        raise ValueError("q and k must share one row stride")
+    v_stride = _rows(v, "v", H_v, d_v)
+    gb_stride = _gates(g, beta, R, H_v)
+    if o is None:
+        o = torch.empty(R, H_v, d_v, dtype=torch.bfloat16, device=q.device)
+    _dense(o, torch.bfloat16, (R, H_v, d_v), "o")
+    hp, se = _slab_table(hi_tables, batch)
+    rc = lib.gdn_verify_parent(_ptr(h_table), _ptr(q), _ptr(k), qk_stride, _ptr(v), v_stride,
+                               _ptr(g), _ptr(beta), gb_stride, _ptr(o), hp, se, batch, H_k, H_v,
+                               d_k, d_v, float(scale), _stream(stream))
+    _lib.check("gdn_verify_parent", rc)
+    return o
+
+
+def gdn_fold(h_table, stash, na_tab, k, engaged_flag, H_v, k_rows=4, hi_tables=None,
+             stream=None):
+    """Post-verdict fold: each state ends as the state after its first
+    na_tab[b] verified rows -- by applying the write-on-accept stash (engaged
+    word set) or by restoring a parent verify's slab (engaged word clear;
+    hi_tables as passed to gdn_verify_parent).  stash may be None when only the
+    parent path is used; k is always given (its shape fixes H_k and d)."""
+    lib = _lib.load()
+    _need(h_table, torch.int64, "h_table")
     _need(k, torch.bfloat16, "k")
     _need(engaged_flag, torch.int32, "engaged_flag")
     batch = h_table.shape[0]
     _dense(na_tab, torch.int32, (batch,), "na_tab")
     _, H_k, d = k.shape
     qk_stride = _rows(k, "k", H_k, d)
-    ssf = int(stash.stride(0)) if batch > 1 else gdn_stash_seq_floats(H_v, d, d)
-    rc = lib.gdn_fold(_ptr(h_table), _ptr(stash), _ptr(na_tab), _ptr(k), qk_stride,
+    if stash is not None:
+        _need(stash, torch.float32, "stash")
+        ssf = int(stash.stride(0)) if batch > 1 else gdn_stash_seq_floats(H_v, d, d)
+        k_ptr = _ptr(k)
+    else:
+        ssf, k_ptr = 0, None
+    hp, se = _slab_table(hi_tables, batch)
+    rc = lib.gdn_fold(_ptr(h_table), _ptr(stash), _ptr(na_tab), k_ptr, qk_stride, hp, se,
                       _ptr(engaged_flag), int(k_rows), batch, H_k, H_v, d, d, ssf,
                       _stream(stream))
     _lib.check("gdn_fold", rc)

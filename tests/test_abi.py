@@ -106,11 +106,32 @@ def test_verify_fold_guards(lib):
                               128, 1.0, P, None) == _lib.GDN_ERR_SHAPE
     assert lib.gdn_verify_woa(P, P, P, 2048, P, 6144, P, P, 48, P, P, 25344, 0, 16, 48, 128,
                               128, 1.0, P, None) == _lib.GDN_OK
-    assert lib.gdn_fold(P, P, P, P, 2048, P, 3, 64, 16, 48, 128, 128, 25344,
+    assert lib.gdn_fold(P, P, P, P, 2048, NULL, 0, P, 3, 64, 16, 48, 128, 128, 25344,
                         None) == _lib.GDN_ERR_SHAPE
     assert "k_rows" in _err(lib)
-    assert lib.gdn_fold(P, P, NULL, P, 2048, P, 4, 64, 16, 48, 128, 128, 25344,
+    assert lib.gdn_fold(P, P, NULL, P, 2048, NULL, 0, P, 4, 64, 16, 48, 128, 128, 25344,
                         None) == _lib.GDN_ERR_NULL
+    # stash and k go together; one of the two branches must have its data
+    assert lib.gdn_fold(P, NULL, P, P, 2048, P, 3, P, 4, 64, 16, 48, 128, 128, 25344,
+                        None) == _lib.GDN_ERR_NULL
+    assert "both" in _err(lib)
+    assert lib.gdn_fold(P, NULL, P, NULL, 2048, NULL, 0, P, 4, 64, 16, 48, 128, 128, 0,
+                        None) == _lib.GDN_ERR_NULL
+    assert "neither" in _err(lib)
+    assert lib.gdn_fold(P, NULL, P, NULL, 2048, P, 2, P, 4, 64, 16, 48, 128, 128, 0,
+                        None) == _lib.GDN_ERR_SHAPE
+    assert "slab_entries" in _err(lib)
+    assert lib.gdn_fold(P, NULL, P, NULL, 2048, P, 3, P, 4, 0, 16, 48, 128, 128, 0,
+                        None) == _lib.GDN_OK
+    # the parent verify: null guards, slab count, strides
+    assert lib.gdn_verify_parent(NULL, P, P, 2048, P, 6144, P, P, 48, P, P, 3, 64, 16, 48, 128,
+                                 128, 1.0, None) == _lib.GDN_ERR_NULL
+    assert lib.gdn_verify_parent(P, P, P, 2048, P, 6144, P, P, 48, P, P, 2, 64, 16, 48, 128,
+                                 128, 1.0, None) == _lib.GDN_ERR_SHAPE
+    assert lib.gdn_verify_parent(P, P, P, 2047, P, 6144, P, P, 48, P, P, 3, 64, 16, 48, 128,
+                                 128, 1.0, None) == _lib.GDN_ERR_STRIDE
+    assert lib.gdn_verify_parent(P, P, P, 2048, P, 6144, P, P, 48, P, NULL, 0, 0, 16, 48, 128,
+                                 128, 1.0, None) == _lib.GDN_OK
     assert lib.gdn_flag_clear(NULL, None) == _lib.GDN_ERR_NULL
 
 
@@ -184,3 +205,16 @@ def test_python_binding_rejects_wrong_table_and_flag_dtypes():
                  torch.zeros(1, dtype=torch.int32), 1)
     with pytest.raises(TypeError, match="engaged_flag"):
         gdn_flag_clear(torch.zeros(1, dtype=torch.float32))
+
+
+def test_static_stash_rejects_oversized_batch(lib):
+    """gdn_verify_woa_static refuses a batch whose stash would not fit its
+    static array, before any launch (so no GPU is needed)."""
+    ssf = lib.gdn_stash_seq_floats(48, 128, 128)
+    too_many = (2 * 1024 * 1024) // ssf + 1
+    stash_ptr = ctypes.c_void_p()
+    rc = lib.gdn_verify_woa_static(0x10000, 0x10000, 0x10000, 2048, 0x10000, 6144, 0x10000,
+                                   0x10000, 48, 0x10000, too_many, 16, 48, 128, 128, 1.0,
+                                   0x10000, ctypes.byref(stash_ptr), None)
+    assert rc == _lib.GDN_ERR_SHAPE
+    assert "exceeds the static stash" in lib.gdn_last_error().decode()

@@ -68,3 +68,34 @@ def test_ba_gates_wide_range():
     ba.w = (ba.w.float() * 20.0).to(torch.bfloat16)
     got = _check(ba)
     assert float(np.abs(got[:, :48]).min()) < 1e-6 < float(np.abs(got[:, :48]).max())
+
+
+@pytest.mark.parametrize("M", [1, 2, 16, 33, 64])
+def test_ba_gates_decode_shapes(M):
+    """Few-token (batched decode) steps at the pages' projection, N = 96,
+    K = 5120: the outputs and the reduction are split across CTAs instead of
+    the tokens (page "ssm_ba_gates_hopper.rs", token-count guard).  Parity at
+    every element, and the time per launch is printed (CUDA events, 50
+    back-to-back launches after a warm-up)."""
+    ba = I.ba_inputs(M, 5120, 48, 3, seed=900 + M)
+    _check(ba)
+    x, w = ba.x.to(DEV), ba.w.to(DEV)
+    a, dt = ba.a_log.to(DEV), ba.dt_bias.to(DEV)
+    out = torch.empty(M, 96, device=DEV)
+    for _ in range(5):
+        gdn_ba_gates(x, w, a, dt, 3, gate_out=out)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(50):
+        gdn_ba_gates(x, w, a, dt, 3, gate_out=out)
+    e1.record()
+    torch.cuda.synchronize()
+    print(f"[timing] ba_gates M={M} N=96 K=5120: {e0.elapsed_time(e1) / 50 * 1e3:.2f} us/launch")
+
+
+@pytest.mark.parametrize("M,K,nv,vpg", [(5, 8, 4, 4), (17, 40, 6, 3), (64, 200, 128, 4),
+                                        (3, 2056, 2, 1)])
+def test_ba_gates_decode_ragged(M, K, nv, vpg):
+    """Few-token shapes with tiny or odd K (one K slice, ragged slices) and
+    output counts that leave the last 8-output group partly idle."""
+    _check(I.ba_inputs(M, K, nv, vpg, seed=M * 7 + K))

@@ -145,3 +145,29 @@ def test_repeat_calls_are_deterministic():
     o2, h2 = _run(p)
     np.testing.assert_array_equal(o1, o2)
     np.testing.assert_array_equal(h1, h2)
+
+
+def test_positive_gates_within_the_bound_are_exact():
+    """Gates of both signs, g ~ N(0, 0.3): the cumulative gate rises and falls
+    within each chunk (by far less than the documented bound of 80), so every
+    decay factor stays finite and the result matches the oracle."""
+    p = I.prefill_inputs([700, 130], 1, 2, 128, 128, seed=20, h0_std=0.02)
+    p.g = torch.randn(p.g.shape, generator=torch.Generator().manual_seed(21)) * 0.3
+    assert float(p.g.max()) > 0.5
+    _check(p, what="positive gates")
+
+
+def test_gate_rise_beyond_the_bound_is_flagged():
+    """A chunk whose cumulative gate rises by more than 80 (g = +2 on all 64
+    rows: a rise of 128) cannot be represented by the f32 decay factors: the
+    prefill sets bit 64 of its device error word instead of returning silent
+    garbage (its outputs are undefined and not compared)."""
+    p = I.prefill_inputs([64], 1, 1, 128, 128, seed=22, h0_std=None)
+    p.g = torch.full(p.g.shape, 2.0)
+    d = _to_dev(p)
+    gdn_chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"])
+    torch.cuda.synchronize()
+    errs = debug_device_errors()
+    assert errs[1] == 64 and errs[0] == errs[2] == errs[3] == 0, errs
+    # the flag does not stick: a normal call afterwards reports nothing
+    _check(I.prefill_inputs([64], 1, 1, 128, 128, seed=23, h0_std=None), what="after flag")

@@ -11,6 +11,7 @@ import torch
 
 import oracle
 from helpers import assert_prefill_close, f64
+from linear_attention_ssm_gdn_b200 import _lib
 from linear_attention_ssm_gdn_b200 import (debug_device_errors, gdn_flag_clear, gdn_fold,
                                            gdn_verify_woa)
 from linear_attention_ssm_gdn_b200 import inputs as I
@@ -81,6 +82,23 @@ def test_fold_with_flag_clear_is_a_no_op():
     gdn_fold(table, stash, torch.full((6,), 4, dtype=torch.int32, device=DEV), d["k"], flag,
              vi.H_v)
     torch.cuda.synchronize()
+    assert torch.equal(pool.cpu(), vi.pool)
+
+
+def test_fold_after_a_failed_verify_changes_no_state():
+    """A verify CTA whose bounded wait ran out ORs GDN_FLAG_ERROR |
+    GDN_FLAG_STASH_BAD into the engaged word (its stash is incomplete).  The
+    bits are planted on the host here, between a normal verify and the fold:
+    the fold must then leave every state bit-identical, whatever na says."""
+    vi = I.verify_inputs(6, 4, 2, 4, 128, 128, slots_total=8, seed=47)
+    pool, table, d, flag = _setup(vi)
+    gdn_flag_clear(flag)
+    _, stash = gdn_verify_woa(table, d["q"], d["k"], d["v"], d["g"], d["beta"], flag)
+    flag.bitwise_or_(_lib.GDN_FLAG_ERROR | _lib.GDN_FLAG_STASH_BAD)
+    gdn_fold(table, stash, torch.full((6,), 4, dtype=torch.int32, device=DEV), d["k"], flag,
+             vi.H_v)
+    torch.cuda.synchronize()
+    assert int(flag.item()) == 7
     assert torch.equal(pool.cpu(), vi.pool)
 
 

@@ -5,8 +5,10 @@ engine that reserved all of it up front in its own pool, or a decode loop that
 must never call cudaMalloc because it can stall the whole device.  For them
 the verify's stash (the scratch it leaves for the fold) lives in a static
 array inside the library.  This test calls that entry point through the C ABI
-twice in a row and checks that its outputs, and the fold driven by the stash
-address it hands back, match the regular gdn_verify_woa path.
+twice in a row, on two different inputs, and checks that its outputs, and the
+fold driven by the stash address it hands back, match the regular
+gdn_verify_woa path on the same inputs.  (The refusal of an oversized batch
+needs no GPU and is tested with the other guards in test_abi.py.)
 
 The file name makes pytest collect it last; it also passes on its own in a
 fresh process.
@@ -47,31 +49,37 @@ def _static_verify(lib, table, d, vi, o, flag):
     return stash_ptr.value
 
 
+def _regular(vi):
+    """Verify + fold through the regular entry point (caller-allocated stash)."""
+    pool, table, d = _prepare(vi)
+    flag = torch.zeros(1, dtype=torch.int32, device=DEV)
+    gdn_flag_clear(flag)
+    o, stash = gdn_verify_woa(table, d["q"], d["k"], d["v"], d["g"], d["beta"], flag)
+    gdn_fold(table, stash, d["na"], d["k"], flag, vi.H_v)
+    torch.cuda.synchronize()
+    return o.float().cpu().numpy(), pool.cpu().numpy()
+
+
 def test_static_stash_verify_matches_regular_twice():
     lib = _lib.load()
-    vi = I.workload(4).verify  # batch 64 x 4 rows, 48 heads, d = 128
-    ssf = lib.gdn_stash_seq_floats(vi.H_v, vi.d_k, vi.d_v)
-    assert vi.batch * ssf <= 2 * 1024 * 1024
+    # Two calls in a row on DIFFERENT inputs (another seed, so other states,
+    # rows and accepted counts): the second call must replace the shared
+    # array's contents, not reuse what the first call left there.
+    first = I.workload(4).verify  # batch 64 x 4 rows, 48 heads, d = 128
+    second = I.verify_inputs(64, 4, 16, 48, 128, 128, slots_total=128, seed=104)
+    assert not torch.equal(first.na, second.na)
+    for call, vi in enumerate((first, second)):
+        ssf = lib.gdn_stash_seq_floats(vi.H_v, vi.d_k, vi.d_v)
+        assert vi.batch * ssf <= 2 * 1024 * 1024
+        o_ref, pool_ref = _regular(vi)
 
-    # Regular path: caller-allocated stash.
-    pool_ref, table_ref, d = _prepare(vi)
-    flag_ref = torch.zeros(1, dtype=torch.int32, device=DEV)
-    gdn_flag_clear(flag_ref)
-    o_ref, stash_ref = gdn_verify_woa(table_ref, d["q"], d["k"], d["v"], d["g"], d["beta"],
-                                      flag_ref)
-    gdn_fold(table_ref, stash_ref, d["na"], d["k"], flag_ref, vi.H_v)
-    torch.cuda.synchronize()
-    o_ref = o_ref.float().cpu().numpy()
-    pool_ref = pool_ref.cpu().numpy()
-
-    for call in range(2):  # two calls in a row share the static array
         pool, table, d2 = _prepare(vi)
         flag = torch.zeros(1, dtype=torch.int32, device=DEV)
         gdn_flag_clear(flag)
         o = torch.empty(vi.batch * 4, vi.H_v, vi.d_v, dtype=torch.bfloat16, device=DEV)
         stash_addr = _static_verify(lib, table, d2, vi, o, flag)
         rc = lib.gdn_fold(table.data_ptr(), stash_addr, d2["na"].data_ptr(), d2["k"].data_ptr(),
-                          vi.H_k * vi.d_k, flag.data_ptr(), 4, vi.batch, vi.H_k, vi.H_v,
+                          vi.H_k * vi.d_k, None, 0, flag.data_ptr(), 4, vi.batch, vi.H_k, vi.H_v,
                           vi.d_k, vi.d_v, ssf, torch.cuda.current_stream().cuda_stream)
         assert rc == 0, lib.gdn_last_error().decode()
         torch.cuda.synchronize()
@@ -85,15 +93,3 @@ def test_static_stash_verify_matches_regular_twice():
         # Same kernel, same inputs: the results are in fact identical.
         np.testing.assert_array_equal(o_np, o_ref)
         np.testing.assert_array_equal(p_np, pool_ref)
-
-
-def test_static_stash_rejects_oversized_batch():
-    lib = _lib.load()
-    ssf = lib.gdn_stash_seq_floats(48, 128, 128)
-    too_many = (2 * 1024 * 1024) // ssf + 1
-    stash_ptr = ctypes.c_void_p()
-    rc = lib.gdn_verify_woa_static(0x10000, 0x10000, 0x10000, 2048, 0x10000, 6144, 0x10000,
-                                   0x10000, 48, 0x10000, too_many, 16, 48, 128, 128, 1.0,
-                                   0x10000, ctypes.byref(stash_ptr), None)
-    assert rc == _lib.GDN_ERR_SHAPE
-    assert "exceeds the static stash" in lib.gdn_last_error().decode()
