@@ -6,9 +6,14 @@ One step = one pass of every hot-path call:
   (x [4576, 5120] -> gates -> prefill, d = 128, H_k = 16, H_v = 48, h0 = 0), then
   gdn_flag_clear + gdn_verify_woa + gdn_fold on the speculative-verify batch
   (64 sequences x 4 rows, states reached through a pointer table).
-value = prefill tokens per second of device time (4576 tokens per step, all
-ranks summed; inputs resident in HBM; the per-step working set, ~560 MB, is
-larger than L2, so no flush is needed between steps).
+value = prefill tokens per second: 4576 tokens over the prefill launch's own
+device time (CUDA events around it inside the timed steps; all ranks summed).
+The whole step's rate is reported beside it (step_tokens_per_s).  Inputs are
+resident in HBM; the per-step working set (~560 MB) is larger than L2, so no
+flush is needed between steps.  The single-sequence (4096 tokens, 32 heads)
+and varlen (8 sequences, 24,674 tokens) prefill workloads are timed after the
+steps, each launch on its own (an L2 flush between launches of the first,
+whose working set fits in L2).
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -91,52 +96,61 @@ def profiled_traffic():
 # --------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clocks and clock-event reasons of this GPU, sampled by nvidia-smi in
+    a child process (read-only queries) while the GPU works; the device is
+    named by its UUID, which stays right under CUDA_VISIBLE_DEVICES."""
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
+    QUERY = "clocks.sm,clocks.max.sm,clocks_event_reasons.active"
 
-    def __init__(self, index: int, period_s: float = 0.002):
-        self.index, self.period = index, period_s
-        self.samples, self.reasons = [], 0
-        self.max_mhz = None
-        self._stop = threading.Event()
-        self._t = None
+    def __init__(self, device, period_ms: int = 50):
+        self.device, self.period_ms = device, period_ms
+        self._p = None
         self.ok = False
 
     def start(self):
+        import shutil
+        import subprocess
         try:
-            import pynvml
-            pynvml.nvmlInit()
-            self._nv = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            import torch
+            exe = shutil.which("nvidia-smi")
+            if exe is None:
+                return self
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(self.device).uuid)
+            self._p = subprocess.Popen(
+                [exe, "-i", uuid, f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", str(self.period_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.ok = True
         except Exception:
-            return self
-        self._t = threading.Thread(target=self._run, daemon=True)
-        self._t.start()
+            self._p = None
         return self
 
-    def _run(self):
-        nv = self._nv
-        while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
-            except Exception:
-                pass
-            time.sleep(self.period)
-
     def stop(self):
-        self._stop.set()
-        if self._t is not None:
-            self._t.join()
-        if not self.ok:
+        if self._p is None:
             return None
-        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
-        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+        self._p.terminate()
+        try:
+            out, _ = self._p.communicate(timeout=10)
+        except Exception:
+            self._p.kill()
+            out, _ = self._p.communicate()
+        mhz, mx, reasons = [], None, 0
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 3:
+                continue
+            try:
+                mhz.append(float(f[0]))
+                mx = float(f[1])
+                reasons |= int(f[2], 16)
+            except ValueError:
+                continue
+        names = [n for b, n in self.REASONS.items() if reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": names, "samples": len(mhz)}
 
 
 # --------------------------------------------------------------------------
@@ -221,13 +235,62 @@ def step_calls(d, meta, ev=None):
 LAUNCHES_PER_STEP = 5  # ba_gates, prefill, flag_clear, verify, fold
 
 
+def progress(msg: str) -> None:
+    """One line on stderr per bench phase (stdout carries only the JSON line)."""
+    print(f"[bench] {time.strftime('%H:%M:%S')} {msg}", file=sys.stderr, flush=True)
+
+
+def roofline_entry(T, N, H_k, H_v, d, us):
+    """Roofline of one prefill launch of T tokens (N sequences) taking `us`."""
+    hbm, tf_burst, _, src = peaks()
+    B = prefill_alg_bytes(T, N, H_k, H_v, d, d)
+    F = prefill_alg_flops(T, H_v, d, d)
+    t = us / 1e6
+    t_roof = max(B / (hbm * 1e9), F / (tf_burst * 1e12))
+    return {"us": us, "tokens_per_s": T / t, "achieved_gbs": B / t / 1e9,
+            "frac": B / t / 1e9 / hbm, "roofline_us": t_roof * 1e6,
+            "frac_of_roofline_time": t_roof / t, "alg_bytes": B, "alg_flops": F,
+            "peak_source": src}
+
+
+def time_prefill(p, dev, reps, flush=None, **kw):
+    """Mean device time (us) of `reps` launches of gdn_chunk_prefill on inputs
+    p (resident in HBM), CUDA events around each launch; `flush` (a tensor
+    larger than L2) is overwritten between launches when given."""
+    import torch
+
+    from linear_attention_ssm_gdn_b200 import gdn_chunk_prefill
+    d = {k: getattr(p, k).to(dev) for k in ("q", "k", "v", "g", "beta", "cu_seqlens", "h0")}
+    o = torch.empty(p.total_tokens, p.H_v, p.d_v, dtype=torch.bfloat16, device=dev)
+    hT = torch.empty_like(d["h0"])
+
+    def call():
+        gdn_chunk_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], h0=d["h0"],
+                          hT=hT, o=o, **kw)
+    for _ in range(3):
+        call()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for e0, e1 in evs:
+        if flush is not None:
+            flush.zero_()
+        e0.record()
+        call()
+        e1.record()
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e3
+
+
 def run_ours(args, rank, world, dist):
     import torch
+
+    from linear_attention_ssm_gdn_b200 import inputs as I
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     host, d, meta = make_inputs(dev)
     stream = torch.cuda.current_stream()
+    progress("inputs ready")
 
     for _ in range(args.warmup):
         step_calls(d, meta)
@@ -242,7 +305,7 @@ def run_ours(args, rank, world, dist):
             None, None, None] for _ in range(K)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(dev.index).start()
+    clocks = ClockSampler(dev).start()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
@@ -253,11 +316,12 @@ def run_ours(args, rank, world, dist):
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    clk = clocks.stop()
     total_ms = t_start.elapsed_time(t_end)
-    t_prefill_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    prefill_ms = sum(e[1].elapsed_time(e[2]) for e in evs)  # K prefill launches
     total_ms = max_over_ranks(total_ms, dist, dev)
+    prefill_ms = max_over_ranks(prefill_ms, dist, dev)
 
+    progress("timed steps done")
     # ---- untimed split: per-kernel events on every kernel of a few steps
     ks = max(1, min(K, 50))
     evs2 = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(ks)]
@@ -292,30 +356,68 @@ def run_ours(args, rank, world, dist):
     if dist:
         dist.barrier()
 
+    progress("end-to-end steps done")
+    # ---- the other prefill workloads, one launch at a time (every rank runs
+    # the same calls; rank 0 reports its own device times)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2 (126 MB)
+    p1 = I.workload(1).prefill
+    p3 = I.workload(3).prefill
+    p2 = I.prefill_inputs([4576], 16, 48, 128, 128, seed=2, h0_std=None)  # drawn gates
+    tp = I.prefill_inputs([16384], 2, 6, 128, 128, seed=2, h0_std=None)
+    others = {
+        "single_sequence": (p1, time_prefill(p1, dev, 10, flush=flush),
+                            "T=4096 H_k=16 H_v=32 d=128, h0~N(0,0.02); L2 flushed per launch"),
+        "varlen": (p3, time_prefill(p3, dev, 5),
+                   f"8 seqs {sum(I.varlen_lengths(3))} tokens H_k=16 H_v=48 d=128; "
+                   "inputs > L2"),
+    }
+    variants = {
+        "prefill_x2_us": time_prefill(p2, dev, 10, limbs=2),
+        "prefill_x1_drawn_gates_us": time_prefill(p2, dev, 10),
+        "tp_shard_single_level_us": time_prefill(tp, dev, 10, flush=flush, segments=1),
+        "tp_shard_two_level_us": time_prefill(tp, dev, 10, flush=flush),
+        "note": "us per launch. x2/x1: the 4576-token 48-head prefill with drawn gates, "
+                "two-limb vs one-limb state operand.  tp_shard: 16384 tokens, H_k=2, "
+                "H_v=6 (the same geometry over 8 GPUs), single-level scan vs the "
+                "library's choice (two-level, segment-parallel)",
+    }
+    del flush
+    clk = clocks.stop()
+    if clk is not None:
+        clk["window"] = ("sampled every 50 ms from the start of the timed steps to the end of "
+                         "the other workloads (the GPU is busy throughout)")
+    progress("other workloads done")
+
     if rank != 0:
         return None
     T = meta["T"]
-    value = job_value(world, K, T, total_ms)
+    value = world * K * T / (prefill_ms / 1e3)
+    step_value = job_value(world, K, T, total_ms)
     e2e_value = job_value(world, K, T, e2e_ms)
     hbm, tf_burst, tf_sust, src = peaks()
-    B = prefill_alg_bytes(T, meta["N"], meta["H_k"], meta["H_v"], meta["d_k"], meta["d_v"])
-    F = prefill_alg_flops(T, meta["H_v"], meta["d_k"], meta["d_v"])
-    t_pf = t_prefill_ms / 1e3
-    achieved = B / t_pf / 1e9
-    t_roof = max(B / (hbm * 1e9), F / (tf_burst * 1e12))
+    t_prefill_us = prefill_ms / K * 1e3
+    rf = roofline_entry(T, meta["N"], meta["H_k"], meta["H_v"], meta["d_k"], t_prefill_us)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "tokens_per_step": T, "l2": "inputs larger than L2 "
                    "(~560 MB per step), no flush", "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": profiled_traffic(),
+        "value_note": "prefill tokens/s: tokens over the prefill launch's device time "
+                      "(CUDA events around it in the timed steps)",
+        "step_tokens_per_s": step_value,
+        "roofline": {"bound": "hbm", "achieved": rf["achieved_gbs"], "peak": hbm, "unit": "GB/s",
+                     "frac": rf["frac"], "traffic": profiled_traffic(),
                      "peak_source": src, "kernel": "prefill_kernel",
-                     "alg_bytes_per_launch": B, "alg_flops_per_launch": F,
-                     "tflops_achieved": F / t_pf / 1e12,
-                     "roofline_time_us": t_roof * 1e6,
-                     "frac_of_roofline_time": t_roof / t_pf},
+                     "alg_bytes_per_launch": rf["alg_bytes"],
+                     "alg_flops_per_launch": rf["alg_flops"],
+                     "tflops_achieved": rf["alg_flops"] / (t_prefill_us / 1e6) / 1e12,
+                     "roofline_time_us": rf["roofline_us"],
+                     "frac_of_roofline_time": rf["frac_of_roofline_time"]},
+        "workloads": {name: dict(roofline_entry(pp.total_tokens, pp.num_seqs, pp.H_k, pp.H_v,
+                                                pp.d_k, us), config=desc)
+                      for name, (pp, us, desc) in others.items()},
+        "variants": variants,
         "kernels_us": {k: v * 1e3 for k, v in per.items()},
         "kernels_us_note": "separate untimed pass with events around every kernel "
                            "(each event record adds about 2.7 us to its interval)",
@@ -331,60 +433,109 @@ def run_ours(args, rank, world, dist):
 # The oracle on the host cores (cpu_baseline leg and the reference arm)
 # --------------------------------------------------------------------------
 
-def oracle_step_seconds(budget_s: float):
-    """Time the oracle on a bounded sample of one step and scale it to the full
-    step.  Returns (seconds per full step, threads, sample description)."""
-    import numpy as np
+def _f64(t):
+    import torch
+    return t.to(dtype=torch.float64).numpy()
 
+
+def oracle_prefill_rate(p, form, threads, heads, seqs=None, max_tokens=None):
+    """Oracle tokens/s for the whole prefill workload p, from a timed sample:
+    `heads` v-heads (each with its own k-head) over the sequences `seqs` (all
+    by default), each cut to its first `max_tokens` tokens, scaled by the
+    heads and tokens left out (the oracle's cost is linear in both).  The
+    oracle's cost does not depend on the gate values."""
+    import numpy as np
+    import torch
+
+    import oracle
+    vpg = p.H_v // p.H_k
+    hs = list(range(heads))
+    kh = [h // vpg for h in hs]
+    cu = p.cu_seqlens.numpy()
+    seqs = list(range(p.num_seqs)) if seqs is None else seqs
+    cap = (lambda n: int(cu[n + 1] - cu[n])) if max_tokens is None else \
+        (lambda n: min(int(cu[n + 1] - cu[n]), max_tokens))
+    rows = torch.from_numpy(np.concatenate([np.arange(cu[n], cu[n] + cap(n)) for n in seqs]))
+    lens = [cap(n) for n in seqs]
+    cu_s = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    # select the sample before widening to f64 (the full varlen tensors would
+    # take gigabytes of host memory in f64)
+    ht, kt = torch.tensor(hs), torch.tensor(kh)
+    rng = np.random.default_rng(0)
+    gs = (_f64(p.g[rows][:, ht]) if p.g is not None
+          else -np.abs(rng.standard_normal((len(rows), heads))) * 0.1)
+    bs = (_f64(p.beta[rows][:, ht]) if p.beta is not None
+          else rng.uniform(0.1, 0.9, (len(rows), heads)))
+    h0 = _f64(p.h0[torch.tensor(seqs)][:, ht])
+    args = (_f64(p.q[rows][:, kt]), _f64(p.k[rows][:, kt]), _f64(p.v[rows][:, ht]), gs, bs,
+            cu_s, h0)
+    fn = oracle.gdn_token if form == "token" else oracle.gdn_chunked
+    t0 = time.perf_counter()
+    fn(*args, nthreads=threads)
+    dt = time.perf_counter() - t0
+    scale = (p.H_v / heads) * (p.total_tokens / max(1, len(rows)))
+    return p.total_tokens / (dt * scale)
+
+
+def cpu_baseline(detail=True):
+    """The oracle on this host's cores, on bounded samples of the workloads.
+    Returns (step seconds, threads, sample text, detail dict or None): a step
+    is BA gates + token-form prefill (4576 tokens, 48 heads) + verify/fold of
+    the speculative batch, all cores; the detail adds both prefill forms on
+    all cores and on one core for the three prefill workloads."""
     import oracle
     from linear_attention_ssm_gdn_b200 import inputs as I
 
-    def f64(t):
-        return t.to(dtype=__import__("torch").float64).numpy()
-
     nt = oracle.default_threads()
     w2 = I.workload(2)
-    p, ba = w2.prefill, w2.ba
+    p2, ba = w2.prefill, w2.ba
     vi = I.workload(4).verify
-    T, H_v, H_k, nv = p.total_tokens, p.H_v, p.H_k, ba.nv
-    vpg = H_v // H_k
+    T = p2.total_tokens
     # BA gates on a row sample
     m_s = min(T, max(32, int(64 * nt)))
-    x, w = f64(ba.x[:m_s]), f64(ba.w)
     t0 = time.perf_counter()
-    g = oracle.ba_gates(x, w, f64(ba.a_log), f64(ba.dt_bias), ba.vheads_per_group, nthreads=nt)
+    oracle.ba_gates(_f64(ba.x[:m_s]), _f64(ba.w), _f64(ba.a_log), _f64(ba.dt_bias),
+                    ba.vheads_per_group, nthreads=nt)
     t_ba = (time.perf_counter() - t0) * T / m_s
-    # prefill (token recurrence, the definition) on a head sample, full length
-    heads = list(range(min(H_v, max(1, nt))))
-    kh = [h // vpg for h in heads]
-    # The oracle's cost does not depend on the gate values, so the sampled heads
-    # use drawn gates instead of running the BA oracle over all rows first.
-    rng = np.random.default_rng(0)
-    gs = -np.abs(rng.standard_normal((T, len(heads)))) * 0.1
-    bs = rng.uniform(0.1, 0.9, (T, len(heads)))
-    args = (f64(p.q)[:, kh], f64(p.k)[:, kh], f64(p.v)[:, heads], gs, bs, [0, T], None)
-    t0 = time.perf_counter()
-    oracle.gdn_token(*args, nthreads=nt)
-    t_pf = (time.perf_counter() - t0) * H_v / len(heads)
     # verify + fold on a batch sample
     b_s = min(vi.batch, max(1, nt))
     sl = slice(0, 4 * b_s)
     t0 = time.perf_counter()
-    oracle.gdn_verify_fold(f64(vi.pool[vi.slots[:b_s]]), f64(vi.q[sl]), f64(vi.k[sl]),
-                           f64(vi.v[sl]), f64(vi.g[sl]), f64(vi.beta[sl]), vi.na[:b_s].numpy(),
-                           nthreads=nt)
+    oracle.gdn_verify_fold(_f64(vi.pool[vi.slots[:b_s]]), _f64(vi.q[sl]), _f64(vi.k[sl]),
+                           _f64(vi.v[sl]), _f64(vi.g[sl]), _f64(vi.beta[sl]),
+                           vi.na[:b_s].numpy(), nthreads=nt)
     t_vf = (time.perf_counter() - t0) * vi.batch / b_s
-    del g
+    heads_all = min(p2.H_v, max(1, nt))
+    rate2 = oracle_prefill_rate(p2, "token", nt, heads_all)
+    step_s = t_ba + T / rate2 + t_vf
     sample = (f"oracle (f64 C, {nt} threads): BA gates on {m_s}/{T} rows, token recurrence on "
-              f"{len(heads)}/{H_v} v-heads x {T} tokens, verify+fold on {b_s}/{vi.batch} "
+              f"{heads_all}/{p2.H_v} v-heads x {T} tokens, verify+fold on {b_s}/{vi.batch} "
               f"sequences; each scaled to the full step")
-    return t_ba + t_pf + t_vf, nt, sample
+    if not detail:
+        return step_s, nt, sample, None
+    det = {"ba_gates_us": t_ba * 1e6, "verify_fold_us": t_vf * 1e6, "cores": nt,
+           "prefill_tokens_per_s": {}}
+    p1 = I.workload(1).prefill
+    p3 = I.workload(3).prefill
+    for name, pp, seqs in (("single_sequence", p1, None), ("ba_geometry", p2, None),
+                           ("varlen", p3, [0])):
+        r = {}
+        for form, cap in (("token", None), ("chunked", 1024)):
+            r[f"{form}_all_cores"] = oracle_prefill_rate(pp, form, nt, min(pp.H_v, nt), seqs,
+                                                         cap)
+            r[f"{form}_1_core"] = oracle_prefill_rate(pp, form, 1, 1, seqs, cap)
+        det["prefill_tokens_per_s"][name] = r
+    det["sample"] = ("each prefill rate from a timed sample scaled to the whole workload: "
+                     f"min(H_v, {nt}) heads on all cores or 1 head on one core, over all "
+                     "sequences (varlen: its first sequence); the chunked form over the "
+                     "first 1024 tokens of each")
+    return step_s, nt, sample, det
 
 
 def run_reference(args):
     steps = []
     for i in range(args.warmup + args.steps):
-        s, nt, sample = oracle_step_seconds(budget_s=5.0)
+        s, nt, sample, _ = cpu_baseline(detail=False)
         if i >= args.warmup:
             steps.append(s)
     T = 4576
@@ -402,6 +553,8 @@ def run_reference(args):
 
 
 def main():
+    import faulthandler
+    faulthandler.enable()  # a crash in native code prints every thread's Python stack
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -434,9 +587,10 @@ def main():
             dist.destroy_process_group()
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            s, nt, sample = oracle_step_seconds(budget_s=20.0)
+            progress("cpu baseline")
+            s, nt, sample, det = cpu_baseline(detail=True)
             line["cpu_baseline"] = {"value": 4576 / s, "unit": UNIT, "cores": nt,
-                                    "kind": "oracle", "sample": sample}
+                                    "kind": "oracle", "sample": sample, "detail": det}
         print(json.dumps(line), flush=True)
     return 0
 

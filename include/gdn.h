@@ -255,10 +255,10 @@ int gdn_verify_woa_static(float* const* h_table, const uint16_t* q, const uint16
 
 /* --------------------------------------------------------------------------
  * gdn_verify_parent -- the parent (not write-on-accept) K = 4 verify.
- * Page "ssm_gdn_woa.rs", gdn_wy4_fold doc: when the engaged word is clear "the
- * parent kernel ran", leaving intermediate states Hi(i) in slabs reached through
- * hi_tables, from which a partial accept is restored.  This entry point is
- * that parent: the same four rows as gdn_verify_woa (same outputs), but the
+ * Page "ssm_gdn_woa.rs", gdn_wy4_fold doc: a clear engaged word means the
+ * non-write-on-accept verify ran instead, and it left the intermediate states
+ * Hi(i) in slabs reached through hi_tables, from which the fold restores a
+ * partial accept.  This entry point is that verify: the same four rows as gdn_verify_woa (same outputs), but the
  * states are written instead of a stash:
  *     Hi(r) = state after rows 0..r  (r = 0..3, from H0 = the live state)
  *   - Hi(0), Hi(1), Hi(2) go to the slabs hi_tables[b * slab_entries + r]
@@ -341,6 +341,20 @@ int gdn_flag_clear(uint32_t* engaged_flag, gdn_stream_t stream);
  * Errors: GDN_ERR_NULL, GDN_ERR_CUDA.
  * ------------------------------------------------------------------------ */
 int gdn_debug_device_errors(uint32_t* out4);
+
+/* --------------------------------------------------------------------------
+ * gdn_debug_set_spin_limit -- diagnostics, not part of the hot path.
+ * Every cross-CTA wait of the prefill's pipeline polls for at most a fixed
+ * number of clock cycles (about 2 s) before it gives up: it then records a
+ * bit in the prefill's device error word, raises the kernel's abort word and
+ * every CTA returns -- the kernel never hangs.  This call sets that limit for
+ * the prefill launches that follow (cycles > 0), or restores the default
+ * (cycles == 0), so that a test can make the waits run out on purpose.  The
+ * final drains of copies and MMAs still in flight always keep the default.
+ * A process-wide setting, read at launch; not for concurrent use.
+ * Errors: GDN_ERR_SHAPE (cycles < 0).
+ * ------------------------------------------------------------------------ */
+int gdn_debug_set_spin_limit(long long cycles);
 
 #ifdef __cplusplus
 }

@@ -7,6 +7,7 @@ synthetic input generators (`inputs`).
 from .gdn import (  # noqa: F401
     GdnError,
     debug_device_errors,
+    debug_set_spin_limit,
     gdn_ba_gates,
     gdn_chunk_prefill,
     gdn_chunk_prefill_workspace_bytes,

@@ -54,6 +54,7 @@ SIGNATURES = {
     "gdn_fold": (_I, [_P, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     "gdn_flag_clear": (_I, [_P, _P]),
     "gdn_debug_device_errors": (_I, [_P]),
+    "gdn_debug_set_spin_limit": (_I, [ctypes.c_longlong]),
 }
 
 _lock = threading.Lock()

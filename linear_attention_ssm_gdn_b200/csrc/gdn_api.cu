@@ -418,6 +418,13 @@ int gdn_flag_clear(uint32_t* engaged_flag, gdn_stream_t stream) {
                      "gdn_flag_clear");
 }
 
+int gdn_debug_set_spin_limit(long long cycles) {
+  if (cycles < 0) return fail(GDN_ERR_SHAPE, "gdn_debug_set_spin_limit: cycles < 0");
+  gdn::set_prefill_spin_limit(cycles);
+  gdn::clear_error();
+  return GDN_OK;
+}
+
 int gdn_debug_device_errors(uint32_t* out4) {
   if (!out4) return fail(GDN_ERR_NULL, "gdn_debug_device_errors: null out4");
   return cuda_status(gdn::read_device_errors(out4), "gdn_debug_device_errors");

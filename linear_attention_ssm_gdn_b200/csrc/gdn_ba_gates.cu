@@ -295,14 +295,18 @@ struct BaSmallParams {
   int k_stride, gate_stride, M, N, K, nv, vpg, ks;
 };
 
+// MB: token rows per CTA (a power of two, the smallest >= M up to
+// kBaSmallMB), so that no CTA carries predicated-off rows in its unrolled
+// loops.
+template <int MB>
 __global__ void __launch_bounds__(32 * kBaSmallNPB, 1)
     ba_gates_small_kernel(const BaSmallParams p) {
-  __shared__ float recv[kBaSmallKS][kBaSmallMB][kBaSmallNPB];
+  __shared__ float recv[kBaSmallKS][MB][kBaSmallNPB];
   const int rank = int(cluster_ctarank());
   const int grp = int(cluster_id_x());
   const int warp = int(threadIdx.x >> 5), lane = int(threadIdx.x & 31);
-  const int m0 = int(blockIdx.y) * kBaSmallMB;
-  const int mb = min(kBaSmallMB, p.M - m0);
+  const int m0 = int(blockIdx.y) * MB;
+  const int mb = min(MB, p.M - m0);
   const int n = grp * kBaSmallNPB + warp;
   // K slice of this rank, in whole 8-column (16-byte) units
   const int units = p.K / 8;
@@ -310,11 +314,13 @@ __global__ void __launch_bounds__(32 * kBaSmallNPB, 1)
   // every CTA of the cluster is running before any remote store lands
   cluster_arrive_relaxed();
   cluster_wait_acquire();
-  float acc[kBaSmallMB];
+  float acc[MB];
 #pragma unroll
-  for (int m = 0; m < kBaSmallMB; ++m) acc[m] = 0.0f;
+  for (int m = 0; m < MB; ++m) acc[m] = 0.0f;
   if (n < p.N) {
     const uint16_t* wrow = p.w + size_t(n) * p.K;
+    constexpr int kUnrollU = MB >= 32 ? 1 : 2;  // two weight loads in flight, within registers
+#pragma unroll kUnrollU
     for (int u = u0 + lane; u < u1; u += 32) {
       const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wrow) + u);
       const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(32 * kBaSmallNPB, 1)
         wf[2 * e + 1] = __uint_as_float(ww[e] & 0xffff0000u);
       }
 #pragma unroll
-      for (int m = 0; m < kBaSmallMB; ++m) {
+      for (int m = 0; m < MB; ++m) {
         if (m < mb) {
           const uint4 xv = __ldg(reinterpret_cast<const uint4*>(
                                      p.x + size_t(m0 + m) * p.k_stride) + u);
@@ -344,7 +350,7 @@ __global__ void __launch_bounds__(32 * kBaSmallNPB, 1)
   // per-token butterfly; lane 0 pushes the warp's column into rank 0
   const uint32_t base = mapa_shared(smem_u32(&recv[rank][0][warp]), 0u);
 #pragma unroll
-  for (int m = 0; m < kBaSmallMB; ++m) {
+  for (int m = 0; m < MB; ++m) {
     if (m < mb) {
       float v = acc[m];
 #pragma unroll
@@ -402,8 +408,10 @@ static cudaError_t launch_ba_gates_small(const uint16_t* x, int k_stride, const 
   ks = ks < 1 ? 1 : (ks > kBaSmallKS ? kBaSmallKS : ks);
   p.ks = ks;
   const int ngroups = (N + kBaSmallNPB - 1) / kBaSmallNPB;
+  int mb = 1;
+  while (mb < M && mb < kBaSmallMB) mb *= 2;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ngroups * ks, (M + kBaSmallMB - 1) / kBaSmallMB);
+  cfg.gridDim = dim3(ngroups * ks, (M + mb - 1) / mb);
   cfg.blockDim = dim3(32 * kBaSmallNPB);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
@@ -414,7 +422,16 @@ static cudaError_t launch_ba_gates_small(const uint16_t* x, int k_stride, const 
   attr.val.clusterDim.z = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel, p);
+  cudaError_t e;
+  switch (mb) {
+    case 1: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<1>, p); break;
+    case 2: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<2>, p); break;
+    case 4: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<4>, p); break;
+    case 8: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<8>, p); break;
+    case 16: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<16>, p); break;
+    case 32: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<32>, p); break;
+    default: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<64>, p); break;
+  }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -76,16 +76,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for phase `parity` of `bar` to complete.  Gives up (returns false) when
-// *abort becomes nonzero or after kSpinLimitCycles; on a timeout it sets
+// *abort becomes nonzero or after `limit` cycles; on a timeout it sets
 // *abort and ORs `err_bit` into *err (a global error word, may be null).
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
                                                     volatile int* abort, uint32_t* err,
-                                                    uint32_t err_bit) {
+                                                    uint32_t err_bit, long long limit) {
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort != nullptr && *abort) return false;
-    if (clock64() - t0 > kSpinLimitCycles) {
+    if (clock64() - t0 > limit) {
       if (abort != nullptr) *abort = 1;
       if (err != nullptr) atomicOr(err, err_bit);
       return false;
@@ -96,9 +96,10 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
 // The common case (the phase is already complete) stays inline: a call costs
 // the caller its live registers around the call site.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* err, uint32_t err_bit) {
+                                          uint32_t* err, uint32_t err_bit,
+                                          long long limit = kSpinLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, abort, err, err_bit);
+  return mbar_wait_slow(bar, parity, abort, err, err_bit, limit);
 }
 
 // ---------------------------------------------------------------------------
@@ -494,13 +495,14 @@ __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
 // timeout it sets *gabort and ORs `err_bit` into *err.
 static __device__ __noinline__ bool poll_geq(const uint32_t* flag, uint32_t target,
                                              volatile uint32_t* gabort, uint32_t* err,
-                                             uint32_t err_bit) {
+                                             uint32_t err_bit,
+                                             long long limit = kSpinLimitCycles) {
   if (ld_acquire_gpu(flag) >= target) return true;
   const long long t0 = clock64();
   while (true) {
     if (ld_acquire_gpu(flag) >= target) return true;
     if (*gabort != 0u) return false;
-    if (clock64() - t0 > kSpinLimitCycles) {
+    if (clock64() - t0 > limit) {
       atomicExch(const_cast<uint32_t*>(gabort), 1u);
       if (err != nullptr) atomicOr(err, err_bit);
       return false;

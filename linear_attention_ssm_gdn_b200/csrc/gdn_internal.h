@@ -75,6 +75,7 @@ struct PrefillCall {
   float* const* hT_tab;       // [num_seqs] per-sequence overrides of hT (NULL entry = not stored)
   uint16_t* o;                // [total_tokens, H_v, D], or NULL (not stored)
   int v_zero;                 // 1: v is read as zeros
+  int h0_identity;            // 1: every initial state is the identity (d_k == d_v)
   int H_k, H_v, D;
   float scale;
   int limbs;                  // 1 or 2 bf16 limbs of the state in the MMAs
@@ -84,6 +85,7 @@ struct PrefillCall {
 // Workspace (hand-off flags + L2 ring) of one launch over `units` (sequence,
 // v-head) units; the most spines a launch uses.
 size_t prefill_ring_bytes(int units);
+void set_prefill_spin_limit(long long cycles);  // 0: the default (about 2 s)
 int prefill_spine_budget();
 cudaError_t launch_prefill_call(const PrefillCall& c, cudaStream_t s);
 

@@ -90,8 +90,7 @@ constexpr uint32_t S_VN = S_HT + 32768;           // Vn^T bf16 [128 x 128B]
 constexpr uint32_t S_VNS = S_VN + 16384;          // e^{G_C - G_r} Vn^T bf16
 constexpr uint32_t S_EG = S_VNS + 16384;          // 2 x 64 f32: scale e^{G_r} per chunk
 constexpr uint32_t S_ECG = S_EG + 512;            // 2 x 64 f32: e^{G_C - G_r} per chunk
-constexpr uint32_t S_OSTG = S_ECG + 512;          // output transpose: 8 warps x 1 KB
-constexpr uint32_t S_BARS = S_OSTG + 8192;
+constexpr uint32_t S_BARS = S_ECG + 512;
 static_assert(S_HT % 1024 == 0 && STG_BYTES % 1024 == 0, "swizzled tiles are 1024-aligned");
 static_assert(STG_GATE + G_GATE_BYTES <= STG_BYTES, "stage layout");
 // ---- prep shared memory: two 128-thread item groups (item k: group k & 1)
@@ -131,9 +130,10 @@ enum {
   SB_AE = 2,       // +stage: part A free: the [W; Q] MMA is done (commit)
   SB_BF = 4,       // +stage: part B landed: K (TMA), U^T and Aqk (bulk)
   SB_BE = 6,       // +stage: part B free: dH and O2 are done (commit)
-  SB_VOFULL = 8,   // H^T [W; Q]^T done (commit)
+  SB_VOFULL = 8,   // Vn'^T = H^T W^T done (commit; two limbs: O1 too)
   SB_DHFULL = 9,   // dH = Vns^T K done (commit)
-  SB_OFULL = 10,   // +buf: O2 (and so O1) done (commit)
+  SB_OFULL = 10,   // O1 and O2 of the chunk done (commit)
+  SB_O1DONE = 11,  // O1 done: the bf16 copy of H may be overwritten (commit; one limb)
   SB_DRAIN = 12,
   SB_COUNT = 13
 };
@@ -153,8 +153,10 @@ enum {
 };
 
 // ---- TMEM columns
-// spine: [H^T W^T | O1^T] x2 (128 columns each), O2^T x2, dH^T (lane j = row j of H^T)
-constexpr uint32_t ST_VO = 0, ST_O2 = 256, ST_DH = 384;
+// spine: Vn'^T = H^T W^T (lane j = d_v index, 64 columns = chunk rows);
+// O1 = Q H and O2 = Aqk Vn as M = 64 accumulators (row r of the chunk in
+// lane 32 (r / 16) + r % 16, 128 columns = d_v); dH^T (lane j = row j of H^T)
+constexpr uint32_t ST_V = 0, ST_O1 = 128, ST_O2 = 256, ST_DH = 384;
 constexpr uint32_t PT_W = 128, PT_U = 192, PT_WG = 256;  // prep, per group: P1 x2 at 0, 64
 
 struct Params {
@@ -172,11 +174,15 @@ struct Params {
   const float* const* h0_tab;
   float* const* hT_tab;
   int v_zero;
+  int h0_identity;  // 1: every initial state is the identity (needs d_k == d_v)
   uint32_t* flags;  // abort line + S * kRing flag lines
   uint8_t* ring;    // S * kRing entries of SLOT_G bytes
   int gb_stride, num_seqs, total_tokens, H_k, H_v, D;
   int S;  // spine CTAs: blockIdx.x < S; the others are preps
   float scale;
+  // cycles a pipeline wait polls before it gives up (drains of in-flight
+  // copies and MMAs before exit always use the full kSpinLimitCycles)
+  long long spin_limit;
 };
 
 __device__ __forceinline__ uint32_t* ready_flag(const Params& p, int s, int e) {
@@ -544,66 +550,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < 8) {
       // ---------------- state warps: warp w serves TMEM lane quadrant w & 3
       // (row j of H^T) and half hh = w >> 2: columns d_k 64 hh .. 64 hh + 63 of
-      // H^T (kept in registers, f32) and chunk rows 32 hh .. 32 hh + 31 of Vn^T
-      // and of the outputs.  Per chunk c:
+      // H^T (kept in registers, f32) and chunk rows 32 hh .. 32 hh + 31 of Vn^T;
+      // for the outputs, chunk rows 16 (w & 3) .. + 15 and d_v columns
+      // 64 hh .. 64 hh + 63.  Per chunk c:
       //   H <- e^{G_C} H + dH (dH of chunk c-1, from TMEM); bf16 copy -> S_HT;
-      //   [Vn' | O1]^T = H^T [W; Q]^T  (one N = 128 MMA);
-      //   outputs of chunk c-1 while it runs;
+      //   Vn'^T = H^T W^T (MMA, the critical one), outputs of chunk c-1
+      //   while it runs (two limbs: before it, see below);
       //   Vn = U - Vn' -> Vn^T, e^{G_C - G_r} Vn^T (bf16);
-      //   dH = Vns^T K,  O2^T = Vn^T Aqk^T;
-      // warp 9 issues the MMAs right after the two named barriers, and chunk
-      // c-1's outputs are written in two halves, one under each of them.
+      //   dH^T = Vns^T K (critical), then O1 = Q H and O2 = Aqk Vn (M = 64
+      //   accumulators: every output row lands in one TMEM lane, so it is
+      //   stored from registers without a transpose through shared memory);
+      // warp 9 issues the MMAs right after the two named barriers.
       const int qd = warp & 3, hh = warp >> 2;
       const int j = 32 * qd + lane;
       const uint32_t lane_off = uint32_t(32 * qd) << 16;
       const bool jv = j < D;
-      const uint32_t ostg = sbase + S_OSTG + uint32_t(warp) * 1024;
       float* eg_s = reinterpret_cast<float*>(smem + S_EG);
       float* ecg_s = reinterpret_cast<float*>(smem + S_ECG);
-      // Outputs of chunk cl, 16 of this warp's rows 32 hh .. + 31 per call
-      // (piece pc), for the d_v lanes of its quadrant: o_r = scale e^{G_r}
-      // O1[r] + O2[r], transposed through this warp's 1 KB buffer and written
-      // as 64-byte row segments.  Piece 0 waits for the chunk's MMAs.
-      auto epilogue = [&](int cl, int pc, int t0l, int Ll, int hl) -> bool {
-        const int ob = cl & 1;
-        bool okE = true;
-        if (pc == 0) okE = mbar_wait(&bars[SB_OFULL + ob], (cl >> 1) & 1, abort_flag, err, 128u);
+      // Outputs of chunk cl: o_r = scale e^{G_r} O1[r] + O2[r].  O1 and O2
+      // hold chunk row r = 16 qd + lane in TMEM lane 32 qd + lane (lane < 16),
+      // d_v along the columns: each such lane stores its row's 64 columns of
+      // half hh straight to global memory as 16-byte vectors.
+      auto epilogue = [&](int cl, int t0l, int Ll, int hl) -> bool {
+        const bool okE = mbar_wait(&bars[SB_OFULL], cl & 1, abort_flag, err, 128u, p.spin_limit);
         tc_fence_after();
-        const float* egp = eg_s + 64 * ob;
-        const int e0 = 32 * qd;
-        {
-          const int r0 = 32 * hh + 16 * pc;
-          // every operand in registers first: the shared stores below carry a
-          // memory clobber, which would serialise loads placed between them
-          float egv[16];
+        const int r = 16 * qd + (lane & 15);
+        const float egr = eg_s[64 * (cl & 1) + r];
+        const bool live = okE && lane < 16 && r < Ll && p.o != nullptr;
+        uint16_t* orow = p.o + (size_t(t0l + r) * p.H_v + hl) * D + 64 * hh;
 #pragma unroll
-          for (int i = 0; i < 16; i += 4) {
-            const float4 e4 = *reinterpret_cast<const float4*>(egp + r0 + i);
-            egv[i] = e4.x;
-            egv[i + 1] = e4.y;
-            egv[i + 2] = e4.z;
-            egv[i + 3] = e4.w;
-          }
+        for (int qt = 0; qt < 4; ++qt) {
+          const uint32_t col = 64u * uint32_t(hh) + 16u * uint32_t(qt);
+          if (col >= uint32_t(D)) break;  // warp-uniform (d = 64: upper half empty)
           float o1[16], o2[16];
-          tmem_ld16(tmem + lane_off + ST_VO + 128u * ob + 64u + uint32_t(r0), o1);
-          tmem_ld16(tmem + lane_off + ST_O2 + 64u * ob + uint32_t(r0), o2);
+          tmem_ld16(tmem + lane_off + ST_O1 + col, o1);
+          tmem_ld16(tmem + lane_off + ST_O2 + col, o2);
           tmem_ld_wait();
-          uint32_t packed[16];
+          if (live) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 16 * qt);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            packed[i] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(egv[i], o1[i], o2[i])));
-          __syncwarp();  // the previous piece's reads of the buffer are done
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            st_shared_u16(ostg + uint32_t(i) * 64 + uint32_t(lane) * 2, uint16_t(packed[i]));
-          __syncwarp();
-#pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            const int id = lane + 32 * m, i = id >> 2, seg = id & 3;
-            const int r = r0 + i;
-            const uint4 val = ld_shared_v4(ostg + uint32_t(i) * 64 + uint32_t(seg) * 16);
-            if (okE && r < Ll && e0 < D && p.o != nullptr)
-              *reinterpret_cast<uint4*>(p.o + (size_t(t0l + r) * p.H_v + hl) * D + e0 + seg * 8) = val;
+            for (int q4 = 0; q4 < 2; ++q4) {
+              const int b8 = 8 * q4;
+              dst[q4] = make_uint4(pack_bf16x2(fmaf(egr, o1[b8], o2[b8]), fmaf(egr, o1[b8 + 1], o2[b8 + 1])),
+                                   pack_bf16x2(fmaf(egr, o1[b8 + 2], o2[b8 + 2]), fmaf(egr, o1[b8 + 3], o2[b8 + 3])),
+                                   pack_bf16x2(fmaf(egr, o1[b8 + 4], o2[b8 + 4]), fmaf(egr, o1[b8 + 5], o2[b8 + 5])),
+                                   pack_bf16x2(fmaf(egr, o1[b8 + 6], o2[b8 + 6]), fmaf(egr, o1[b8 + 7], o2[b8 + 7])));
+            }
           }
         }
         return okE;
@@ -627,6 +619,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 64; ++i)
             H[i] = (h0 != nullptr && 64 * hh + i < D) ? h0[size_t(64 * hh + i) * D] : 0.f;
+          if (p.h0_identity) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) H[i] = (64 * hh + i == j) ? 1.f : 0.f;
+          }
         }
         const int c_first = c;
         float dec_prev = 1.f;
@@ -635,10 +631,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int st = c & 1;
           const float* sg = reinterpret_cast<const float*>(smem + S_STG + st * STG_BYTES + STG_GATE);
           if (c > c_first) {  // dH of the previous chunk landed
-            ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u) && ok;
+            ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u, p.spin_limit) && ok;
             tc_fence_after();
           }
-          ok = ok && mbar_wait(&bars[SB_AF + st], (c >> 1) & 1, abort_flag, err, 16u);
+          ok = ok && mbar_wait(&bars[SB_AF + st], (c >> 1) & 1, abort_flag, err, 16u, p.spin_limit);
           if (c > c_first) {  // H <- e^{G_C} H + dH
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
@@ -653,32 +649,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           // part A is released after the [W; Q] MMA: keep the gate factors
           if (tid < 64) eg_s[64 * st + tid] = sg[tid] * p.scale;
           else if (tid < 128) ecg_s[64 * st + tid - 64] = sg[tid];
+          if constexpr (kLimbs == 1) {
+            // chunk c-1's O1 MMA (issued after dH) reads the bf16 copy of H
+            if (c > c_first)
+              ok = mbar_wait(&bars[SB_O1DONE], (c - 1) & 1, abort_flag, err, 16u, p.spin_limit) && ok;
+          }
           st_row64_bf16(sbase + S_HT + uint32_t(hh) * 16384, uint32_t(j), H);
           if constexpr (kLimbs == 2) {
-            // the previous chunk's O2 MMA reads the Vn buffers: done first
-            if (c > c_first)
-              ok = mbar_wait(&bars[SB_OFULL + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag, err,
-                             16u) && ok;
+            // The low limb goes into the Vn buffers, which the previous
+            // chunk's O2 MMA reads (and O1 of this chunk will, before this
+            // chunk's Vn lands there): chunk c-1's outputs are taken first.
+            if (c > c_first) ok = epilogue(c - 1, prev_t0, prev_L, h) && ok;
             st_row64_bf16_lo(sbase + S_VN + uint32_t(hh) * 16384, uint32_t(j), H);
           }
           fence_proxy_async_smem();
           tc_fence_before();
-          if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts [W; Q]
+          if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts Vn' (and O1)
             agreed = false;
             break;
           }
-          bool okE = true;
-          if (c > c_first) okE = epilogue(c - 1, 0, prev_t0, prev_L, h);
-          ok = ok && okE;
+          if constexpr (kLimbs == 1) {
+            if (c > c_first) ok = epilogue(c - 1, prev_t0, prev_L, h) && ok;
+          }
           // Vn = U - Vn'  ->  Vn^T and e^{G_C - G_r} Vn^T rows in bf16
-          ok = mbar_wait(&bars[SB_VOFULL], c & 1, abort_flag, err, 16u) && ok;
-          ok = mbar_wait(&bars[SB_BF + st], (c >> 1) & 1, abort_flag, err, 16u) && ok;
+          ok = mbar_wait(&bars[SB_VOFULL], c & 1, abort_flag, err, 16u, p.spin_limit) && ok;
+          ok = mbar_wait(&bars[SB_BF + st], (c >> 1) & 1, abort_flag, err, 16u, p.spin_limit) && ok;
           tc_fence_after();
           {
             const uint8_t* urow = smem + S_STG + st * STG_BYTES + STG_U;
             const float* ecp = ecg_s + 64 * st;
             float vn[32];
-            tmem_ld32(tmem + lane_off + ST_VO + 128u * st + 32u * uint32_t(hh), vn);
+            tmem_ld32(tmem + lane_off + ST_V + 32u * uint32_t(hh), vn);
             tmem_ld_wait();
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
@@ -717,11 +718,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
           tc_fence_before();
-          if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts dH, O2
+          tc_fence_before();  // this chunk's TMEM reads (Vn', outputs) before O1 / O2
+          if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts dH, O1, O2
             agreed = false;
             break;
           }
-          if (c > c_first) ok = epilogue(c - 1, 1, prev_t0, prev_L, h) && okE && ok;
           dec_prev = dec_cur;
           prev_t0 = t0;
           prev_L = min(C, te - t0);
@@ -731,7 +732,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         if (te > tb) {  // the last chunk: its update and its outputs
-          ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u) && ok;
+          ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u, p.spin_limit) && ok;
           tc_fence_after();
 #pragma unroll
           for (int q2 = 0; q2 < 2; ++q2) {
@@ -741,8 +742,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) H[32 * q2 + i] = fmaf(dec_prev, H[32 * q2 + i], d[i]);
           }
-          ok = epilogue(c - 1, 0, prev_t0, prev_L, h) && ok;
-          ok = epilogue(c - 1, 1, prev_t0, prev_L, h) && ok;
+          ok = epilogue(c - 1, prev_t0, prev_L, h) && ok;
+          tc_fence_before();
           if (!named_all(1, kSpineSync, ok)) {  // the issuer warp takes part
             ok = false;
             break;
@@ -759,12 +760,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 9) {
       // ---------------- issuer: joins the state warps' two barriers per chunk
       // (bar.red: every participant gets the same outcome) and issues
-      //   after the first:  [Vn' | O1]^T = H^T [W; Q]^T              (N = 128)
-      //   after the second: dH^T = Vns^T K (fresh), O2^T = Vn^T Aqk^T
-      const uint32_t id_vo = make_idesc_bf16(128, 128, 0, 0);
+      //   after the first:  Vn'^T = H^T W^T   (N = 64; two limbs: then O1)
+      //   after the second: dH^T = Vns^T K (fresh), then O1 = Q H and
+      //                     O2 = Aqk Vn (M = 64, N = d_v)
+      // Part A of the stage (W, Q) is free once O1 is done, part B (K, U^T,
+      // Aqk) once dH and O2 are.
+      const uint32_t id_v = make_idesc_bf16(128, 64, 0, 0);
       const uint32_t id_dh = make_idesc_bf16(128, 128, 0, 1);
-      const uint32_t id_o2 = make_idesc_bf16(128, 64, 0, 0);
+      const uint32_t id_o = make_idesc_bf16(64, 128, 0, 0);
       const bool leader = lane == 0;
+      auto issue_o1 = [&](uint32_t stg) {
+        for (int kk = 0; kk < ksteps_d; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + ST_O1, make_sdesc_sw128(stg + STG_WQ + 8192 + off, 16, 1024),
+                      make_sdesc_sw128(sbase + S_HT + off, 16, 1024), id_o, kk > 0);
+        }
+        if constexpr (kLimbs == 2) {
+          for (int kk = 0; kk < ksteps_d; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_bf16_ss(tmem + ST_O1, make_sdesc_sw128(stg + STG_WQ + 8192 + off, 16, 1024),
+                        make_sdesc_sw128(sbase + S_VN + off, 16, 1024), id_o, 1u);
+          }
+        }
+      };
       int c = 0;
       for (int u = s; u < units; u += p.S) {
         int tb, te;
@@ -781,18 +799,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             for (int kk = 0; kk < ksteps_d; ++kk) {
               const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_bf16_ss(tmem + ST_VO + 128u * st, make_sdesc_sw128(sbase + S_HT + off, 16, 1024),
-                          make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_vo, kk > 0);
+              mma_bf16_ss(tmem + ST_V, make_sdesc_sw128(sbase + S_HT + off, 16, 1024),
+                          make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_v, kk > 0);
             }
             if constexpr (kLimbs == 2) {
               for (int kk = 0; kk < ksteps_d; ++kk) {
                 const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16_ss(tmem + ST_VO + 128u * st, make_sdesc_sw128(sbase + S_VN + off, 16, 1024),
-                            make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_vo, 1u);
+                mma_bf16_ss(tmem + ST_V, make_sdesc_sw128(sbase + S_VN + off, 16, 1024),
+                            make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_v, 1u);
               }
+              issue_o1(stg);  // reads the low limb before this chunk's Vn lands on it
+              mma_commit(&bars[SB_AE + st]);
             }
             mma_commit(&bars[SB_VOFULL]);
-            mma_commit(&bars[SB_AE + st]);
           }
           __syncwarp();
           if (!named_all(1, kSpineSync, true)) {
@@ -805,11 +824,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_bf16_ss(tmem + ST_DH, make_sdesc_sw128(sbase + S_VNS + kk * 32, 16, 1024),
                           make_sdesc_sw128(stg + STG_K + kk * 2048, 8192, 1024), id_dh, kk > 0);
             mma_commit(&bars[SB_DHFULL]);
+            if constexpr (kLimbs == 1) {
+              issue_o1(stg);
+              mma_commit(&bars[SB_O1DONE]);
+              mma_commit(&bars[SB_AE + st]);
+            }
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(tmem + ST_O2 + 64u * st,
-                          make_sdesc_sw128(sbase + S_VN + kk * 32, 16, 1024),
-                          make_sdesc_sw128(stg + STG_AQK + kk * 32, 16, 1024), id_o2, kk > 0);
-            mma_commit(&bars[SB_OFULL + st]);
+              mma_bf16_ss(tmem + ST_O2, make_sdesc_sw128(stg + STG_AQK + kk * 32, 16, 1024),
+                          make_sdesc_sw128(sbase + S_VN + kk * 32, 16, 1024), id_o, kk > 0);
+            mma_commit(&bars[SB_OFULL]);
             mma_commit(&bars[SB_BE + st]);
           }
           __syncwarp();
@@ -840,7 +863,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint8_t* src = ring_entry(p, s, cc % kRing);
           // ---- part A
           if (cc >= 2) {
-            ok = mbar_wait(&bars[SB_AE + st], ((cc >> 1) & 1) ^ 1, abort_flag, err, 1u);
+            ok = mbar_wait(&bars[SB_AE + st], ((cc >> 1) & 1) ^ 1, abort_flag, err, 1u, p.spin_limit);
             if (!ok) break;
           }
           uint64_t* fa = &bars[SB_AF + st];
@@ -850,7 +873,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int b = 0; b < nbox; ++b)
             tma_load_3d(stg + STG_WQ + b * 16384 + 8192, &tm_q, fa, b * 64, hk, fd.t0);
           issued_a = cc + 1;
-          ok = poll_geq(ready_flag(p, s, cc % kRing), uint32_t(cc + 1), gabort, err, 1u);
+          ok = poll_geq(ready_flag(p, s, cc % kRing), uint32_t(cc + 1), gabort, err, 1u, p.spin_limit);
           if (!ok) {  // the phase still completes once the Q tiles landed
             mbar_arrive(fa);
             break;
@@ -862,7 +885,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_load_g2s(stg + STG_GATE, src + G_GATE, G_GATE_BYTES, fa);
           // ---- part B
           if (cc >= 2) {
-            ok = mbar_wait(&bars[SB_BE + st], ((cc >> 1) & 1) ^ 1, abort_flag, err, 1u);
+            ok = mbar_wait(&bars[SB_BE + st], ((cc >> 1) & 1) ^ 1, abort_flag, err, 1u, p.spin_limit);
             if (!ok) break;
             // chunk cc - 2 is fully consumed: its ring entry may be reused
             st_release_gpu(free_flag(p, s, (cc - 2) % kRing), uint32_t(cc - 1));
@@ -904,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       while (it.ok && ok) {
         const int k = it.k, t = k % 3, g = k & 1, gb = (k >> 1) & 1;
-        ok = k < 3 || mbar_wait(&bars[PB_STORED + t], ((k / 3) & 1) ^ 1, abort_flag, err, 1u);
+        ok = k < 3 || mbar_wait(&bars[PB_STORED + t], ((k / 3) & 1) ^ 1, abort_flag, err, 1u, p.spin_limit);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
@@ -1050,7 +1073,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (prog) {
             last = clock64();
           } else {
-            if (clock64() - last > kSpinLimitCycles) {
+            if (clock64() - last > p.spin_limit) {
               *abort_flag = 1;
               atomicExch(const_cast<uint32_t*>(gabort), 1u);
               atomicOr(err, 2u);
@@ -1073,9 +1096,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         while (it.ok && ok) {
           const int k = it.k, t = k % 3, g = k & 1, kg = k >> 1;
           const int e = it.j % kRing;
-          ok = mbar_wait(&bars[PB_STAGED + g], kg & 1, abort_flag, err, 4u);
+          ok = mbar_wait(&bars[PB_STAGED + g], kg & 1, abort_flag, err, 4u, p.spin_limit);
           if (ok && it.j >= kRing)  // entry e is free once the spine copied item j - kRing
-            ok = poll_geq(free_flag(p, it.s, e), uint32_t(it.j - kRing + 1), gabort, err, 4u);
+            ok = poll_geq(free_flag(p, it.s, e), uint32_t(it.j - kRing + 1), gabort, err, 4u, p.spin_limit);
           if (!ok) break;
           fence_proxy_async_global();
           uint8_t* dst = ring_entry(p, it.s, e);
@@ -1117,9 +1140,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // gates written, P1 done; the group's Aqk buffer was read by the store
         // of its previous item k - 2
         const bool ready =
-            mbar_wait(&bars[PB_GATEF + 2 * g + pb], (kg >> 1) & 1, abort_flag, err, 4u) &&
-            mbar_wait(&bars[PB_P1F + 2 * g + pb], (kg >> 1) & 1, abort_flag, err, 4u) &&
-            (k < 2 || mbar_wait(&bars[PB_STORED + (k - 2) % 3], ((k - 2) / 3) & 1, abort_flag, err, 4u));
+            mbar_wait(&bars[PB_GATEF + 2 * g + pb], (kg >> 1) & 1, abort_flag, err, 4u, p.spin_limit) &&
+            mbar_wait(&bars[PB_P1F + 2 * g + pb], (kg >> 1) & 1, abort_flag, err, 4u, p.spin_limit) &&
+            (k < 2 || mbar_wait(&bars[PB_STORED + (k - 2) % 3], ((k - 2) / 3) & 1, abort_flag, err, 4u, p.spin_limit));
         if (!named_all(gbar, 128, ready)) break;
         tc_fence_after();
         // ---- P1 row pt: K K^T (pt < 64) or Q K^T (pt >= 64), times e^{G_r - G_s}
@@ -1213,7 +1236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         mbar_arrive(&bars[PB_TREADY + g]);
         // ---- W (row-major), U^T into [0, 32 KB) of the item's set
-        if (!named_all(gbar, 128, mbar_wait(&bars[PB_WUF + g], kg & 1, abort_flag, err, 4u))) break;
+        if (!named_all(gbar, 128, mbar_wait(&bars[PB_WUF + g], kg & 1, abort_flag, err, 4u, p.spin_limit))) break;
         tc_fence_after();
         {
           uint8_t* wcol = set + G_W + uint32_t(pt >> 6) * 8192;
@@ -1299,6 +1322,12 @@ size_t flag_bytes(int S) { return (size_t(1 + S * kRing) * kFlagLine + 1023) / 1
 
 }  // namespace
 
+// Diagnostics only (gdn_debug_set_spin_limit): a shorter give-up time for the
+// prefill's pipeline waits, so that a test can make them run out.
+static long long g_spin_limit_override = 0;
+
+void set_prefill_spin_limit(long long cycles) { g_spin_limit_override = cycles > 0 ? cycles : 0; }
+
 size_t prefill_ring_bytes(int units) {
   int G = 0, S = 0;
   plan(units, &G, &S);
@@ -1345,6 +1374,7 @@ cudaError_t launch_prefill_call(const PrefillCall& c, cudaStream_t s) {
   p.h0_tab = c.h0_tab;
   p.hT_tab = c.hT_tab;
   p.v_zero = c.v_zero;
+  p.h0_identity = c.h0_identity;
   p.flags = static_cast<uint32_t*>(c.workspace);
   p.ring = static_cast<uint8_t*>(c.workspace) + flag_bytes(S);
   p.gb_stride = c.gb_stride;
@@ -1355,6 +1385,7 @@ cudaError_t launch_prefill_call(const PrefillCall& c, cudaStream_t s) {
   p.D = D;
   p.S = S;
   p.scale = c.scale;
+  p.spin_limit = g_spin_limit_override > 0 ? g_spin_limit_override : kSpinLimitCycles;
   // The hand-off counters start from zero on every launch.
   e = cudaMemsetAsync(c.workspace, 0, flag_bytes(S), s);
   if (e != cudaSuccess) return e;

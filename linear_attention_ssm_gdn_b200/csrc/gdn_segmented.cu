@@ -9,8 +9,9 @@
 //   A1  every segment but the last runs its chunks from a given entry: the
 //       first from the caller's h0 (its outputs are final), the others from
 //       zero, which leaves L_s (the state the segment adds) in its final state;
-//   A2  every middle segment runs its chunks on v = 0 from H = I, which leaves
-//       M_s (the segment's transition) in its final state;
+//   A2  every middle segment runs its chunks on v = 0 from H = I (the kernel's
+//       identity-initial-state switch), which leaves M_s (the segment's
+//       transition) in its final state;
 //   C   entry(1) = L_0 (the first segment's true exit) and
 //       entry(s + 1) = M_s entry(s) + L_s, a short sequential combine in f32;
 //   B   every segment but the first runs again from its true entry state and
@@ -38,7 +39,7 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 // Workspace layout of a segmented call (byte offsets, all 256-aligned).
 struct SegLayout {
-  size_t ring, segA1, segA2, segB, tabs, ident, loc, trans, total;
+  size_t ring, segA1, segA2, segB, tabs, loc, trans, total;
 };
 
 SegLayout seg_layout(int num_seqs, int H_v, int D, int S) {
@@ -56,8 +57,6 @@ SegLayout seg_layout(int num_seqs, int H_v, int D, int S) {
   off += align256(n1 * sizeof(int2));
   L.tabs = off;  // A1 h0, A1 hT, A2 h0, A2 hT, B h0, B hT: n1 pointers each
   off += align256(6 * n1 * sizeof(void*));
-  L.ident = off;
-  off += align256(state);
   L.loc = off;  // L_s of segments 0 .. S-2, overwritten in place by entry(s + 1)
   off += align256(n1 * state);
   L.trans = off;  // M_s of segments 1 .. S-2
@@ -67,11 +66,11 @@ SegLayout seg_layout(int num_seqs, int H_v, int D, int S) {
 }
 
 // One CTA: the segment ranges and state-pointer tables of the three launches,
-// and the identity initial state of A2, from the device cu_seqlens.
+// from the device cu_seqlens.
 __global__ void segment_plan_kernel(const int32_t* cu_seqlens, int num_seqs, int total_tokens,
                                     int S, int H_v, int D, const float* h0, float* hT,
                                     int2* segA1, int2* segA2, int2* segB, void** tabs,
-                                    float* ident, float* loc, float* trans) {
+                                    float* loc, float* trans) {
   const size_t state = size_t(H_v) * D * D;
   const size_t n1 = size_t(num_seqs) * (S - 1);
   // six tables of n1 state pointers (initial states are only read)
@@ -97,7 +96,7 @@ __global__ void segment_plan_kernel(const int32_t* cu_seqlens, int num_seqs, int
     for (int s = 1; s < S - 1; ++s) {  // A2: segments 1 .. S-2
       const size_t i = size_t(n) * (S - 2) + (s - 1);
       segA2[i] = make_int2(t(s), t(s + 1));
-      a2_h0[i] = ident;
+      a2_h0[i] = nullptr;  // the identity, by the launch's switch
       a2_hT[i] = trans + i * state;
     }
     for (int s = 1; s < S; ++s) {  // B: segments 1 .. S-1 from entry(s)
@@ -107,29 +106,26 @@ __global__ void segment_plan_kernel(const int32_t* cu_seqlens, int num_seqs, int
       b_hT[i] = (s == S - 1 && hT != nullptr) ? hT + size_t(n) * state : nullptr;
     }
   }
-  for (size_t x = threadIdx.x; x < state; x += blockDim.x) {
-    const size_t ij = x % (size_t(D) * D);
-    ident[x] = (ij / D == ij % D) ? 1.0f : 0.0f;
-  }
 }
 
 // entry(s + 1) = M_s entry(s) + L_s for s = 1 .. S-2, in place over L_s;
-// entry(1) = L_0.  grid = (num_seqs * H_v, D / 32): CTA (unit, cb) owns
-// columns 32 cb .. 32 cb + 31 of the unit's states (the columns of a state
+// entry(1) = L_0.  grid = (num_seqs * H_v, D / 16): CTA (unit, cb) owns
+// columns 16 cb .. 16 cb + 15 of the unit's states (the columns of a state
 // evolve independently), in f32.  Per step the CTA stages M_s in shared
 // memory (rows padded by one float: conflict-free row-parallel reads) and
-// thread t computes D / 8 consecutive columns of row t / (256 / D).
-constexpr int kCombCols = 32;
+// thread t computes D / 16 consecutive columns of row t / (256 / D).
+constexpr int kCombCols = 16;
 
-__global__ void __launch_bounds__(256) segment_combine_kernel(int S, int H_v, int D,
-                                                              float* loc, const float* trans) {
-  extern __shared__ float cm[];  // Ms [D][D + 1], then E [D][kCombCols]
+template <int D>
+__global__ void __launch_bounds__(256) segment_combine_kernel(int S, int H_v, float* loc,
+                                                              const float* trans) {
+  constexpr int CPT = D * kCombCols / 256;  // columns per thread: 8 (D = 128) or 4 (D = 64)
+  extern __shared__ float cm[];             // Ms [D][D + 1], then E [D][kCombCols]
   float* Ms = cm;
   float* E = cm + D * (D + 1);
   const int unit = blockIdx.x, n = unit / H_v, h = unit % H_v, c0 = kCombCols * blockIdx.y;
   const size_t state = size_t(H_v) * D * D, head = size_t(h) * D * D;
-  const int cpt = D * kCombCols / 256;   // columns per thread: 16 (D = 128) or 8 (D = 64)
-  const int i = threadIdx.x / (kCombCols / cpt), cb = (threadIdx.x % (kCombCols / cpt)) * cpt;
+  const int i = threadIdx.x / (kCombCols / CPT), cb = (threadIdx.x % (kCombCols / CPT)) * CPT;
   const float* L0 = loc + (size_t(n) * (S - 1)) * state + head;
   for (int idx = threadIdx.x; idx < D * kCombCols; idx += blockDim.x)
     E[idx] = L0[size_t(idx / kCombCols) * D + c0 + idx % kCombCols];
@@ -146,17 +142,25 @@ __global__ void __launch_bounds__(256) segment_combine_kernel(int S, int H_v, in
       dst[3] = m.w;
     }
     __syncthreads();  // M staged; E holds entry(s)
-    float acc[16];
-    for (int j = 0; j < cpt; ++j) acc[j] = Ls[size_t(i) * D + c0 + cb + j];
+    float acc[CPT];
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) acc[j] = Ls[size_t(i) * D + c0 + cb + j];
+#pragma unroll 4
     for (int k = 0; k < D; ++k) {
       const float m = Ms[i * (D + 1) + k];
-      const float* er = E + k * kCombCols + cb;
+      const float4* er = reinterpret_cast<const float4*>(E + k * kCombCols + cb);
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
-        if (j < cpt) acc[j] = fmaf(m, er[j], acc[j]);
+      for (int j4 = 0; j4 < CPT / 4; ++j4) {
+        const float4 e = er[j4];
+        acc[4 * j4 + 0] = fmaf(m, e.x, acc[4 * j4 + 0]);
+        acc[4 * j4 + 1] = fmaf(m, e.y, acc[4 * j4 + 1]);
+        acc[4 * j4 + 2] = fmaf(m, e.z, acc[4 * j4 + 2]);
+        acc[4 * j4 + 3] = fmaf(m, e.w, acc[4 * j4 + 3]);
+      }
     }
     __syncthreads();  // every read of Ms and E for this step is done
-    for (int j = 0; j < cpt; ++j) {
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
       E[i * kCombCols + cb + j] = acc[j];
       Ls[size_t(i) * D + c0 + cb + j] = acc[j];
     }
@@ -174,15 +178,19 @@ size_t prefill_segmented_workspace_bytes(int total_tokens, int num_seqs, int H_v
 
 int prefill_auto_segments(int total_tokens, int num_seqs, int H_v) {
   // Two levels pay when the single-level launch leaves most spines idle and
-  // every segment still spans a few chunks: A1, A2 and B each run about
-  // nc / S chunk steps per spine, against nc for one level.
+  // the sequences are long: A1, A2 and B each run about nc / S chunk steps
+  // per spine against nc for one level, but each launch also costs a fixed
+  // start-up (the first ring entries, the last chunk's outputs) of some ten
+  // chunk steps, and the combine S - 2 small products.  Measured on a B200
+  // with 6 units: 4576 tokens (72 chunks) are faster in one level, so every
+  // segment must span at least 24 chunks.
   const int units = num_seqs * H_v;
   const int budget = prefill_spine_budget();
   if (units <= 0 || units * 3 > budget) return 1;
   const int avg_chunks = (total_tokens / num_seqs + kChunk - 1) / kChunk;
   int S = budget / units + 1;  // units * (S - 1) <= budget
   if (S > 8) S = 8;
-  if (S > avg_chunks / 3) S = avg_chunks / 3;
+  if (S > avg_chunks / 24) S = avg_chunks / 24;
   return S >= 4 ? S : 1;
 }
 
@@ -194,12 +202,11 @@ cudaError_t launch_prefill_segmented(const PrefillCall& c, int S, void* workspac
   int2* segA2 = reinterpret_cast<int2*>(ws + L.segA2);
   int2* segB = reinterpret_cast<int2*>(ws + L.segB);
   void** tabs = reinterpret_cast<void**>(ws + L.tabs);
-  float* ident = reinterpret_cast<float*>(ws + L.ident);
   float* loc = reinterpret_cast<float*>(ws + L.loc);
   float* trans = reinterpret_cast<float*>(ws + L.trans);
   const size_t n1 = size_t(c.num_seqs) * (S - 1);
   segment_plan_kernel<<<1, 256, 0, s>>>(c.cu_seqlens, c.num_seqs, c.total_tokens, S, c.H_v, c.D,
-                                        c.h0, c.hT, segA1, segA2, segB, tabs, ident, loc, trans);
+                                        c.h0, c.hT, segA1, segA2, segB, tabs, loc, trans);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -222,14 +229,14 @@ cudaError_t launch_prefill_segmented(const PrefillCall& c, int S, void* workspac
     a2.hT_tab = reinterpret_cast<float* const*>(tabs + 3 * n1);
     a2.o = nullptr;
     a2.v_zero = 1;
+    a2.h0_identity = 1;
     if ((e = launch_prefill_call(a2, s)) != cudaSuccess) return e;
     const int smem = int((c.D * (c.D + 1) + c.D * kCombCols) * sizeof(float));
-    if ((e = cudaFuncSetAttribute(segment_combine_kernel,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+    auto comb = c.D == 128 ? segment_combine_kernel<128> : segment_combine_kernel<64>;
+    if ((e = cudaFuncSetAttribute(comb, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
       return e;
-    segment_combine_kernel<<<dim3(c.num_seqs * c.H_v, c.D / kCombCols), 256, smem, s>>>(
-        S, c.H_v, c.D, loc, trans);
+    comb<<<dim3(c.num_seqs * c.H_v, c.D / kCombCols), 256, smem, s>>>(S, c.H_v, loc, trans);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
 

@@ -284,3 +284,10 @@ def debug_device_errors() -> list[int]:
     rc = _lib.load().gdn_debug_device_errors(ctypes.addressof(out))
     _lib.check("gdn_debug_device_errors", rc)
     return list(out)
+
+
+def debug_set_spin_limit(cycles: int) -> None:
+    """Give-up time (clock cycles) of the prefill's pipeline waits for the
+    launches that follow; 0 restores the default (about 2 s).  Diagnostics."""
+    rc = _lib.load().gdn_debug_set_spin_limit(int(cycles))
+    _lib.check("gdn_debug_set_spin_limit", rc)

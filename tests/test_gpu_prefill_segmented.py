@@ -7,7 +7,7 @@ sequence: ragged and empty sequences, no initial state, an in-place final
 state, weak decay with a large initial state (where every segment's
 transition matters), and the two-limb spine.  The timing test prints the
 single-level and two-level launch times on a tensor-parallel-sized shard of
-the pages' geometry (6 v-heads, 4576 tokens).
+the pages' geometry (6 v-heads) over a 16384-token sequence.
 """
 import numpy as np
 import pytest
@@ -85,7 +85,7 @@ def test_segmented_matches_single_level_and_is_chosen_for_few_heads():
     and call agree), and the result matches the single-level scan within the
     tolerances; the two launch times are printed."""
     lib = _lib.load()
-    T, H_k, H_v = 4576, 2, 6
+    T, H_k, H_v = 16384, 2, 6
     auto = int(lib.gdn_chunk_prefill_workspace_bytes(T, 1, H_k, H_v, 128, 128))
     single = int(lib.gdn_chunk_prefill_segmented_workspace_bytes(T, 1, H_k, H_v, 128, 128, 1))
     assert auto > single  # the per-segment states live in the workspace

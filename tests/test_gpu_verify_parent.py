@@ -1,6 +1,6 @@
 """GPU checks of the parent (not write-on-accept) verify and the fold's restore
-branch (page "ssm_gdn_woa.rs", gdn_wy4_fold: with the engaged word clear a
-partial accept restores Hi(na - 1) from hi_tables), through the C ABI.
+branch, through the C ABI (page "ssm_gdn_woa.rs", gdn_wy4_fold doc: a clear
+engaged word sends the fold to the kept intermediate states in hi_tables).
 
 Against the f64 oracle (prefill tolerances): the outputs, every kept
 intermediate state Hi(0..2) = the state after 1..3 rows, and the live state
