@@ -90,7 +90,8 @@ constexpr uint32_t S_VN = S_HT + 32768;           // Vn^T bf16 [128 x 128B]
 constexpr uint32_t S_VNS = S_VN + 16384;          // e^{G_C - G_r} Vn^T bf16
 constexpr uint32_t S_EG = S_VNS + 16384;          // 2 x 64 f32: scale e^{G_r} per chunk
 constexpr uint32_t S_ECG = S_EG + 512;            // 2 x 64 f32: e^{G_C - G_r} per chunk
-constexpr uint32_t S_BARS = S_ECG + 512;
+constexpr uint32_t S_OSTG = S_ECG + 512;          // output transpose: 8 warps x 1 KB
+constexpr uint32_t S_BARS = S_OSTG + 8192;
 static_assert(S_HT % 1024 == 0 && STG_BYTES % 1024 == 0, "swizzled tiles are 1024-aligned");
 static_assert(STG_GATE + G_GATE_BYTES <= STG_BYTES, "stage layout");
 // ---- prep shared memory: two 128-thread item groups (item k: group k & 1)
@@ -130,10 +131,9 @@ enum {
   SB_AE = 2,       // +stage: part A free: the [W; Q] MMA is done (commit)
   SB_BF = 4,       // +stage: part B landed: K (TMA), U^T and Aqk (bulk)
   SB_BE = 6,       // +stage: part B free: dH and O2 are done (commit)
-  SB_VOFULL = 8,   // Vn'^T = H^T W^T done (commit; two limbs: O1 too)
+  SB_VOFULL = 8,   // H^T [W; Q]^T done (commit)
   SB_DHFULL = 9,   // dH = Vns^T K done (commit)
-  SB_OFULL = 10,   // O1 and O2 of the chunk done (commit)
-  SB_O1DONE = 11,  // O1 done: the bf16 copy of H may be overwritten (commit; one limb)
+  SB_OFULL = 10,   // +buf: O2 (and so O1) done (commit)
   SB_DRAIN = 12,
   SB_COUNT = 13
 };
@@ -153,10 +153,8 @@ enum {
 };
 
 // ---- TMEM columns
-// spine: Vn'^T = H^T W^T (lane j = d_v index, 64 columns = chunk rows);
-// O1 = Q H and O2 = Aqk Vn as M = 64 accumulators (row r of the chunk in
-// lane 32 (r / 16) + r % 16, 128 columns = d_v); dH^T (lane j = row j of H^T)
-constexpr uint32_t ST_V = 0, ST_O1 = 128, ST_O2 = 256, ST_DH = 384;
+// spine: [H^T W^T | O1^T] x2 (128 columns each), O2^T x2, dH^T (lane j = row j of H^T)
+constexpr uint32_t ST_VO = 0, ST_O2 = 256, ST_DH = 384;
 constexpr uint32_t PT_W = 128, PT_U = 192, PT_WG = 256;  // prep, per group: P1 x2 at 0, 64
 
 struct Params {
@@ -195,8 +193,9 @@ __device__ __forceinline__ uint8_t* ring_entry(const Params& p, int s, int e) {
   return p.ring + size_t(s * kRing + e) * SLOT_G;
 }
 
+template <bool kSeg>
 __device__ __forceinline__ void seq_range(const Params& p, int n, int& b, int& e) {
-  if (p.seg != nullptr) {
+  if (kSeg && p.seg != nullptr) {
     const int2 r = p.seg[n];
     b = min(max(r.x, 0), p.total_tokens);
     e = min(max(r.y, b), p.total_tokens);
@@ -206,9 +205,10 @@ __device__ __forceinline__ void seq_range(const Params& p, int n, int& b, int& e
   e = min(max(p.cu_seqlens[n + 1], b), p.total_tokens);
 }
 
+template <bool kSeg>
 __device__ __forceinline__ int unit_chunks(const Params& p, int u) {
   int b, e;
-  seq_range(p, u / p.H_v, b, e);
+  seq_range<kSeg>(p, u / p.H_v, b, e);
   return (e - b + C - 1) / C;
 }
 
@@ -219,13 +219,15 @@ struct ChunkIter {
   bool ok;
 };
 
+template <bool kSeg>
 __device__ __forceinline__ void it_load_unit(ChunkIter& it, const Params& p) {
   it.n = it.u / p.H_v;
   it.h = it.u % p.H_v;
-  seq_range(p, it.n, it.tb, it.te);
+  seq_range<kSeg>(p, it.n, it.tb, it.te);
   it.t0 = it.tb;
 }
 
+template <bool kSeg>
 __device__ __forceinline__ void it_skip_empty(ChunkIter& it, const Params& p) {
   const int units = p.num_seqs * p.H_v;
   while (it.ok && it.t0 >= it.te) {
@@ -234,22 +236,24 @@ __device__ __forceinline__ void it_skip_empty(ChunkIter& it, const Params& p) {
       it.ok = false;
       break;
     }
-    it_load_unit(it, p);
+    it_load_unit<kSeg>(it, p);
   }
 }
 
+template <bool kSeg>
 __device__ __forceinline__ void it_start(ChunkIter& it, const Params& p, int s) {
   it.u = s;
   it.c = 0;
   it.ok = s < p.num_seqs * p.H_v;
-  if (it.ok) it_load_unit(it, p);
-  it_skip_empty(it, p);
+  if (it.ok) it_load_unit<kSeg>(it, p);
+  it_skip_empty<kSeg>(it, p);
 }
 
+template <bool kSeg>
 __device__ __forceinline__ void it_next(ChunkIter& it, const Params& p) {
   it.t0 += C;
   ++it.c;
-  it_skip_empty(it, p);
+  it_skip_empty<kSeg>(it, p);
 }
 
 // The items of one prep CTA: global item i = j * S + s (chunk j of spine s),
@@ -259,6 +263,7 @@ struct PrepIter {
   bool ok;
 };
 
+template <bool kSeg>
 __device__ __forceinline__ bool pi_fill(PrepIter& it, const Params& p, const int* sJ, int iend) {
   while (it.i < iend) {
     const int s = it.i % p.S, j = it.i / p.S;
@@ -266,10 +271,10 @@ __device__ __forceinline__ bool pi_fill(PrepIter& it, const Params& p, const int
       const int units = p.num_seqs * p.H_v;
       int jj = j;
       for (int u = s; u < units; u += p.S) {
-        const int nc = unit_chunks(p, u);
+        const int nc = unit_chunks<kSeg>(p, u);
         if (jj < nc) {
           int tb, te;
-          seq_range(p, u / p.H_v, tb, te);
+          seq_range<kSeg>(p, u / p.H_v, tb, te);
           it.s = s;
           it.j = j;
           it.h = u % p.H_v;
@@ -285,22 +290,25 @@ __device__ __forceinline__ bool pi_fill(PrepIter& it, const Params& p, const int
   return false;
 }
 
+template <bool kSeg>
 __device__ __forceinline__ void pi_start(PrepIter& it, const Params& p, const int* sJ, int iend,
                                          int prank) {
   it.i = prank;
   it.k = 0;
-  it.ok = pi_fill(it, p, sJ, iend);
+  it.ok = pi_fill<kSeg>(it, p, sJ, iend);
 }
 
+template <bool kSeg>
 __device__ __forceinline__ void pi_next(PrepIter& it, const Params& p, const int* sJ, int iend) {
   it.i += gridDim.x - p.S;
   ++it.k;
-  it.ok = pi_fill(it, p, sJ, iend);
+  it.ok = pi_fill<kSeg>(it, p, sJ, iend);
 }
 
+template <bool kSeg>
 __device__ __forceinline__ void pi_align(PrepIter& it, const Params& p, const int* sJ, int iend,
                                          int w) {
-  while (it.ok && (it.k & 1) != w) pi_next(it, p, sJ, iend);
+  while (it.ok && (it.k & 1) != w) pi_next<kSeg>(it, p, sJ, iend);
 }
 
 // Write 64 bf16 values as a 128-byte row of a 128B-swizzled tile (local smem).
@@ -478,7 +486,7 @@ using namespace pf;
 // two bf16 limbs hi + lo (page "ssm_gdn_tc_route.rs": the _tcfuse spine uses
 // one limb of S_c, the _tcfuse_x2 spine two), the low limb staged in the Vn
 // buffers, which that MMA does not read.
-template <int kLimbs>
+template <int kLimbs, bool kSeg>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -529,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (!spine) {
     for (int s = tid; s < p.S; s += kThreads) {
       int J = 0;
-      for (int u = s; u < units; u += p.S) J += unit_chunks(p, u);
+      for (int u = s; u < units; u += p.S) J += unit_chunks<kSeg>(p, u);
       sJ[s] = J;
     }
   }
@@ -550,52 +558,66 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < 8) {
       // ---------------- state warps: warp w serves TMEM lane quadrant w & 3
       // (row j of H^T) and half hh = w >> 2: columns d_k 64 hh .. 64 hh + 63 of
-      // H^T (kept in registers, f32) and chunk rows 32 hh .. 32 hh + 31 of Vn^T;
-      // for the outputs, chunk rows 16 (w & 3) .. + 15 and d_v columns
-      // 64 hh .. 64 hh + 63.  Per chunk c:
+      // H^T (kept in registers, f32) and chunk rows 32 hh .. 32 hh + 31 of Vn^T
+      // and of the outputs.  Per chunk c:
       //   H <- e^{G_C} H + dH (dH of chunk c-1, from TMEM); bf16 copy -> S_HT;
-      //   Vn'^T = H^T W^T (MMA, the critical one), outputs of chunk c-1
-      //   while it runs (two limbs: before it, see below);
+      //   [Vn' | O1]^T = H^T [W; Q]^T  (one N = 128 MMA);
+      //   outputs of chunk c-1 while it runs;
       //   Vn = U - Vn' -> Vn^T, e^{G_C - G_r} Vn^T (bf16);
-      //   dH^T = Vns^T K (critical), then O1 = Q H and O2 = Aqk Vn (M = 64
-      //   accumulators: every output row lands in one TMEM lane, so it is
-      //   stored from registers without a transpose through shared memory);
-      // warp 9 issues the MMAs right after the two named barriers.
+      //   dH = Vns^T K,  O2^T = Vn^T Aqk^T;
+      // warp 9 issues the MMAs right after the two named barriers, and chunk
+      // c-1's outputs are written in two halves, one under each of them.
       const int qd = warp & 3, hh = warp >> 2;
       const int j = 32 * qd + lane;
       const uint32_t lane_off = uint32_t(32 * qd) << 16;
       const bool jv = j < D;
+      const uint32_t ostg = sbase + S_OSTG + uint32_t(warp) * 1024;
       float* eg_s = reinterpret_cast<float*>(smem + S_EG);
       float* ecg_s = reinterpret_cast<float*>(smem + S_ECG);
-      // Outputs of chunk cl: o_r = scale e^{G_r} O1[r] + O2[r].  O1 and O2
-      // hold chunk row r = 16 qd + lane in TMEM lane 32 qd + lane (lane < 16),
-      // d_v along the columns: each such lane stores its row's 64 columns of
-      // half hh straight to global memory as 16-byte vectors.
-      auto epilogue = [&](int cl, int t0l, int Ll, int hl) -> bool {
-        const bool okE = mbar_wait(&bars[SB_OFULL], cl & 1, abort_flag, err, 128u, p.spin_limit);
+      // Outputs of chunk cl, 16 of this warp's rows 32 hh .. + 31 per call
+      // (piece pc), for the d_v lanes of its quadrant: o_r = scale e^{G_r}
+      // O1[r] + O2[r], transposed through this warp's 1 KB buffer and written
+      // as 64-byte row segments.  Piece 0 waits for the chunk's MMAs.
+      auto epilogue = [&](int cl, int pc, int t0l, int Ll, int hl) -> bool {
+        const int ob = cl & 1;
+        bool okE = true;
+        if (pc == 0) okE = mbar_wait(&bars[SB_OFULL + ob], (cl >> 1) & 1, abort_flag, err, 128u, p.spin_limit);
         tc_fence_after();
-        const int r = 16 * qd + (lane & 15);
-        const float egr = eg_s[64 * (cl & 1) + r];
-        const bool live = okE && lane < 16 && r < Ll && p.o != nullptr;
-        uint16_t* orow = p.o + (size_t(t0l + r) * p.H_v + hl) * D + 64 * hh;
+        const float* egp = eg_s + 64 * ob;
+        const int e0 = 32 * qd;
+        {
+          const int r0 = 32 * hh + 16 * pc;
+          // every operand in registers first: the shared stores below carry a
+          // memory clobber, which would serialise loads placed between them
+          float egv[16];
 #pragma unroll
-        for (int qt = 0; qt < 4; ++qt) {
-          const uint32_t col = 64u * uint32_t(hh) + 16u * uint32_t(qt);
-          if (col >= uint32_t(D)) break;  // warp-uniform (d = 64: upper half empty)
+          for (int i = 0; i < 16; i += 4) {
+            const float4 e4 = *reinterpret_cast<const float4*>(egp + r0 + i);
+            egv[i] = e4.x;
+            egv[i + 1] = e4.y;
+            egv[i + 2] = e4.z;
+            egv[i + 3] = e4.w;
+          }
           float o1[16], o2[16];
-          tmem_ld16(tmem + lane_off + ST_O1 + col, o1);
-          tmem_ld16(tmem + lane_off + ST_O2 + col, o2);
+          tmem_ld16(tmem + lane_off + ST_VO + 128u * ob + 64u + uint32_t(r0), o1);
+          tmem_ld16(tmem + lane_off + ST_O2 + 64u * ob + uint32_t(r0), o2);
           tmem_ld_wait();
-          if (live) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + 16 * qt);
+          uint32_t packed[16];
 #pragma unroll
-            for (int q4 = 0; q4 < 2; ++q4) {
-              const int b8 = 8 * q4;
-              dst[q4] = make_uint4(pack_bf16x2(fmaf(egr, o1[b8], o2[b8]), fmaf(egr, o1[b8 + 1], o2[b8 + 1])),
-                                   pack_bf16x2(fmaf(egr, o1[b8 + 2], o2[b8 + 2]), fmaf(egr, o1[b8 + 3], o2[b8 + 3])),
-                                   pack_bf16x2(fmaf(egr, o1[b8 + 4], o2[b8 + 4]), fmaf(egr, o1[b8 + 5], o2[b8 + 5])),
-                                   pack_bf16x2(fmaf(egr, o1[b8 + 6], o2[b8 + 6]), fmaf(egr, o1[b8 + 7], o2[b8 + 7])));
-            }
+          for (int i = 0; i < 16; ++i)
+            packed[i] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(egv[i], o1[i], o2[i])));
+          __syncwarp();  // the previous piece's reads of the buffer are done
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            st_shared_u16(ostg + uint32_t(i) * 64 + uint32_t(lane) * 2, uint16_t(packed[i]));
+          __syncwarp();
+#pragma unroll
+          for (int m = 0; m < 2; ++m) {
+            const int id = lane + 32 * m, i = id >> 2, seg = id & 3;
+            const int r = r0 + i;
+            const uint4 val = ld_shared_v4(ostg + uint32_t(i) * 64 + uint32_t(seg) * 16);
+            if (okE && r < Ll && e0 < D && p.o != nullptr)
+              *reinterpret_cast<uint4*>(p.o + (size_t(t0l + r) * p.H_v + hl) * D + e0 + seg * 8) = val;
           }
         }
         return okE;
@@ -607,11 +629,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = s; u < units; u += p.S) {
         const int n = u / p.H_v, h = u % p.H_v;
         int tb, te;
-        seq_range(p, n, tb, te);
+        seq_range<kSeg>(p, n, tb, te);
         const size_t seq_off = size_t(n) * p.H_v * size_t(D) * D, head_off = size_t(h) * D * D;
-        const float* h0b = p.h0_tab != nullptr ? p.h0_tab[n]
+        const float* h0b = (kSeg && p.h0_tab != nullptr) ? p.h0_tab[n]
                                                : (p.h0 != nullptr ? p.h0 + seq_off : nullptr);
-        float* hTb = p.hT_tab != nullptr ? p.hT_tab[n] : (p.hT != nullptr ? p.hT + seq_off : nullptr);
+        float* hTb = (kSeg && p.hT_tab != nullptr) ? p.hT_tab[n] : (p.hT != nullptr ? p.hT + seq_off : nullptr);
         bool agreed = true;
         float H[64];
         {
@@ -619,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 64; ++i)
             H[i] = (h0 != nullptr && 64 * hh + i < D) ? h0[size_t(64 * hh + i) * D] : 0.f;
-          if (p.h0_identity) {
+          if (kSeg && p.h0_identity) {
 #pragma unroll
             for (int i = 0; i < 64; ++i) H[i] = (64 * hh + i == j) ? 1.f : 0.f;
           }
@@ -649,28 +671,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           // part A is released after the [W; Q] MMA: keep the gate factors
           if (tid < 64) eg_s[64 * st + tid] = sg[tid] * p.scale;
           else if (tid < 128) ecg_s[64 * st + tid - 64] = sg[tid];
-          if constexpr (kLimbs == 1) {
-            // chunk c-1's O1 MMA (issued after dH) reads the bf16 copy of H
-            if (c > c_first)
-              ok = mbar_wait(&bars[SB_O1DONE], (c - 1) & 1, abort_flag, err, 16u, p.spin_limit) && ok;
-          }
           st_row64_bf16(sbase + S_HT + uint32_t(hh) * 16384, uint32_t(j), H);
           if constexpr (kLimbs == 2) {
-            // The low limb goes into the Vn buffers, which the previous
-            // chunk's O2 MMA reads (and O1 of this chunk will, before this
-            // chunk's Vn lands there): chunk c-1's outputs are taken first.
-            if (c > c_first) ok = epilogue(c - 1, prev_t0, prev_L, h) && ok;
+            // the previous chunk's O2 MMA reads the Vn buffers: done first
+            if (c > c_first)
+              ok = mbar_wait(&bars[SB_OFULL + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag, err,
+                             16u, p.spin_limit) && ok;
             st_row64_bf16_lo(sbase + S_VN + uint32_t(hh) * 16384, uint32_t(j), H);
           }
           fence_proxy_async_smem();
           tc_fence_before();
-          if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts Vn' (and O1)
+          if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts [W; Q]
             agreed = false;
             break;
           }
-          if constexpr (kLimbs == 1) {
-            if (c > c_first) ok = epilogue(c - 1, prev_t0, prev_L, h) && ok;
-          }
+          bool okE = true;
+          if (c > c_first) okE = epilogue(c - 1, 0, prev_t0, prev_L, h);
+          ok = ok && okE;
           // Vn = U - Vn'  ->  Vn^T and e^{G_C - G_r} Vn^T rows in bf16
           ok = mbar_wait(&bars[SB_VOFULL], c & 1, abort_flag, err, 16u, p.spin_limit) && ok;
           ok = mbar_wait(&bars[SB_BF + st], (c >> 1) & 1, abort_flag, err, 16u, p.spin_limit) && ok;
@@ -679,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint8_t* urow = smem + S_STG + st * STG_BYTES + STG_U;
             const float* ecp = ecg_s + 64 * st;
             float vn[32];
-            tmem_ld32(tmem + lane_off + ST_V + 32u * uint32_t(hh), vn);
+            tmem_ld32(tmem + lane_off + ST_VO + 128u * st + 32u * uint32_t(hh), vn);
             tmem_ld_wait();
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
@@ -718,11 +735,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
           tc_fence_before();
-          tc_fence_before();  // this chunk's TMEM reads (Vn', outputs) before O1 / O2
-          if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts dH, O1, O2
+          if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts dH, O2
             agreed = false;
             break;
           }
+          if (c > c_first) ok = epilogue(c - 1, 1, prev_t0, prev_L, h) && okE && ok;
           dec_prev = dec_cur;
           prev_t0 = t0;
           prev_L = min(C, te - t0);
@@ -742,8 +759,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) H[32 * q2 + i] = fmaf(dec_prev, H[32 * q2 + i], d[i]);
           }
-          ok = epilogue(c - 1, prev_t0, prev_L, h) && ok;
-          tc_fence_before();
+          ok = epilogue(c - 1, 0, prev_t0, prev_L, h) && ok;
+          ok = epilogue(c - 1, 1, prev_t0, prev_L, h) && ok;
           if (!named_all(1, kSpineSync, ok)) {  // the issuer warp takes part
             ok = false;
             break;
@@ -760,33 +777,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 9) {
       // ---------------- issuer: joins the state warps' two barriers per chunk
       // (bar.red: every participant gets the same outcome) and issues
-      //   after the first:  Vn'^T = H^T W^T   (N = 64; two limbs: then O1)
-      //   after the second: dH^T = Vns^T K (fresh), then O1 = Q H and
-      //                     O2 = Aqk Vn (M = 64, N = d_v)
-      // Part A of the stage (W, Q) is free once O1 is done, part B (K, U^T,
-      // Aqk) once dH and O2 are.
-      const uint32_t id_v = make_idesc_bf16(128, 64, 0, 0);
+      //   after the first:  [Vn' | O1]^T = H^T [W; Q]^T              (N = 128)
+      //   after the second: dH^T = Vns^T K (fresh), O2^T = Vn^T Aqk^T
+      const uint32_t id_vo = make_idesc_bf16(128, 128, 0, 0);
       const uint32_t id_dh = make_idesc_bf16(128, 128, 0, 1);
-      const uint32_t id_o = make_idesc_bf16(64, 128, 0, 0);
+      const uint32_t id_o2 = make_idesc_bf16(128, 64, 0, 0);
       const bool leader = lane == 0;
-      auto issue_o1 = [&](uint32_t stg) {
-        for (int kk = 0; kk < ksteps_d; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(tmem + ST_O1, make_sdesc_sw128(stg + STG_WQ + 8192 + off, 16, 1024),
-                      make_sdesc_sw128(sbase + S_HT + off, 16, 1024), id_o, kk > 0);
-        }
-        if constexpr (kLimbs == 2) {
-          for (int kk = 0; kk < ksteps_d; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16_ss(tmem + ST_O1, make_sdesc_sw128(stg + STG_WQ + 8192 + off, 16, 1024),
-                        make_sdesc_sw128(sbase + S_VN + off, 16, 1024), id_o, 1u);
-          }
-        }
-      };
       int c = 0;
       for (int u = s; u < units; u += p.S) {
         int tb, te;
-        seq_range(p, u / p.H_v, tb, te);
+        seq_range<kSeg>(p, u / p.H_v, tb, te);
         bool agreed = true;
         for (int t0 = tb; t0 < te; t0 += C, ++c) {
           const int st = c & 1;
@@ -799,19 +799,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             for (int kk = 0; kk < ksteps_d; ++kk) {
               const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_bf16_ss(tmem + ST_V, make_sdesc_sw128(sbase + S_HT + off, 16, 1024),
-                          make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_v, kk > 0);
+              mma_bf16_ss(tmem + ST_VO + 128u * st, make_sdesc_sw128(sbase + S_HT + off, 16, 1024),
+                          make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_vo, kk > 0);
             }
             if constexpr (kLimbs == 2) {
               for (int kk = 0; kk < ksteps_d; ++kk) {
                 const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16_ss(tmem + ST_V, make_sdesc_sw128(sbase + S_VN + off, 16, 1024),
-                            make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_v, 1u);
+                mma_bf16_ss(tmem + ST_VO + 128u * st, make_sdesc_sw128(sbase + S_VN + off, 16, 1024),
+                            make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_vo, 1u);
               }
-              issue_o1(stg);  // reads the low limb before this chunk's Vn lands on it
-              mma_commit(&bars[SB_AE + st]);
             }
             mma_commit(&bars[SB_VOFULL]);
+            mma_commit(&bars[SB_AE + st]);
           }
           __syncwarp();
           if (!named_all(1, kSpineSync, true)) {
@@ -824,15 +823,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_bf16_ss(tmem + ST_DH, make_sdesc_sw128(sbase + S_VNS + kk * 32, 16, 1024),
                           make_sdesc_sw128(stg + STG_K + kk * 2048, 8192, 1024), id_dh, kk > 0);
             mma_commit(&bars[SB_DHFULL]);
-            if constexpr (kLimbs == 1) {
-              issue_o1(stg);
-              mma_commit(&bars[SB_O1DONE]);
-              mma_commit(&bars[SB_AE + st]);
-            }
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(tmem + ST_O2, make_sdesc_sw128(stg + STG_AQK + kk * 32, 16, 1024),
-                          make_sdesc_sw128(sbase + S_VN + kk * 32, 16, 1024), id_o, kk > 0);
-            mma_commit(&bars[SB_OFULL]);
+              mma_bf16_ss(tmem + ST_O2 + 64u * st,
+                          make_sdesc_sw128(sbase + S_VN + kk * 32, 16, 1024),
+                          make_sdesc_sw128(stg + STG_AQK + kk * 32, 16, 1024), id_o2, kk > 0);
+            mma_commit(&bars[SB_OFULL + st]);
             mma_commit(&bars[SB_BE + st]);
           }
           __syncwarp();
@@ -853,7 +848,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // to the preps.
       if (lane == 0) {
         ChunkIter fd;
-        it_start(fd, p, s);
+        it_start<kSeg>(fd, p, s);
         int issued_a = 0, issued_b = 0;
         bool ok = true;
         while (fd.ok && ok) {
@@ -897,7 +892,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_load_g2s(stg + STG_U, src + G_U, 16384, fb);
           bulk_load_g2s(stg + STG_AQK, src + G_AQK, 8192, fb);
           issued_b = cc + 1;
-          it_next(fd, p);
+          it_next<kSeg>(fd, p);
         }
         if (!ok) {
           *abort_flag = 1;
@@ -920,10 +915,148 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int prank = int(blockIdx.x) - p.S;
     if (warp == 8) {
       // ---------------- loader: item k's K, Q, V tiles (TMA, lane 0) once set
-      // k % 3 is free (item k - 3 stored), and its gate factors (whole warp)
+      // k % 3 is free (item k - 3 stored)
       PrepIter it;
-      pi_start(it, p, sJ, iend, prank);
+      pi_start<kSeg>(it, p, sJ, iend, prank);
       int last_k = -1;
+      bool ok = true;
+      while (it.ok && ok) {
+        const int k = it.k, t = k % 3;
+        ok = k < 3 || mbar_wait(&bars[PB_STORED + t], ((k / 3) & 1) ^ 1, abort_flag, err, 1u, p.spin_limit);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          uint64_t* fb = &bars[PB_KQVF + t];
+          mbar_arrive_expect_tx(fb, uint32_t(nbox) * ((kSeg && p.v_zero) ? 2 : 3) * 8192);
+          uint8_t* set = smem + t * P_SET;
+          const int hk = it.h / vpg;
+          for (int b2 = 0; b2 < nbox; ++b2) {
+            tma_load_3d(set + P_KQ + b2 * 16384, &tm_k, fb, b2 * 64, hk, it.t0);
+            tma_load_3d(set + P_KQ + b2 * 16384 + 8192, &tm_q, fb, b2 * 64, hk, it.t0);
+            // v read as zeros: the V boxes keep the zeros of the start-up clear
+            if (!(kSeg && p.v_zero)) tma_load_3d(set + P_V + b2 * 8192, &tm_v, fb, b2 * 64, it.h, it.t0);
+          }
+          last_k = k;
+        }
+        pi_next<kSeg>(it, p, sJ, iend);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicExch(const_cast<uint32_t*>(gabort), 1u);
+      }
+      if (lane == 0)  // nothing may still be landing in shared memory at exit
+        for (int k = last_k - 2; k <= last_k; ++k)
+          if (k >= 0) mbar_wait(&bars[PB_KQVF + k % 3], (k / 3) & 1, nullptr, err, 32u);
+      __syncwarp();
+    } else if (warp == 9) {
+      // ---------------- MMA issue for both groups, whichever is ready: P1 of
+      // items in order (tiles landed, the group's P1 buffer read back), W/U of
+      // each group's next item once its T is ready
+      if (elect_one()) {
+        const uint32_t id_p1 = make_idesc_bf16(128, 64, 0, 0);
+        const uint32_t id_wu = make_idesc_bf16(128, 64, 1, 0);
+        PrepIter itp;
+        pi_start<kSeg>(itp, p, sJ, iend, prank);
+        int kp = 0;                // next item for P1
+        int kw[2] = {0, 0};        // next in-group index for W/U
+        long long last = clock64();
+        while (true) {
+          bool prog = false;
+          if (itp.ok) {
+            const int t = kp % 3, g = kp & 1, kg = kp >> 1, pb = kg & 1;
+            if (mbar_test_wait(&bars[PB_KQVF + t], (kp / 3) & 1) &&
+                (kg < 2 || mbar_test_wait(&bars[PB_P1FREE + 2 * g + pb], ((kg >> 1) & 1) ^ 1))) {
+              tc_fence_after();
+              const uint32_t set = sbase + t * P_SET;
+              const uint32_t tm = tmem + PT_WG * g + 64u * pb;
+              for (int kk = 0; kk < ksteps_d; ++kk) {
+                const uint32_t a = set + P_KQ + (kk >> 2) * 16384 + (kk & 3) * 32;
+                mma_bf16_ss(tm, make_sdesc_sw128(a, 16, 1024), make_sdesc_sw128(a, 16, 1024), id_p1,
+                            kk > 0);
+              }
+              mma_commit(&bars[PB_P1F + 2 * g + pb]);
+              ++kp;
+              pi_next<kSeg>(itp, p, sJ, iend);
+              prog = true;
+            }
+          }
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            const int kwg = kw[g], k = 2 * kwg + g;
+            if (k < kp && mbar_test_wait(&bars[PB_TREADY + g], kwg & 1)) {
+              tc_fence_after();
+              const uint32_t set = sbase + (k % 3) * P_SET;
+              const uint32_t tm = tmem + PT_WG * g;
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tm + PT_W, make_sdesc_sw128(set + P_KQ + kk * 2048, 16384, 1024),
+                            make_sdesc_sw128(set + P_T1B + kk * 32, 16, 1024), id_wu, kk > 0);
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tm + PT_U, make_sdesc_sw128(set + P_V + kk * 2048, 8192, 1024),
+                            make_sdesc_sw128(set + P_T2B + kk * 32, 16, 1024), id_wu, kk > 0);
+              mma_commit(&bars[PB_WUF + g]);
+              ++kw[g];
+              prog = true;
+            }
+          }
+          if ((!itp.ok && 2 * kw[0] >= kp && 2 * kw[1] + 1 >= kp) || *abort_flag) break;
+          if (prog) {
+            last = clock64();
+          } else {
+            if (clock64() - last > p.spin_limit) {
+              *abort_flag = 1;
+              atomicExch(const_cast<uint32_t*>(gabort), 1u);
+              atomicOr(err, 2u);
+              break;
+            }
+            __nanosleep(32);
+          }
+        }
+        mma_commit(&bars[PB_DRAIN]);
+        mbar_wait(&bars[PB_DRAIN], 0, nullptr, err, 8u);
+      }
+      __syncwarp();
+    } else if (warp == 10) {
+      // ---------------- store: each staged item to its spine's ring entry, in
+      // item order
+      if (lane == 0) {
+        PrepIter it;
+        pi_start<kSeg>(it, p, sJ, iend, prank);
+        bool ok = true;
+        while (it.ok && ok) {
+          const int k = it.k, t = k % 3, g = k & 1, kg = k >> 1;
+          const int e = it.j % kRing;
+          ok = mbar_wait(&bars[PB_STAGED + g], kg & 1, abort_flag, err, 4u, p.spin_limit);
+          if (ok && it.j >= kRing)  // entry e is free once the spine copied item j - kRing
+            ok = poll_geq(free_flag(p, it.s, e), uint32_t(it.j - kRing + 1), gabort, err, 4u, p.spin_limit);
+          if (!ok) break;
+          fence_proxy_async_global();
+          uint8_t* dst = ring_entry(p, it.s, e);
+          const uint8_t* ga = smem + P_GRP + g * P_GS;
+          bulk_store_s2g(dst + G_W, smem + t * P_SET, 32768);
+          bulk_store_s2g(dst + G_AQK, ga + GA_AQK, 8192);
+          bulk_store_s2g(dst + G_GATE, ga + GA_GT + (kg & 1) * PG_BYTES + PG_EG * 4, G_GATE_BYTES);
+          tma_store_commit();
+          tma_store_wait_read<0>();
+          mbar_arrive(&bars[PB_STORED + t]);
+          tma_store_wait_all<0>();
+          fence_proxy_async_global();
+          st_release_gpu(ready_flag(p, it.s, e), uint32_t(it.j + 1));
+          pi_next<kSeg>(it, p, sJ, iend);
+        }
+        if (!ok) {
+          *abort_flag = 1;
+          atomicExch(const_cast<uint32_t*>(gabort), 1u);
+        }
+      }
+      __syncwarp();
+    } else if (warp == 11) {
+      // ---------------- gate factors of item k (whole warp), into gate block
+      // kg & 1 of group k & 1 once item k - 3 is stored (so the block's last
+      // reader, the store of item k - 4, is done), beside the loader
+      PrepIter it;
+      pi_start<kSeg>(it, p, sJ, iend, prank);
       bool ok = true;
       while (it.ok && ok) {
         const int k = it.k, t = k % 3, g = k & 1, gb = (k >> 1) & 1;
@@ -932,21 +1065,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        if (lane == 0) {
-          uint64_t* fb = &bars[PB_KQVF + t];
-          mbar_arrive_expect_tx(fb, uint32_t(nbox) * (p.v_zero ? 2 : 3) * 8192);
-          uint8_t* set = smem + t * P_SET;
-          const int hk = it.h / vpg;
-          for (int b2 = 0; b2 < nbox; ++b2) {
-            tma_load_3d(set + P_KQ + b2 * 16384, &tm_k, fb, b2 * 64, hk, it.t0);
-            tma_load_3d(set + P_KQ + b2 * 16384 + 8192, &tm_q, fb, b2 * 64, hk, it.t0);
-            // v read as zeros: the V boxes keep the zeros of the start-up clear
-            if (!p.v_zero) tma_load_3d(set + P_V + b2 * 8192, &tm_v, fb, b2 * 64, it.h, it.t0);
-          }
-          last_k = k;
-        }
-        // Gates of this item (padded rows: g = beta = 0); lane l owns rows 2l,
-        // 2l+1.  The block was last read by the store of item k - 4.
+        // padded rows: g = beta = 0; lane l owns rows 2l, 2l + 1
         float* gt = reinterpret_cast<float*>(smem + P_GRP + g * P_GS + GA_GT + gb * PG_BYTES);
         {
           const int r0 = 2 * lane;
@@ -1009,115 +1128,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         mbar_arrive(&bars[PB_GATEF + 2 * g + gb]);  // release: this lane's gate writes
-        pi_next(it, p, sJ, iend);
+        pi_next<kSeg>(it, p, sJ, iend);
       }
       if (!ok) {
         *abort_flag = 1;
         atomicExch(const_cast<uint32_t*>(gabort), 1u);
-      }
-      if (lane == 0)  // nothing may still be landing in shared memory at exit
-        for (int k = last_k - 2; k <= last_k; ++k)
-          if (k >= 0) mbar_wait(&bars[PB_KQVF + k % 3], (k / 3) & 1, nullptr, err, 32u);
-      __syncwarp();
-    } else if (warp == 9) {
-      // ---------------- MMA issue for both groups, whichever is ready: P1 of
-      // items in order (tiles landed, the group's P1 buffer read back), W/U of
-      // each group's next item once its T is ready
-      if (elect_one()) {
-        const uint32_t id_p1 = make_idesc_bf16(128, 64, 0, 0);
-        const uint32_t id_wu = make_idesc_bf16(128, 64, 1, 0);
-        PrepIter itp;
-        pi_start(itp, p, sJ, iend, prank);
-        int kp = 0;                // next item for P1
-        int kw[2] = {0, 0};        // next in-group index for W/U
-        long long last = clock64();
-        while (true) {
-          bool prog = false;
-          if (itp.ok) {
-            const int t = kp % 3, g = kp & 1, kg = kp >> 1, pb = kg & 1;
-            if (mbar_test_wait(&bars[PB_KQVF + t], (kp / 3) & 1) &&
-                (kg < 2 || mbar_test_wait(&bars[PB_P1FREE + 2 * g + pb], ((kg >> 1) & 1) ^ 1))) {
-              tc_fence_after();
-              const uint32_t set = sbase + t * P_SET;
-              const uint32_t tm = tmem + PT_WG * g + 64u * pb;
-              for (int kk = 0; kk < ksteps_d; ++kk) {
-                const uint32_t a = set + P_KQ + (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16_ss(tm, make_sdesc_sw128(a, 16, 1024), make_sdesc_sw128(a, 16, 1024), id_p1,
-                            kk > 0);
-              }
-              mma_commit(&bars[PB_P1F + 2 * g + pb]);
-              ++kp;
-              pi_next(itp, p, sJ, iend);
-              prog = true;
-            }
-          }
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            const int kwg = kw[g], k = 2 * kwg + g;
-            if (k < kp && mbar_test_wait(&bars[PB_TREADY + g], kwg & 1)) {
-              tc_fence_after();
-              const uint32_t set = sbase + (k % 3) * P_SET;
-              const uint32_t tm = tmem + PT_WG * g;
-              for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tm + PT_W, make_sdesc_sw128(set + P_KQ + kk * 2048, 16384, 1024),
-                            make_sdesc_sw128(set + P_T1B + kk * 32, 16, 1024), id_wu, kk > 0);
-              for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tm + PT_U, make_sdesc_sw128(set + P_V + kk * 2048, 8192, 1024),
-                            make_sdesc_sw128(set + P_T2B + kk * 32, 16, 1024), id_wu, kk > 0);
-              mma_commit(&bars[PB_WUF + g]);
-              ++kw[g];
-              prog = true;
-            }
-          }
-          if ((!itp.ok && 2 * kw[0] >= kp && 2 * kw[1] + 1 >= kp) || *abort_flag) break;
-          if (prog) {
-            last = clock64();
-          } else {
-            if (clock64() - last > p.spin_limit) {
-              *abort_flag = 1;
-              atomicExch(const_cast<uint32_t*>(gabort), 1u);
-              atomicOr(err, 2u);
-              break;
-            }
-            __nanosleep(32);
-          }
-        }
-        mma_commit(&bars[PB_DRAIN]);
-        mbar_wait(&bars[PB_DRAIN], 0, nullptr, err, 8u);
-      }
-      __syncwarp();
-    } else if (warp == 10) {
-      // ---------------- store: each staged item to its spine's ring entry, in
-      // item order
-      if (lane == 0) {
-        PrepIter it;
-        pi_start(it, p, sJ, iend, prank);
-        bool ok = true;
-        while (it.ok && ok) {
-          const int k = it.k, t = k % 3, g = k & 1, kg = k >> 1;
-          const int e = it.j % kRing;
-          ok = mbar_wait(&bars[PB_STAGED + g], kg & 1, abort_flag, err, 4u, p.spin_limit);
-          if (ok && it.j >= kRing)  // entry e is free once the spine copied item j - kRing
-            ok = poll_geq(free_flag(p, it.s, e), uint32_t(it.j - kRing + 1), gabort, err, 4u, p.spin_limit);
-          if (!ok) break;
-          fence_proxy_async_global();
-          uint8_t* dst = ring_entry(p, it.s, e);
-          const uint8_t* ga = smem + P_GRP + g * P_GS;
-          bulk_store_s2g(dst + G_W, smem + t * P_SET, 32768);
-          bulk_store_s2g(dst + G_AQK, ga + GA_AQK, 8192);
-          bulk_store_s2g(dst + G_GATE, ga + GA_GT + (kg & 1) * PG_BYTES + PG_EG * 4, G_GATE_BYTES);
-          tma_store_commit();
-          tma_store_wait_read<0>();
-          mbar_arrive(&bars[PB_STORED + t]);
-          tma_store_wait_all<0>();
-          fence_proxy_async_global();
-          st_release_gpu(ready_flag(p, it.s, e), uint32_t(it.j + 1));
-          pi_next(it, p, sJ, iend);
-        }
-        if (!ok) {
-          *abort_flag = 1;
-          atomicExch(const_cast<uint32_t*>(gabort), 1u);
-        }
       }
       __syncwarp();
     } else if (warp < 8) {
@@ -1130,8 +1145,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* Xs = reinterpret_cast<float*>(ga + GA_XS);
       const int gbar = 1 + 3 * g;  // this group's named barriers: gbar (all), gbar+1, gbar+2
       PrepIter it;
-      pi_start(it, p, sJ, iend, prank);
-      pi_align(it, p, sJ, iend, g);
+      pi_start<kSeg>(it, p, sJ, iend, prank);
+      pi_align<kSeg>(it, p, sJ, iend, g);
       while (it.ok) {
         const int k = it.k, kg = k >> 1, t = k % 3, pb = kg & 1;
         uint8_t* set = smem + t * P_SET;
@@ -1266,8 +1281,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         named_sync(gbar, 128);
         if (pt == 0) mbar_arrive(&bars[PB_STAGED + g]);
-        pi_next(it, p, sJ, iend);
-        pi_align(it, p, sJ, iend, g);
+        pi_next<kSeg>(it, p, sJ, iend);
+        pi_align<kSeg>(it, p, sJ, iend, g);
       }
     }
   }
@@ -1293,9 +1308,9 @@ int resident_ctas() {
   int* slot = (dev >= 0 && dev < 64) ? &cache[dev] : nullptr;
   if (slot != nullptr && *slot > 0) return *slot;
   int per_sm = 0;
-  cudaFuncSetAttribute(prefill_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaFuncSetAttribute(prefill_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        int(kSmemAlloc));
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prefill_kernel<1>, kThreads,
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prefill_kernel<1, false>, kThreads,
                                                     kSmemAlloc) != cudaSuccess) {
     cudaGetLastError();
     per_sm = 0;
@@ -1356,7 +1371,12 @@ cudaError_t launch_prefill_call(const PrefillCall& c, cudaStream_t s) {
     uint32_t box[3] = {64, 1, 64};
     if (!encode_tmap_bf16(&tv, c.v, 3, dims, strides, box, true)) return cudaErrorInvalidValue;
   }
-  auto kernel = c.limbs == 2 ? prefill_kernel<2> : prefill_kernel<1>;
+  // The plain form (whole sequences, h0 / hT arrays, real v) carries none of
+  // the segment-pass branches.
+  const bool seg = c.seg != nullptr || c.h0_tab != nullptr || c.hT_tab != nullptr || c.v_zero ||
+                   c.h0_identity;
+  auto kernel = c.limbs == 2 ? (seg ? prefill_kernel<2, true> : prefill_kernel<2, false>)
+                             : (seg ? prefill_kernel<1, true> : prefill_kernel<1, false>);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(kSmemAlloc));
   if (e != cudaSuccess) return e;
