@@ -8,11 +8,13 @@
 //
 //   D[128 tokens x N] = X[128 x K] * W[N x K]^T
 //
-// One cluster of KS CTAs per 128 tokens, each CTA over its own K / KS slice
-// (split-K, so that the 4576 x 5120 activation streams through ~all SMs).
-// TMA streams 128x64 X tiles and Nx64 W tiles (128-byte swizzle) through a
-// STAGES-deep mbarrier ring; one thread issues tcgen05.mma (M=128, N=N_pad,
-// K=16 steps) into a TMEM accumulator.  Rank r owns rows r*128/KS .. of the
+// One cluster of KS CTAs per BM tokens, each CTA over its own K / KS slice
+// (split-K, so that the activation streams through ~all SMs): BM = 64 while
+// the 64-row tiles in pairs fit the SMs in one wave (4576 tokens: 72 tiles x
+// KS 2 = 144 CTAs), else 128; few tiles split K up to 8 ways.
+// TMA streams BMx64 X tiles and Nx64 W tiles (128-byte swizzle) through a
+// STAGES-deep mbarrier ring; one thread issues tcgen05.mma (M=BM, N=N_pad,
+// K=16 steps) into a TMEM accumulator.  Rank r owns rows r*BM/KS .. of the
 // tile: every CTA pushes each of its partial rows into the owner's receive
 // buffer with distributed-shared-memory stores (no dependent remote loads),
 // one cluster barrier publishes them, and the owner sums the KS partials of
@@ -32,10 +34,10 @@ namespace gdn {
 
 __device__ uint32_t g_err_ba_gates;
 
-constexpr int kBaBM = 128;       // tokens per CTA (MMA M)
+// tokens per CTA (MMA M): 64 while 64-row tiles in pairs fill the SMs, else 128
 constexpr int kBaBK = 64;        // K per TMA box (one 128-byte swizzle row)
 constexpr int kBaNB = 2;         // boxes per pipeline stage: 2 x 128 contiguous bytes per row
-constexpr int kBaMaxKS = 2;      // largest K split (CTAs per cluster): measured best
+constexpr int kBaMaxKS = 8;      // largest K split (CTAs per cluster, the portable limit)
 constexpr int kBaThreads = 512;  // TMA (warp 0), MMA (warp 1); all 16 warps: epilogue
 
 struct BaParams {
@@ -71,6 +73,7 @@ __device__ __forceinline__ float log1p_unit(float t) {
   return __logf(1.0f + t);
 }
 
+template <int BM>
 __global__ void __launch_bounds__(kBaThreads, 1)
     ba_gates_kernel(const __grid_constant__ CUtensorMap tmap_x,
                     const __grid_constant__ CUtensorMap tmap_w, const BaParams p) {
@@ -79,7 +82,7 @@ __global__ void __launch_bounds__(kBaThreads, 1)
   // that accesses through it stay shared-space (not generic) loads and stores
   uint8_t* smem = smem_raw + ((uint32_t(1024) - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int stages = p.stages;
-  const uint32_t a_box = kBaBM * 128, b_box = uint32_t(p.n_pad) * 128;
+  const uint32_t a_box = BM * 128, b_box = uint32_t(p.n_pad) * 128;
   const uint32_t a_bytes = kBaNB * a_box;
   const uint32_t b_bytes = kBaNB * b_box;
   uint8_t* a_s = smem;
@@ -98,7 +101,7 @@ __global__ void __launch_bounds__(kBaThreads, 1)
   const uint32_t warp = warp_id_sync();
   const uint32_t lane = threadIdx.x & 31;
   const int rank = int(cluster_ctarank());
-  const int m0 = int(cluster_id_x()) * kBaBM;
+  const int m0 = int(cluster_id_x()) * BM;
   // K is split into boxes of kBaBK; this CTA owns boxes [kb_begin, kb_end),
   // consumed kBaNB boxes per pipeline stage (the last stage may be partial).
   const int kb_all = (p.K + kBaBK - 1) / kBaBK;
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(kBaThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (elect_one()) {  // MMA issuer
-      const uint32_t idesc = make_idesc_bf16(kBaBM, p.n_pad, 0, 0);
+      const uint32_t idesc = make_idesc_bf16(BM, p.n_pad, 0, 0);
       bool ok = true;
       for (int kb = 0; kb < num_kb && ok; ++kb) {
         const int s = kb % stages;
@@ -185,10 +188,10 @@ __global__ void __launch_bounds__(kBaThreads, 1)
     __syncwarp();
   }
 
-  // Partial sums: warp w reads TMEM lanes 32 (w % 4) .. + 31 (tile row r =
-  // 32 (w % 4) + lane), column blocks of 16 from 16 (w / 4) in steps of 64.
-  // Row r belongs to rank r / (128 / KS); this CTA's copy of it goes to slot
-  // [my rank][r % (128 / KS)] of that rank's receive buffer.  When the buffer
+  // Partial sums: warp w reads TMEM lane quadrant w % 4 (tile rows
+  // BM/4 (w % 4) ..), column blocks of 16 from 16 (w / 4) in steps of 64.
+  // Row r belongs to rank r / (BM / KS); this CTA's copy of it goes to slot
+  // [my rank][r % (BM / KS)] of that rank's receive buffer.  When the buffer
   // reuses pipeline memory, every CTA of the cluster must be done with its
   // pipeline first (the barrier below is then a full one).
   const bool ok = num_kb == 0 || mbar_wait(done_bar, 0, abort_flag, &g_err_ba_gates, 4u);
@@ -196,10 +199,14 @@ __global__ void __launch_bounds__(kBaThreads, 1)
   if (p.overlay) cluster_arrive_release();
   cluster_wait_acquire();  // every CTA of the cluster is running (and idle, overlaid)
   const int pstride = p.n_pad + 4;
-  const int rows = kBaBM / p.ks;
+  const int rows = BM / p.ks;
+  // (M = 128: tile row r in TMEM lane r; M = 64: row r in lane r % 16 +
+  // 32 (r / 16), so lanes 16..31 of each quadrant hold nothing: they take
+  // part in the warp-wide TMEM loads and store nothing)
   {
     const uint32_t lq = warp & 3u;
-    const int r = int(lq) * 32 + int(lane);
+    const bool holds = BM == 128 || lane < 16;
+    const int r = int(lq) * (BM / 4) + (holds ? int(lane) : 0);
     const int owner = r / rows;
     const uint32_t dst = mapa_shared(
         smem_u32(recv + size_t(rank * rows + (r - owner * rows)) * pstride), uint32_t(owner));
@@ -208,12 +215,14 @@ __global__ void __launch_bounds__(kBaThreads, 1)
       float acc[16];
       tmem_ld16(tmem + ((lq * 32u) << 16) + uint32_t(c), acc);
       tmem_ld_wait();
+      if (holds) {
 #pragma unroll
-      for (int j = 0; j < 16; j += 4)
-        st_cluster_v4(dst + uint32_t(c + j) * 4, live ? __float_as_uint(acc[j]) : 0u,
-                      live ? __float_as_uint(acc[j + 1]) : 0u,
-                      live ? __float_as_uint(acc[j + 2]) : 0u,
-                      live ? __float_as_uint(acc[j + 3]) : 0u);
+        for (int j = 0; j < 16; j += 4)
+          st_cluster_v4(dst + uint32_t(c + j) * 4, live ? __float_as_uint(acc[j]) : 0u,
+                        live ? __float_as_uint(acc[j + 1]) : 0u,
+                        live ? __float_as_uint(acc[j + 2]) : 0u,
+                        live ? __float_as_uint(acc[j + 3]) : 0u);
+      }
     }
   }
   tc_fence_before();
@@ -264,9 +273,10 @@ __global__ void __launch_bounds__(kBaThreads, 1)
 //
 // Page "ssm_ba_gates_hopper.rs", module doc: one CTA per token starves the
 // device when the step has few tokens (16 rows put 16 CTAs on the machine),
-// hence its token-count guard.  With M <= kBaSmallM the 128-row tensor-core
-// tile above would leave the GPU just as empty, so these shapes split the
-// OUTPUTS and the REDUCTION across CTAs instead of the tokens:
+// hence its token-count guard.  Down to 9 tokens the tensor-core kernel above
+// still fills enough SMs (one 64-row tile split 8 ways along K); at M <=
+// kBaSmallM (measured: 8 tokens, 9 us, against 13 us there) these shapes
+// split the OUTPUTS and the REDUCTION across CTAs instead of the tokens:
 //   grid = NG output groups of kBaSmallNPB outputs x KS K slices, as clusters
 //   of KS CTAs along K (one cluster per output group);
 //   warp w of a CTA computes output n0 + w for every token of the chunk: each
@@ -281,8 +291,8 @@ __global__ void __launch_bounds__(kBaThreads, 1)
 // cores, f32 accumulation: at these sizes the weight read and the launch, not
 // the arithmetic, set the time.
 // ---------------------------------------------------------------------------
-constexpr int kBaSmallM = 64;     // largest M sent to the few-token kernel
-constexpr int kBaSmallMB = 64;    // tokens per CTA row
+constexpr int kBaSmallM = 8;      // largest M sent to the few-token kernel (measured crossover)
+constexpr int kBaSmallMB = 8;     // tokens per CTA row
 constexpr int kBaSmallNPB = 8;    // outputs per CTA (one per warp)
 constexpr int kBaSmallKS = 8;     // CTAs per cluster along K (portable cluster size)
 
@@ -427,10 +437,7 @@ static cudaError_t launch_ba_gates_small(const uint16_t* x, int k_stride, const 
     case 1: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<1>, p); break;
     case 2: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<2>, p); break;
     case 4: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<4>, p); break;
-    case 8: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<8>, p); break;
-    case 16: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<16>, p); break;
-    case 32: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<32>, p); break;
-    default: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<64>, p); break;
+    default: e = cudaLaunchKernelEx(&cfg, ba_gates_small_kernel<8>, p); break;
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -462,11 +469,16 @@ cudaError_t launch_ba_gates(const uint16_t* x, int k_stride, const uint16_t* w,
   p.vpg = vpg;
   p.n_pad = (N + 15) / 16 * 16;
   p.tmem_cols = pow2_at_least(p.n_pad);
-  // Layout: [stages][receive buffer, f32 [128][n_pad + 4]][constants][barriers].
+  // Tile height: 64-row tiles in clusters of two while they fit the SMs in
+  // one wave (4576 tokens: 72 tiles x 2 = 144 CTAs, each streaming 1/144 of
+  // the activations), 128-row tiles beyond.
+  const int kb_all = (K + kBaBK - 1) / kBaBK;
+  const int BM = ((M + 63) / 64) * 2 <= sm_count() && kb_all >= 2 ? 64 : 128;
+  // Layout: [stages][receive buffer, f32 [BM][n_pad + 4]][constants][barriers].
   // The receive buffer gets its own space when that still leaves two or more
   // stages, and otherwise reuses the (then idle) pipeline memory.
-  const uint32_t stage_bytes = kBaNB * (kBaBM * 128 + uint32_t(p.n_pad) * 128);
-  const uint32_t recv_bytes = uint32_t(kBaBM) * (p.n_pad + 4) * 4;
+  const uint32_t stage_bytes = kBaNB * (uint32_t(BM) * 128 + uint32_t(p.n_pad) * 128);
+  const uint32_t recv_bytes = uint32_t(BM) * (p.n_pad + 4) * 4;
   const uint32_t const_bytes = uint32_t(4 * nv) * 4;
   const uint32_t tail = const_bytes + 16 + (2 * 6 + 1) * 8 + 16;
   int stages = int((kBaMaxSmem - 1024 - recv_bytes - tail) / stage_bytes);
@@ -486,7 +498,7 @@ cudaError_t launch_ba_gates(const uint16_t* x, int k_stride, const uint16_t* w,
   {
     uint64_t dims[2] = {uint64_t(K), uint64_t(M)};
     uint64_t strides[1] = {uint64_t(k_stride) * 2};
-    uint32_t box[2] = {uint32_t(kBaBK), uint32_t(kBaBM)};
+    uint32_t box[2] = {uint32_t(kBaBK), uint32_t(BM)};
     if (!encode_tmap_bf16(&tx, x, 2, dims, strides, box, true)) return cudaErrorInvalidValue;
   }
   {
@@ -495,15 +507,20 @@ cudaError_t launch_ba_gates(const uint16_t* x, int k_stride, const uint16_t* w,
     uint32_t box[2] = {uint32_t(kBaBK), uint32_t(p.n_pad)};
     if (!encode_tmap_bf16(&tw, w, 2, dims, strides, box, true)) return cudaErrorInvalidValue;
   }
+  auto kernel = BM == 64 ? ba_gates_kernel<64> : ba_gates_kernel<128>;
   cudaError_t e =
-      cudaFuncSetAttribute(ba_gates_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   // K split: the largest power of two <= kBaMaxKS that keeps the grid within
   // the SMs and leaves every CTA at least one K box (KS = 2 for 4576 tokens).
-  const int mtiles = (M + kBaBM - 1) / kBaBM;
-  const int kb_all = (K + kBaBK - 1) / kBaBK;
+  // Clusters of 4 and 8 only while few enough of them are placed at once
+  // (at most ~33 clusters of 4 of these CTAs are resident together), so that
+  // a few tiles still spread their K over many SMs.
+  const int mtiles = (M + BM - 1) / BM;
   int ks = 1;
-  while (ks < kBaMaxKS && mtiles * ks * 2 <= sm_count() && ks * 2 <= kb_all) ks *= 2;
+  while (ks < kBaMaxKS && mtiles * ks * 2 <= sm_count() && ks * 2 <= kb_all &&
+         (ks < 2 || mtiles <= (ks == 2 ? 32 : 16)))
+    ks *= 2;
   p.ks = ks;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(mtiles * ks);
@@ -517,7 +534,7 @@ cudaError_t launch_ba_gates(const uint16_t* x, int k_stride, const uint16_t* w,
   attr.val.clusterDim.z = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, ba_gates_kernel, tx, tw, p);
+  e = cudaLaunchKernelEx(&cfg, kernel, tx, tw, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -32,8 +32,12 @@ def test_ba_gates_full_size_4576x5120():
 
 
 @pytest.mark.parametrize("M,K,nv,vpg", [(1, 5120, 48, 3), (100, 64, 6, 3), (129, 72, 8, 2),
-                                        (300, 8, 4, 4), (256, 1000, 16, 1), (77, 2048, 128, 4)])
+                                        (300, 8, 4, 4), (256, 1000, 16, 1), (77, 2048, 128, 4),
+                                        (40, 5120, 48, 3), (1500, 2048, 48, 3),
+                                        (5000, 1024, 48, 3)])
 def test_ba_gates_ragged_shapes(M, K, nv, vpg):
+    """Includes 64-row tiles split 8 ways along K (M = 40), 4 ways (M = 1500)
+    and 128-row tiles once 64-row pairs no longer fit the SMs (M = 5000)."""
     _check(I.ba_inputs(M, K, nv, vpg, seed=M + K))
 
 
