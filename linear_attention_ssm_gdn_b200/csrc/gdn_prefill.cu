@@ -13,8 +13,9 @@
 //       H^T <- e^{G_C} H^T + (e^{G_C - G_r} Vn)^T K,
 //     and the outputs  o_r = e^{G_r} scale O1_r + (Aqk Vn)_r;
 //   PREPS (all other CTAs) compute everything that does not depend on H, for
-//     chunk items taken from one global order (chunk index major, spine minor;
-//     prep p takes every Pn-th item), two items at a time per CTA:
+//     chunk items of one spine each (prep p serves spine p % S and, with the
+//     other preps of that spine, takes every n-th of its chunks), two items
+//     at a time per CTA:
 //       P1 = [K;Q] K^T                                 (MMA)
 //       A[r][s]   = beta_r e^{G_r-G_s} k_r.k_s, s < r   (f32)
 //       Aqk[r][s] = scale e^{G_r-G_s} q_r.k_s, s <= r
@@ -43,6 +44,7 @@
 // on a younger one (its ring entry was freed by an older, already produced
 // item), so the pipeline cannot deadlock while all CTAs are resident.
 #include <cuda.h>
+#include <string.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -85,14 +87,13 @@ constexpr uint32_t kFlagLine = 64;
 constexpr uint32_t STG_WQ = 0, STG_K = 32768, STG_U = 49152, STG_AQK = 65536, STG_GATE = 73728;
 constexpr uint32_t STG_BYTES = 74752;  // 73 KB
 constexpr uint32_t S_STG = 0;
-constexpr uint32_t S_HT = S_STG + 2 * STG_BYTES;  // H^T bf16, [2 boxes][128 x 128B]
-constexpr uint32_t S_VN = S_HT + 32768;           // Vn^T bf16 [128 x 128B]
+constexpr uint32_t S_OT = S_STG + 2 * STG_BYTES;  // outputs, 2 chunks x 64 rows x d_v bf16
+constexpr uint32_t S_VN = S_OT + 32768;           // Vn^T bf16 [128 x 128B]
 constexpr uint32_t S_VNS = S_VN + 16384;          // e^{G_C - G_r} Vn^T bf16
 constexpr uint32_t S_EG = S_VNS + 16384;          // 2 x 64 f32: scale e^{G_r} per chunk
 constexpr uint32_t S_ECG = S_EG + 512;            // 2 x 64 f32: e^{G_C - G_r} per chunk
-constexpr uint32_t S_OSTG = S_ECG + 512;          // output transpose: 8 warps x 1 KB
-constexpr uint32_t S_BARS = S_OSTG + 8192;
-static_assert(S_HT % 1024 == 0 && STG_BYTES % 1024 == 0, "swizzled tiles are 1024-aligned");
+constexpr uint32_t S_BARS = S_ECG + 512;
+static_assert(S_OT % 1024 == 0 && STG_BYTES % 1024 == 0, "swizzled tiles are 1024-aligned");
 static_assert(STG_GATE + G_GATE_BYTES <= STG_BYTES, "stage layout");
 // ---- prep shared memory: two 128-thread item groups (item k: group k & 1)
 // and three tile sets that rotate over the items (item k: set k % 3), so that
@@ -119,7 +120,8 @@ constexpr uint32_t kSmemBytes =
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 static_assert(S_BARS % 8 == 0 && P_BARS % 8 == 0, "barrier alignment");
-static_assert(P_V >= 32768, "W | U^T staging fits in a tile set");
+static_assert(P_V == 32768 && G_U == 16384 && G_AQK == 32768 && P_SET >= P_V + 8192,
+              "W | U^T | Aqk staging mirrors the ring entry");
 static_assert((GA_GT + PG_EG * 4) % 16 == 0 && (GA_GT + PG_BYTES + PG_EG * 4) % 16 == 0 &&
                   P_GS % 16 == 0, "gate blocks are bulk-copy sources");
 static_assert(P_SET % 1024 == 0 && P_GRP % 1024 == 0 && P_GS % 1024 == 0 && GA_AQK % 1024 == 0,
@@ -259,33 +261,34 @@ __device__ __forceinline__ void it_next(ChunkIter& it, const Params& p) {
 // The items of one prep CTA: global item i = j * S + s (chunk j of spine s),
 // i = prank, prank + Pn, ...; k counts the valid ones (k & 1 picks the group).
 struct PrepIter {
-  int i, k, s, j, h, t0, L;
+  int i, k, s, j, h, t0, L, stride;
   bool ok;
 };
 
+// Prep CTA prank serves one spine, s = prank % S, together with the other
+// preps of the same residue: the n = ceil((Pn - s) / S) of them take its
+// chunks j = prank / S, + n, + 2n, ...  A prep that waits for a free ring
+// entry of its spine therefore never holds back another spine's items.
 template <bool kSeg>
 __device__ __forceinline__ bool pi_fill(PrepIter& it, const Params& p, const int* sJ, int iend) {
-  while (it.i < iend) {
-    const int s = it.i % p.S, j = it.i / p.S;
-    if (j < sJ[s]) {
-      const int units = p.num_seqs * p.H_v;
-      int jj = j;
-      for (int u = s; u < units; u += p.S) {
-        const int nc = unit_chunks<kSeg>(p, u);
-        if (jj < nc) {
-          int tb, te;
-          seq_range<kSeg>(p, u / p.H_v, tb, te);
-          it.s = s;
-          it.j = j;
-          it.h = u % p.H_v;
-          it.t0 = tb + jj * C;
-          it.L = min(C, te - it.t0);
-          return true;
-        }
-        jj -= nc;
+  (void)iend;
+  const int s = it.s;
+  if (it.i < sJ[s]) {
+    const int units = p.num_seqs * p.H_v;
+    int jj = it.i;
+    for (int u = s; u < units; u += p.S) {
+      const int nc = unit_chunks<kSeg>(p, u);
+      if (jj < nc) {
+        int tb, te;
+        seq_range<kSeg>(p, u / p.H_v, tb, te);
+        it.j = it.i;
+        it.h = u % p.H_v;
+        it.t0 = tb + jj * C;
+        it.L = min(C, te - it.t0);
+        return true;
       }
+      jj -= nc;
     }
-    it.i += gridDim.x - p.S;
   }
   return false;
 }
@@ -293,14 +296,17 @@ __device__ __forceinline__ bool pi_fill(PrepIter& it, const Params& p, const int
 template <bool kSeg>
 __device__ __forceinline__ void pi_start(PrepIter& it, const Params& p, const int* sJ, int iend,
                                          int prank) {
-  it.i = prank;
+  const int pn = int(gridDim.x) - p.S;
+  it.s = prank % p.S;
+  it.i = prank / p.S;
+  it.stride = (pn - it.s + p.S - 1) / p.S;
   it.k = 0;
   it.ok = pi_fill<kSeg>(it, p, sJ, iend);
 }
 
 template <bool kSeg>
 __device__ __forceinline__ void pi_next(PrepIter& it, const Params& p, const int* sJ, int iend) {
-  it.i += gridDim.x - p.S;
+  it.i += it.stride;
   ++it.k;
   it.ok = pi_fill<kSeg>(it, p, sJ, iend);
 }
@@ -489,7 +495,8 @@ using namespace pf;
 template <int kLimbs, bool kSeg>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                   const Params p) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned start, kept as an offset from the __shared__ array so
   // that accesses through it stay shared-space (not generic) loads and stores
@@ -531,6 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    if (spine && p.o != nullptr) tma_prefetch_desc(&tm_o);
   }
   // Chunks per spine, for the preps' item walk.
   int Jmax = 0;
@@ -560,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (row j of H^T) and half hh = w >> 2: columns d_k 64 hh .. 64 hh + 63 of
       // H^T (kept in registers, f32) and chunk rows 32 hh .. 32 hh + 31 of Vn^T
       // and of the outputs.  Per chunk c:
-      //   H <- e^{G_C} H + dH (dH of chunk c-1, from TMEM); bf16 copy -> S_HT;
+      //   H <- e^{G_C} H + dH (dH of chunk c-1, from TMEM); bf16 copy -> TMEM;
       //   [Vn' | O1]^T = H^T [W; Q]^T  (one N = 128 MMA);
       //   outputs of chunk c-1 while it runs;
       //   Vn = U - Vn' -> Vn^T, e^{G_C - G_r} Vn^T (bf16);
@@ -571,22 +579,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int j = 32 * qd + lane;
       const uint32_t lane_off = uint32_t(32 * qd) << 16;
       const bool jv = j < D;
-      const uint32_t ostg = sbase + S_OSTG + uint32_t(warp) * 1024;
       float* eg_s = reinterpret_cast<float*>(smem + S_EG);
       float* ecg_s = reinterpret_cast<float*>(smem + S_ECG);
       // Outputs of chunk cl, 16 of this warp's rows 32 hh .. + 31 per call
       // (piece pc), for the d_v lanes of its quadrant: o_r = scale e^{G_r}
-      // O1[r] + O2[r], transposed through this warp's 1 KB buffer and written
-      // as 64-byte row segments.  Piece 0 waits for the chunk's MMAs.
+      // O1[r] + O2[r].  The four warps of half hh write rows r0 .. r0 + 15 of
+      // the chunk's row-major output tile (each warp its 32 columns, 64
+      // contiguous bytes per row) into the chunk's output tile (one per chunk
+      // parity), and one of them stores the 16 rows with a TMA tensor store;
+      // a ragged block (the last chunk of a sequence) goes out row by row
+      // with plain stores instead.  Piece 0 waits for the chunk's MMAs.  A
+      // tile is rewritten two chunks later, after a spine barrier before
+      // which the issuing thread saw all but its two latest stores finish
+      // reading (a chunk's two stores per half).
+      const bool issuer_lane = qd == 0 && lane == 0;
+      const uint32_t row_bytes = uint32_t(2 * D);
       auto epilogue = [&](int cl, int pc, int t0l, int Ll, int hl) -> bool {
         const int ob = cl & 1;
         bool okE = true;
         if (pc == 0) okE = mbar_wait(&bars[SB_OFULL + ob], (cl >> 1) & 1, abort_flag, err, 128u, p.spin_limit);
         tc_fence_after();
         const float* egp = eg_s + 64 * ob;
-        const int e0 = 32 * qd;
+        const int r0 = 32 * hh + 16 * pc;
+        const uint32_t blk = S_OT + 16384u * uint32_t(ob) + uint32_t(r0) * row_bytes;
         {
-          const int r0 = 32 * hh + 16 * pc;
           // every operand in registers first: the shared stores below carry a
           // memory clobber, which would serialise loads placed between them
           float egv[16];
@@ -606,18 +622,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             packed[i] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(egv[i], o1[i], o2[i])));
-          __syncwarp();  // the previous piece's reads of the buffer are done
+          if (jv) {
+            const uint32_t col = sbase + blk + uint32_t(j) * 2;
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            st_shared_u16(ostg + uint32_t(i) * 64 + uint32_t(lane) * 2, uint16_t(packed[i]));
-          __syncwarp();
-#pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            const int id = lane + 32 * m, i = id >> 2, seg = id & 3;
-            const int r = r0 + i;
-            const uint4 val = ld_shared_v4(ostg + uint32_t(i) * 64 + uint32_t(seg) * 16);
-            if (okE && r < Ll && e0 < D && p.o != nullptr)
-              *reinterpret_cast<uint4*>(p.o + (size_t(t0l + r) * p.H_v + hl) * D + e0 + seg * 8) = val;
+            for (int i = 0; i < 16; ++i) st_shared_u16(col + uint32_t(i) * row_bytes, uint16_t(packed[i]));
+          }
+        }
+        fence_proxy_async_smem();  // the tile, before the tensor store reads it
+        named_sync(2 + hh, 128);
+        if (okE && p.o != nullptr && r0 < Ll) {
+          if (r0 + 16 <= Ll) {
+            if (issuer_lane) {
+              tma_store_3d(&tm_o, smem + blk, 0, hl, t0l + r0);
+              tma_store_commit();
+            }
+          } else {  // rows r0 .. Ll - 1 only: 16-byte pieces, 128 threads
+            const int t = 32 * qd + lane, per_row = D / 8;
+            for (int id = t; id < 16 * per_row; id += 128) {
+              const int i = id / per_row, sg = id - i * per_row;
+              if (r0 + i < Ll)
+                *reinterpret_cast<uint4*>(p.o + (size_t(t0l + r0 + i) * p.H_v + hl) * D + 8 * sg) =
+                    ld_shared_v4(sbase + blk + uint32_t(i) * row_bytes + uint32_t(sg) * 16);
+            }
           }
         }
         return okE;
@@ -671,7 +697,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           // part A is released after the [W; Q] MMA: keep the gate factors
           if (tid < 64) eg_s[64 * st + tid] = sg[tid] * p.scale;
           else if (tid < 128) ecg_s[64 * st + tid - 64] = sg[tid];
-          st_row64_bf16(sbase + S_HT + uint32_t(hh) * 16384, uint32_t(j), H);
+          {
+            // bf16 H^T row j, d_k 64 hh .. + 63, as the A operand of the [W; Q]
+            // MMA in tensor memory: the Vn' columns of the other VO buffer
+            // (read out in the previous chunk; its O1 half is left alone)
+            uint32_t hp[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) hp[i] = pack_bf16x2(H[2 * i], H[2 * i + 1]);
+            tmem_st32u(tmem + lane_off + ST_VO + 128u * uint32_t(st ^ 1) + 32u * uint32_t(hh), hp);
+            tmem_st_wait();
+          }
           if constexpr (kLimbs == 2) {
             // the previous chunk's O2 MMA reads the Vn buffers: done first
             if (c > c_first)
@@ -681,6 +716,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
           tc_fence_before();
+          // the output-tile stores of two chunks ago have read their rows (so
+          // the pieces after this barrier may rewrite them)
+          if (issuer_lane) tma_store_wait_read<2>();
           if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts [W; Q]
             agreed = false;
             break;
@@ -735,6 +773,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
           tc_fence_before();
+          if (issuer_lane) tma_store_wait_read<2>();
           if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts dH, O2
             agreed = false;
             break;
@@ -760,6 +799,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) H[32 * q2 + i] = fmaf(dec_prev, H[32 * q2 + i], d[i]);
           }
           ok = epilogue(c - 1, 0, prev_t0, prev_L, h) && ok;
+          // piece 1's rows were last stored two chunks ago, after the latest
+          // barrier: wait for that store here
+          if (issuer_lane) tma_store_wait_read<2>();
+          named_sync(2 + hh, 128);
           ok = epilogue(c - 1, 1, prev_t0, prev_L, h) && ok;
           if (!named_all(1, kSpineSync, ok)) {  // the issuer warp takes part
             ok = false;
@@ -774,6 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
       }
+      if (issuer_lane) tma_store_wait_all<0>();  // every output-tile store is complete
     } else if (warp == 9) {
       // ---------------- issuer: joins the state warps' two barriers per chunk
       // (bar.red: every participant gets the same outcome) and issues
@@ -799,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             for (int kk = 0; kk < ksteps_d; ++kk) {
               const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_bf16_ss(tmem + ST_VO + 128u * st, make_sdesc_sw128(sbase + S_HT + off, 16, 1024),
+              mma_bf16_ts(tmem + ST_VO + 128u * st, tmem + ST_VO + 128u * uint32_t(st ^ 1) + 8u * kk,
                           make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_vo, kk > 0);
             }
             if constexpr (kLimbs == 2) {
@@ -1034,8 +1078,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_global();
           uint8_t* dst = ring_entry(p, it.s, e);
           const uint8_t* ga = smem + P_GRP + g * P_GS;
-          bulk_store_s2g(dst + G_W, smem + t * P_SET, 32768);
-          bulk_store_s2g(dst + G_AQK, ga + GA_AQK, 8192);
+          // W | U^T | Aqk: the set's first 40 KB, laid out as the ring entry
+          bulk_store_s2g(dst + G_W, smem + t * P_SET, 40960);
           bulk_store_s2g(dst + G_GATE, ga + GA_GT + (kg & 1) * PG_BYTES + PG_EG * 4, G_GATE_BYTES);
           tma_store_commit();
           tma_store_wait_read<0>();
@@ -1152,12 +1196,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* set = smem + t * P_SET;
         const float* gt = reinterpret_cast<const float*>(ga + GA_GT + pb * PG_BYTES);
         const uint32_t tm = tmem + PT_WG * g;
-        // gates written, P1 done; the group's Aqk buffer was read by the store
-        // of its previous item k - 2
+        // gates written, P1 done (the group's Aqk buffer was copied into the
+        // set of its previous item k - 2 at that item's end)
         const bool ready =
             mbar_wait(&bars[PB_GATEF + 2 * g + pb], (kg >> 1) & 1, abort_flag, err, 4u, p.spin_limit) &&
-            mbar_wait(&bars[PB_P1F + 2 * g + pb], (kg >> 1) & 1, abort_flag, err, 4u, p.spin_limit) &&
-            (k < 2 || mbar_wait(&bars[PB_STORED + (k - 2) % 3], ((k - 2) / 3) & 1, abort_flag, err, 4u, p.spin_limit));
+            mbar_wait(&bars[PB_P1F + 2 * g + pb], (kg >> 1) & 1, abort_flag, err, 4u, p.spin_limit);
         if (!named_all(gbar, 128, ready)) break;
         tc_fence_after();
         // ---- P1 row pt: K K^T (pt < 64) or Q K^T (pt >= 64), times e^{G_r - G_s}
@@ -1276,6 +1319,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               *reinterpret_cast<uint16_t*>(wcol + sw128_offset(uint32_t(32 * hf + i), wbyte)) =
                   __bfloat16_as_ushort(__float2bfloat16_rn(wv[i]));
           }
+          // Aqk into the set's V boxes (free once the U MMA is done), so that
+          // the group's buffer is its own again for item k + 2
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t off = uint32_t(pt) * 64u + uint32_t(q) * 16u;
+            *reinterpret_cast<uint4*>(set + P_V + off) = *reinterpret_cast<const uint4*>(ga + GA_AQK + off);
+          }
         }
         tc_fence_before();
         fence_proxy_async_smem();
@@ -1371,6 +1421,15 @@ cudaError_t launch_prefill_call(const PrefillCall& c, cudaStream_t s) {
     uint32_t box[3] = {64, 1, 64};
     if (!encode_tmap_bf16(&tv, c.v, 3, dims, strides, box, true)) return cudaErrorInvalidValue;
   }
+  // o [T, H_v, d_v]: the spines store 16 rows x d_v of one head at a time
+  CUtensorMap to;
+  memset(&to, 0, sizeof(to));
+  if (c.o != nullptr) {
+    uint64_t dims[3] = {uint64_t(D), uint64_t(c.H_v), uint64_t(c.total_tokens)};
+    uint64_t strides[2] = {uint64_t(D) * 2, uint64_t(c.H_v) * uint64_t(D) * 2};
+    uint32_t box[3] = {uint32_t(D), 1, 16};
+    if (!encode_tmap_bf16(&to, c.o, 3, dims, strides, box, false)) return cudaErrorInvalidValue;
+  }
   // The plain form (whole sequences, h0 / hT arrays, real v) carries none of
   // the segment-pass branches.
   const bool seg = c.seg != nullptr || c.h0_tab != nullptr || c.hT_tab != nullptr || c.v_zero ||
@@ -1419,7 +1478,7 @@ cudaError_t launch_prefill_call(const PrefillCall& c, cudaStream_t s) {
   attr.val.cooperative = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, p);
+  e = cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, to, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
