@@ -78,7 +78,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for phase `parity` of `bar` to complete.  Gives up (returns false) when
 // *abort becomes nonzero or after `limit` cycles; on a timeout it sets
 // *abort and ORs `err_bit` into *err (a global error word, may be null).
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
+// Inlined: kernels that re-allocate registers per warpgroup (setmaxnreg)
+// cannot share one out-of-line body between warpgroups of different sizes.
+static __device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
                                                     volatile int* abort, uint32_t* err,
                                                     uint32_t err_bit, long long limit) {
   const long long t0 = clock64();
@@ -190,6 +192,17 @@ __device__ __forceinline__ void tma_store_wait_all() {
 
 // Warp-wide: allocate `ncols` TMEM columns (power of two >= 32); the base
 // address is written to *dst_smem.
+// Per-warpgroup register re-allocation (every warp of the warpgroup executes
+// it); the sum over warpgroups must stay within the launch's allocation.
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                    smem_u32(dst_smem)),
@@ -272,6 +285,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
       : "r"(taddr));
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 16 lanes from `taddr` (its lane field picks them) x 2 repetitions of 8
+// columns: thread t gets lanes l = t / 4 and l + 8 at columns c = 2 (t % 4)
+// and c + 1, first for columns 0..7, then 8..15 (v[0..3]: (l, c), (l, c+1),
+// (l+8, c), (l+8, c+1); v[4..7]: the same at c + 8).
+__device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                 "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tmem_ld_wait() {
@@ -370,6 +398,17 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                "r"(d)
+               : "memory");
+}
+
+// Four 8x8 b16 matrices, each stored transposed: thread t holds element
+// (t / 4, 2 (t % 4) + e) of matrix m in the e-th half of reg m; threads
+// 8 m .. 8 m + 7 give the addresses of the stored rows 0..7 of matrix m
+// (16 contiguous bytes each), stored row k being the matrix's column k.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                                  uint32_t d) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+               "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
 
@@ -520,7 +559,7 @@ __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
 // Poll a flag in global memory until it reaches `target` (values only grow).
 // Gives up when *gabort becomes nonzero or after kSpinLimitCycles; on a
 // timeout it sets *gabort and ORs `err_bit` into *err.
-static __device__ __noinline__ bool poll_geq(const uint32_t* flag, uint32_t target,
+static __device__ __forceinline__ bool poll_geq(const uint32_t* flag, uint32_t target,
                                              volatile uint32_t* gabort, uint32_t* err,
                                              uint32_t err_bit,
                                              long long limit = kSpinLimitCycles) {

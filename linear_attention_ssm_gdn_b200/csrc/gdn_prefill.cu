@@ -58,7 +58,10 @@ __device__ uint32_t g_err_prefill;
 namespace pf {
 
 constexpr int C = 64;          // chunk rows
-constexpr int kThreads = 384;  // 12 warps
+constexpr int kThreads = 512;  // 16 warps: 128 registers each at launch, re-allocated below
+constexpr uint32_t kRegsWide = 176, kRegsNarrow = 80;  // warps 0-7 / warps 8-15
+static_assert(2 * 128 * kRegsWide + 2 * 128 * kRegsNarrow == 128 * kThreads,
+              "the re-allocated registers add up to the launch's allocation");
 constexpr int kAS = 68;        // f32 row stride of the A / T scratch (16-byte rows)
 constexpr int kRing = 4;       // ring entries per spine
 constexpr int kMaxSpines = 256;
@@ -73,7 +76,6 @@ constexpr uint32_t kErrGateRise = 64u;
 constexpr uint32_t G_W = 0, G_U = 16384, G_AQK = 32768, G_GATE = 40960;
 constexpr uint32_t G_GATE_BYTES = 528;  // e^{G_r} 64 | e^{G_C-G_r} 64 | e^{G_C} | pad
 constexpr uint32_t SLOT_G = 41984;      // 41 KB, a multiple of 1024
-constexpr uint32_t SLOT_TX = G_GATE + G_GATE_BYTES;
 // ---- flags (workspace head): one 64-byte line for the abort word, then one
 // line per (spine, ring entry): ready count at +0, free count at +32 bytes.
 constexpr uint32_t kFlagLine = 64;
@@ -90,8 +92,8 @@ constexpr uint32_t S_STG = 0;
 constexpr uint32_t S_OT = S_STG + 2 * STG_BYTES;  // outputs, 2 chunks x 64 rows x d_v bf16
 constexpr uint32_t S_VN = S_OT + 32768;           // Vn^T bf16 [128 x 128B]
 constexpr uint32_t S_VNS = S_VN + 16384;          // e^{G_C - G_r} Vn^T bf16
-constexpr uint32_t S_EG = S_VNS + 16384;          // 2 x 64 f32: scale e^{G_r} per chunk
-constexpr uint32_t S_ECG = S_EG + 512;            // 2 x 64 f32: e^{G_C - G_r} per chunk
+constexpr uint32_t S_EG = S_VNS + 16384;          // 4 x 64 f32: scale e^{G_r} per chunk
+constexpr uint32_t S_ECG = S_EG + 1024;           // 2 x 64 f32: e^{G_C - G_r} per chunk
 constexpr uint32_t S_BARS = S_ECG + 512;
 static_assert(S_OT % 1024 == 0 && STG_BYTES % 1024 == 0, "swizzled tiles are 1024-aligned");
 static_assert(STG_GATE + G_GATE_BYTES <= STG_BYTES, "stage layout");
@@ -137,7 +139,8 @@ enum {
   SB_DHFULL = 9,   // dH = Vns^T K done (commit)
   SB_OFULL = 10,   // +buf: O2 (and so O1) done (commit)
   SB_DRAIN = 12,
-  SB_COUNT = 13
+  SB_OEMPTY = 13,  // +buf: the output warps have read O1 / O2 of the chunk (1)
+  SB_COUNT = 15
 };
 // ---- barriers (prep).  Item k: group g = k & 1, kg = k >> 1 its index in
 // the group, tile set k % 3, P1 buffer and gate block kg & 1 of group g.
@@ -557,6 +560,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (!spine)
     for (int s = 0; s < p.S; ++s) Jmax = max(Jmax, sJ[s]);
   const int iend = Jmax * p.S;  // items i < iend (some invalid: chunk j beyond its spine)
+  // Warps 0-7 (the spine's state warps, the preps' item groups) hold the
+  // large register sets; the single-thread roles and the output warps give
+  // theirs up: each role branch below starts with its warpgroup's change
+  // (every warp of a warpgroup makes the same one).
 
   if (spine) {
     // =====================================================================
@@ -564,90 +571,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     // =====================================================================
     const int s = int(blockIdx.x);
     if (warp < 8) {
+      setmaxnreg_inc<kRegsWide>();
       // ---------------- state warps: warp w serves TMEM lane quadrant w & 3
       // (row j of H^T) and half hh = w >> 2: columns d_k 64 hh .. 64 hh + 63 of
       // H^T (kept in registers, f32) and chunk rows 32 hh .. 32 hh + 31 of Vn^T
       // and of the outputs.  Per chunk c:
       //   H <- e^{G_C} H + dH (dH of chunk c-1, from TMEM); bf16 copy -> TMEM;
       //   [Vn' | O1]^T = H^T [W; Q]^T  (one N = 128 MMA);
-      //   outputs of chunk c-1 while it runs;
       //   Vn = U - Vn' -> Vn^T, e^{G_C - G_r} Vn^T (bf16);
       //   dH = Vns^T K,  O2^T = Vn^T Aqk^T;
-      // warp 9 issues the MMAs right after the two named barriers, and chunk
-      // c-1's outputs are written in two halves, one under each of them.
+      // warp 9 issues the MMAs right after the two named barriers; the
+      // outputs are the output warps' (12 - 15), off this chain.
       const int qd = warp & 3, hh = warp >> 2;
       const int j = 32 * qd + lane;
       const uint32_t lane_off = uint32_t(32 * qd) << 16;
       const bool jv = j < D;
       float* eg_s = reinterpret_cast<float*>(smem + S_EG);
       float* ecg_s = reinterpret_cast<float*>(smem + S_ECG);
-      // Outputs of chunk cl, 16 of this warp's rows 32 hh .. + 31 per call
-      // (piece pc), for the d_v lanes of its quadrant: o_r = scale e^{G_r}
-      // O1[r] + O2[r].  The four warps of half hh write rows r0 .. r0 + 15 of
-      // the chunk's row-major output tile (each warp its 32 columns, 64
-      // contiguous bytes per row) into the chunk's output tile (one per chunk
-      // parity), and one of them stores the 16 rows with a TMA tensor store;
-      // a ragged block (the last chunk of a sequence) goes out row by row
-      // with plain stores instead.  Piece 0 waits for the chunk's MMAs.  A
-      // tile is rewritten two chunks later, after a spine barrier before
-      // which the issuing thread saw all but its two latest stores finish
-      // reading (a chunk's two stores per half).
-      const bool issuer_lane = qd == 0 && lane == 0;
-      const uint32_t row_bytes = uint32_t(2 * D);
-      auto epilogue = [&](int cl, int pc, int t0l, int Ll, int hl) -> bool {
-        const int ob = cl & 1;
-        bool okE = true;
-        if (pc == 0) okE = mbar_wait(&bars[SB_OFULL + ob], (cl >> 1) & 1, abort_flag, err, 128u, p.spin_limit);
-        tc_fence_after();
-        const float* egp = eg_s + 64 * ob;
-        const int r0 = 32 * hh + 16 * pc;
-        const uint32_t blk = S_OT + 16384u * uint32_t(ob) + uint32_t(r0) * row_bytes;
-        {
-          // every operand in registers first: the shared stores below carry a
-          // memory clobber, which would serialise loads placed between them
-          float egv[16];
-#pragma unroll
-          for (int i = 0; i < 16; i += 4) {
-            const float4 e4 = *reinterpret_cast<const float4*>(egp + r0 + i);
-            egv[i] = e4.x;
-            egv[i + 1] = e4.y;
-            egv[i + 2] = e4.z;
-            egv[i + 3] = e4.w;
-          }
-          float o1[16], o2[16];
-          tmem_ld16(tmem + lane_off + ST_VO + 128u * ob + 64u + uint32_t(r0), o1);
-          tmem_ld16(tmem + lane_off + ST_O2 + 64u * ob + uint32_t(r0), o2);
-          tmem_ld_wait();
-          uint32_t packed[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            packed[i] = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(egv[i], o1[i], o2[i])));
-          if (jv) {
-            const uint32_t col = sbase + blk + uint32_t(j) * 2;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) st_shared_u16(col + uint32_t(i) * row_bytes, uint16_t(packed[i]));
-          }
-        }
-        fence_proxy_async_smem();  // the tile, before the tensor store reads it
-        named_sync(2 + hh, 128);
-        if (okE && p.o != nullptr && r0 < Ll) {
-          if (r0 + 16 <= Ll) {
-            if (issuer_lane) {
-              tma_store_3d(&tm_o, smem + blk, 0, hl, t0l + r0);
-              tma_store_commit();
-            }
-          } else {  // rows r0 .. Ll - 1 only: 16-byte pieces, 128 threads
-            const int t = 32 * qd + lane, per_row = D / 8;
-            for (int id = t; id < 16 * per_row; id += 128) {
-              const int i = id / per_row, sg = id - i * per_row;
-              if (r0 + i < Ll)
-                *reinterpret_cast<uint4*>(p.o + (size_t(t0l + r0 + i) * p.H_v + hl) * D + 8 * sg) =
-                    ld_shared_v4(sbase + blk + uint32_t(i) * row_bytes + uint32_t(sg) * 16);
-            }
-          }
-        }
-        return okE;
-      };
       // Every exit from these loops follows a bar.red agreement that the
       // issuer warp takes part in, so the two sides always leave together.
       int c = 0;
@@ -674,7 +614,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int c_first = c;
         float dec_prev = 1.f;
-        int prev_t0 = tb, prev_L = 0;
         for (int t0 = tb; t0 < te; t0 += C, ++c) {
           const int st = c & 1;
           const float* sg = reinterpret_cast<const float*>(smem + S_STG + st * STG_BYTES + STG_GATE);
@@ -695,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float dec_cur = sg[128];
           // part A is released after the [W; Q] MMA: keep the gate factors
-          if (tid < 64) eg_s[64 * st + tid] = sg[tid] * p.scale;
+          if (tid < 64) eg_s[64 * (c & 3) + tid] = sg[tid] * p.scale;
           else if (tid < 128) ecg_s[64 * st + tid - 64] = sg[tid];
           {
             // bf16 H^T row j, d_k 64 hh .. + 63, as the A operand of the [W; Q]
@@ -716,16 +655,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
           tc_fence_before();
-          // the output-tile stores of two chunks ago have read their rows (so
-          // the pieces after this barrier may rewrite them)
-          if (issuer_lane) tma_store_wait_read<2>();
           if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts [W; Q]
             agreed = false;
             break;
           }
-          bool okE = true;
-          if (c > c_first) okE = epilogue(c - 1, 0, prev_t0, prev_L, h);
-          ok = ok && okE;
           // Vn = U - Vn'  ->  Vn^T and e^{G_C - G_r} Vn^T rows in bf16
           ok = mbar_wait(&bars[SB_VOFULL], c & 1, abort_flag, err, 16u, p.spin_limit) && ok;
           ok = mbar_wait(&bars[SB_BF + st], (c >> 1) & 1, abort_flag, err, 16u, p.spin_limit) && ok;
@@ -773,21 +706,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
           tc_fence_before();
-          if (issuer_lane) tma_store_wait_read<2>();
           if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts dH, O2
             agreed = false;
             break;
           }
-          if (c > c_first) ok = epilogue(c - 1, 1, prev_t0, prev_L, h) && okE && ok;
           dec_prev = dec_cur;
-          prev_t0 = t0;
-          prev_L = min(C, te - t0);
         }
         if (!agreed) {
           ok = false;
           break;
         }
-        if (te > tb) {  // the last chunk: its update and its outputs
+        if (te > tb) {  // the last chunk's update
           ok = mbar_wait(&bars[SB_DHFULL], (c - 1) & 1, abort_flag, err, 16u, p.spin_limit) && ok;
           tc_fence_after();
 #pragma unroll
@@ -798,12 +727,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) H[32 * q2 + i] = fmaf(dec_prev, H[32 * q2 + i], d[i]);
           }
-          ok = epilogue(c - 1, 0, prev_t0, prev_L, h) && ok;
-          // piece 1's rows were last stored two chunks ago, after the latest
-          // barrier: wait for that store here
-          if (issuer_lane) tma_store_wait_read<2>();
-          named_sync(2 + hh, 128);
-          ok = epilogue(c - 1, 1, prev_t0, prev_L, h) && ok;
+          tc_fence_before();
           if (!named_all(1, kSpineSync, ok)) {  // the issuer warp takes part
             ok = false;
             break;
@@ -817,8 +741,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
       }
-      if (issuer_lane) tma_store_wait_all<0>();  // every output-tile store is complete
-    } else if (warp == 9) {
+    } else {
+      setmaxnreg_dec<kRegsNarrow>();
+      if (warp == 9) {
       // ---------------- issuer: joins the state warps' two barriers per chunk
       // (bar.red: every participant gets the same outcome) and issues
       //   after the first:  [Vn' | O1]^T = H^T [W; Q]^T              (N = 128)
@@ -840,6 +765,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           if (leader) {
+            // the output warps are done with this parity's O1 / O2 (chunk c - 2)
+            if (c >= 2)
+              mbar_wait(&bars[SB_OEMPTY + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 16u, p.spin_limit);
             tc_fence_after();
             for (int kk = 0; kk < ksteps_d; ++kk) {
               const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -884,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&bars[SB_DRAIN], 0, nullptr, err, 8u);
       }
       __syncwarp();
-    } else if (warp == 8) {
+      } else if (warp == 8) {
       // ---------------- feeder: chunk c into stage c & 1, part by part.
       // Part A (Q by TMA; W and the gates from the ring entry) as soon as
       // chunk c - 2's [W; Q] MMA is done; part B (K by TMA; U^T and Aqk) once
@@ -949,6 +877,105 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (cc >= 0) mbar_wait(&bars[SB_BF + (cc & 1)], (cc >> 1) & 1, nullptr, err, 32u);
       }
       __syncwarp();
+      } else if (warp >= 12) {
+        // ---------------- output warps, off the chain: for every chunk c of
+        // this spine, once OFULL(c), warp 12 + q reads TMEM lane quadrant q
+        // (d_v 32 q .. 32 q + 31) of O1^T (upper half of the VO buffer) and
+        // O2^T, 16 lanes x 16 chunk rows at a time in the 16x256b form, forms
+        // o_r = scale e^{G_r} O1[r] + O2[r] in bf16 and writes it with
+        // transposing matrix stores into the output tile of the chunk's
+        // parity: two 64-column halves of [64 rows][128 B], 16-byte chunks
+        // swizzled by row (the tensor stores' 128-byte swizzle).  Then it
+        // hands the TMEM buffers back to the issuer (OEMPTY), and one thread
+        // stores the full 16-row blocks with TMA tensor stores; the rows of a
+        // ragged block go out with plain stores.  A tile is rewritten two
+        // chunks later, and the storing thread sees every earlier store
+        // finish reading before the barrier that precedes that rewrite.
+        const int qd = warp & 3;
+        const int tq = lane & 3;                  // fragment column pair
+        const int sm = lane >> 3, sk = lane & 7;  // stored matrix, stored row
+        const float* eg_s = reinterpret_cast<const float*>(smem + S_EG);
+        const bool elect = warp == 12 && lane == 0;
+        const int halves = D / 64;
+        int c = 0;
+        bool ok = true;
+        for (int u = s; u < units && ok; u += p.S) {
+          const int h = u % p.H_v;
+          int tb, te;
+          seq_range<kSeg>(p, u / p.H_v, tb, te);
+          for (int t0 = tb; t0 < te; t0 += C, ++c) {
+            const int ob = c & 1, L = min(C, te - t0);
+            bool okc =
+                mbar_wait(&bars[SB_OFULL + ob], (c >> 1) & 1, abort_flag, err, 128u, p.spin_limit);
+            tc_fence_after();
+            const float* egp = eg_s + 64 * (c & 3);
+            const uint32_t tile = S_OT + 16384u * uint32_t(ob);
+#pragma unroll 1
+            for (int r0 = 0; r0 < 64; r0 += 16) {
+              // both 16-lane halves of the quadrant: four loads, one wait
+              float a1[2][8], a2[2][8];
+#pragma unroll
+              for (int hf = 0; hf < 2; ++hf) {
+                const uint32_t lb = uint32_t(32 * qd + 16 * hf);  // TMEM lane base (d_v)
+                if (int(lb) < D) {  // warp-uniform (d = 64: quadrants 2, 3 empty)
+                  tmem_ld_16x256b_x2(tmem + (lb << 16) + ST_VO + 128u * uint32_t(ob) + 64u + uint32_t(r0), a1[hf]);
+                  tmem_ld_16x256b_x2(tmem + (lb << 16) + ST_O2 + 64u * uint32_t(ob) + uint32_t(r0), a2[hf]);
+                }
+              }
+              tmem_ld_wait();
+              const float2 e0 = *reinterpret_cast<const float2*>(egp + r0 + 2 * tq);
+              const float2 e1 = *reinterpret_cast<const float2*>(egp + r0 + 8 + 2 * tq);
+#pragma unroll
+              for (int hf = 0; hf < 2; ++hf) {
+                const int lb = 32 * qd + 16 * hf;
+                if (lb >= D) continue;
+                // fragments: rows = d_v lb + t / 4 (+ 8), columns = chunk rows
+                // r0 + 2 (t % 4), + 1 (+ 8)
+                const float* x = a1[hf];
+                const float* y = a2[hf];
+                const uint32_t m0 = pack_bf16x2(fmaf(e0.x, x[0], y[0]), fmaf(e0.y, x[1], y[1]));
+                const uint32_t m1 = pack_bf16x2(fmaf(e0.x, x[2], y[2]), fmaf(e0.y, x[3], y[3]));
+                const uint32_t m2 = pack_bf16x2(fmaf(e1.x, x[4], y[4]), fmaf(e1.y, x[5], y[5]));
+                const uint32_t m3 = pack_bf16x2(fmaf(e1.x, x[6], y[6]), fmaf(e1.y, x[7], y[7]));
+                // stored row sk of matrix sm: chunk row r0 + sk (+ 8), d_v lb (+ 8)
+                const int row = r0 + sk + 8 * (sm >> 1);
+                const int c0 = lb + 8 * (sm & 1);
+                const uint32_t addr = sbase + tile + uint32_t(c0 >> 6) * 8192u + uint32_t(row) * 128u +
+                                      (uint32_t(((c0 & 63) >> 3) ^ (row & 7)) << 4);
+                if (okc) stmatrix_x4_trans(addr, m0, m1, m2, m3);
+              }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();  // the tile, before the tensor stores read it
+            if (elect) tma_store_wait_read<0>();  // the other tile's stores (chunk c - 1)
+            if (!named_all(2, 128, okc)) {
+              ok = false;
+              break;
+            }
+            if (elect) {
+              mbar_arrive(&bars[SB_OEMPTY + ob]);
+              if (p.o != nullptr) {
+                for (int r0 = 0; r0 + 16 <= L; r0 += 16)
+                  for (int hf = 0; hf < halves; ++hf)
+                    tma_store_3d(&tm_o, smem + tile + uint32_t(hf) * 8192u + uint32_t(r0) * 128u, 64 * hf,
+                                 h, t0 + r0);
+                tma_store_commit();
+              }
+            }
+            if ((L & 15) != 0 && p.o != nullptr) {  // rows L & ~15 .. L - 1: 16-byte pieces
+              const int rb = L & ~15, per_row = D / 8, t = 32 * qd + lane;
+              for (int id = t; id < (L - rb) * per_row; id += 128) {
+                const int i = id / per_row, sg = id - i * per_row, row = rb + i;
+                *reinterpret_cast<uint4*>(p.o + (size_t(t0 + row) * p.H_v + h) * D + 8 * sg) =
+                    ld_shared_v4(sbase + tile + uint32_t(sg >> 3) * 8192u + uint32_t(row) * 128u +
+                                 (uint32_t((sg & 7) ^ (row & 7)) << 4));
+              }
+            }
+          }
+        }
+        if (elect) tma_store_wait_all<0>();  // every output store is complete
+        __syncwarp();
+      }  // warps 10 and 11: no spine role
     }
   } else {
     // =====================================================================
@@ -957,7 +984,165 @@ __global__ void __launch_bounds__(kThreads, 1)
     // group, tile set k % 3, P1 TMEM buffer and gate block kg & 1 of group g.
     // =====================================================================
     const int prank = int(blockIdx.x) - p.S;
-    if (warp == 8) {
+    if (warp < 8) {
+      setmaxnreg_inc<kRegsWide>();
+      // ---------------- groups: 128 threads each, items k = g, g + 2, ...
+      const int g = warp >> 2;
+      const int pt = tid & 127;
+      const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+      uint8_t* ga = smem + P_GRP + g * P_GS;
+      float* M = reinterpret_cast<float*>(ga + GA_AF);
+      float* Xs = reinterpret_cast<float*>(ga + GA_XS);
+      const int gbar = 1 + 3 * g;  // this group's named barriers: gbar (all), gbar+1, gbar+2
+      PrepIter it;
+      pi_start<kSeg>(it, p, sJ, iend, prank);
+      pi_align<kSeg>(it, p, sJ, iend, g);
+      while (it.ok) {
+        const int k = it.k, kg = k >> 1, t = k % 3, pb = kg & 1;
+        uint8_t* set = smem + t * P_SET;
+        const float* gt = reinterpret_cast<const float*>(ga + GA_GT + pb * PG_BYTES);
+        const uint32_t tm = tmem + PT_WG * g;
+        // gates written, P1 done (the group's Aqk buffer was copied into the
+        // set of its previous item k - 2 at that item's end)
+        const bool ready =
+            mbar_wait(&bars[PB_GATEF + 2 * g + pb], (kg >> 1) & 1, abort_flag, err, 4u, p.spin_limit) &&
+            mbar_wait(&bars[PB_P1F + 2 * g + pb], (kg >> 1) & 1, abort_flag, err, 4u, p.spin_limit);
+        if (!named_all(gbar, 128, ready)) break;
+        tc_fence_after();
+        // ---- P1 row pt: K K^T (pt < 64) or Q K^T (pt >= 64), times e^{G_r - G_s}
+        // (s <= r): two factors <= 1 for the blocks of s before r's 16-row
+        // block, a direct exponential inside it.
+        {
+          const int r = pt & 63, rb = r >> 4;
+          const float Gr = gt[PG_G + r];
+          const float e1 = gt[PG_E1 + r];
+          const float br = gt[PG_BET + r];
+          const float* e2 = gt + PG_E2 + 64 * rb;
+          float v[64];
+          tmem_ld32(tm + lane_off + 64u * pb, *reinterpret_cast<float(*)[32]>(v));
+          tmem_ld32(tm + lane_off + 64u * pb + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(&bars[PB_P1FREE + 2 * g + pb]);
+#pragma unroll
+          for (int sb = 0; sb < 4; ++sb) {
+            float f[16];
+            if (sb < rb) {
+#pragma unroll
+              for (int jj = 0; jj < 16; jj += 4) {
+                const float4 e4 = *reinterpret_cast<const float4*>(e2 + 16 * sb + jj);
+                f[jj] = e1 * e4.x;
+                f[jj + 1] = e1 * e4.y;
+                f[jj + 2] = e1 * e4.z;
+                f[jj + 3] = e1 * e4.w;
+              }
+            } else if (sb == rb) {
+#pragma unroll
+              for (int jj = 0; jj < 16; jj += 4) {
+                const int s2 = 16 * sb + jj;
+                const float4 g4 = *reinterpret_cast<const float4*>(gt + PG_G + s2);
+                f[jj] = (s2 <= r) ? __expf(Gr - g4.x) : 0.f;
+                f[jj + 1] = (s2 + 1 <= r) ? __expf(Gr - g4.y) : 0.f;
+                f[jj + 2] = (s2 + 2 <= r) ? __expf(Gr - g4.z) : 0.f;
+                f[jj + 3] = (s2 + 3 <= r) ? __expf(Gr - g4.w) : 0.f;
+              }
+            } else {
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj) f[jj] = 0.f;
+            }
+            if (pt < 64) {  // A[r][s] = beta_r e^{G_r-G_s} k_r.k_s, s < r
+#pragma unroll
+              for (int jj = 0; jj < 16; jj += 4) {
+                const int s2 = 16 * sb + jj;
+                *reinterpret_cast<float4*>(M + r * kAS + s2) = make_float4(
+                    s2 + 0 < r ? br * f[jj] * v[s2] : 0.f,
+                    s2 + 1 < r ? br * f[jj + 1] * v[s2 + 1] : 0.f,
+                    s2 + 2 < r ? br * f[jj + 2] * v[s2 + 2] : 0.f,
+                    s2 + 3 < r ? br * f[jj + 3] * v[s2 + 3] : 0.f);
+              }
+            } else {  // Aqk[r][s] = scale e^{G_r-G_s} q_r.k_s, s <= r  (bf16, swizzled)
+              const float sc = p.scale;
+#pragma unroll
+              for (int hc = 0; hc < 2; ++hc) {
+                const int s2 = 16 * sb + 8 * hc, o = 8 * hc;
+                *reinterpret_cast<uint4*>(ga + GA_AQK + sw128_offset(r, (2 * sb + hc) * 16)) =
+                    make_uint4(pack_bf16x2(sc * f[o] * v[s2], sc * f[o + 1] * v[s2 + 1]),
+                               pack_bf16x2(sc * f[o + 2] * v[s2 + 2], sc * f[o + 3] * v[s2 + 3]),
+                               pack_bf16x2(sc * f[o + 4] * v[s2 + 4], sc * f[o + 5] * v[s2 + 5]),
+                               pack_bf16x2(sc * f[o + 6] * v[s2 + 6], sc * f[o + 7] * v[s2 + 7]));
+              }
+            }
+          }
+        }
+        named_sync(gbar, 128);
+        // ---- T = (I + A)^{-1}, in place
+        invert_unit_lower64(M, Xs, pt, gbar);
+        // ---- T1 = T diag(beta e^G) (rows pt < 64), T2 = T diag(beta) (rows pt >= 64),
+        // into the item's Q boxes (Q was last read by P1)
+        {
+          const int r = pt & 63;
+          const float* scv = gt + (pt < 64 ? PG_BEG : PG_BET);
+          uint8_t* tile = set + (pt < 64 ? P_T1B : P_T2B);
+#pragma unroll 1
+          for (int cc = 0; cc < 8; ++cc) {
+            const float4 ta = *reinterpret_cast<const float4*>(M + r * kAS + 8 * cc);
+            const float4 tb2 = *reinterpret_cast<const float4*>(M + r * kAS + 8 * cc + 4);
+            const float4 sa = *reinterpret_cast<const float4*>(scv + 8 * cc);
+            const float4 sb2 = *reinterpret_cast<const float4*>(scv + 8 * cc + 4);
+            const int s0 = 8 * cc;
+            *reinterpret_cast<uint4*>(tile + sw128_offset(r, cc * 16)) = make_uint4(
+                pack_bf16x2(s0 + 0 <= r ? ta.x * sa.x : 0.f, s0 + 1 <= r ? ta.y * sa.y : 0.f),
+                pack_bf16x2(s0 + 2 <= r ? ta.z * sa.z : 0.f, s0 + 3 <= r ? ta.w * sa.w : 0.f),
+                pack_bf16x2(s0 + 4 <= r ? tb2.x * sb2.x : 0.f, s0 + 5 <= r ? tb2.y * sb2.y : 0.f),
+                pack_bf16x2(s0 + 6 <= r ? tb2.z * sb2.z : 0.f, s0 + 7 <= r ? tb2.w * sb2.w : 0.f));
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars[PB_TREADY + g]);
+        // ---- W (row-major), U^T into [0, 32 KB) of the item's set
+        if (!named_all(gbar, 128, mbar_wait(&bars[PB_WUF + g], kg & 1, abort_flag, err, 4u, p.spin_limit))) break;
+        tc_fence_after();
+        {
+          uint8_t* wcol = set + G_W + uint32_t(pt >> 6) * 8192;
+          const uint32_t wbyte = uint32_t(pt & 63) * 2;
+#pragma unroll 1
+          for (int hf = 0; hf < 2; ++hf) {
+            float wv[32], uv[32];
+            tmem_ld32(tm + lane_off + PT_W + 32u * hf, wv);
+            tmem_ld32(tm + lane_off + PT_U + 32u * hf, uv);
+            tmem_ld_wait();
+#pragma unroll
+            for (int hc = 0; hc < 4; ++hc) {
+              const uint32_t off = sw128_offset(pt, (4 * hf + hc) * 16);
+              *reinterpret_cast<uint4*>(set + G_U + off) =
+                  make_uint4(pack_bf16x2(uv[8 * hc], uv[8 * hc + 1]),
+                             pack_bf16x2(uv[8 * hc + 2], uv[8 * hc + 3]),
+                             pack_bf16x2(uv[8 * hc + 4], uv[8 * hc + 5]),
+                             pack_bf16x2(uv[8 * hc + 6], uv[8 * hc + 7]));
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              *reinterpret_cast<uint16_t*>(wcol + sw128_offset(uint32_t(32 * hf + i), wbyte)) =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(wv[i]));
+          }
+          // Aqk into the set's V boxes (free once the U MMA is done), so that
+          // the group's buffer is its own again for item k + 2
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t off = uint32_t(pt) * 64u + uint32_t(q) * 16u;
+            *reinterpret_cast<uint4*>(set + P_V + off) = *reinterpret_cast<const uint4*>(ga + GA_AQK + off);
+          }
+        }
+        tc_fence_before();
+        fence_proxy_async_smem();
+        named_sync(gbar, 128);
+        if (pt == 0) mbar_arrive(&bars[PB_STAGED + g]);
+        pi_next<kSeg>(it, p, sJ, iend);
+        pi_align<kSeg>(it, p, sJ, iend, g);
+      }
+    } else {
+      setmaxnreg_dec<kRegsNarrow>();
+      if (warp == 8) {
       // ---------------- loader: item k's K, Q, V tiles (TMA, lane 0) once set
       // k % 3 is free (item k - 3 stored)
       PrepIter it;
@@ -1179,161 +1364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicExch(const_cast<uint32_t*>(gabort), 1u);
       }
       __syncwarp();
-    } else if (warp < 8) {
-      // ---------------- groups: 128 threads each, items k = g, g + 2, ...
-      const int g = warp >> 2;
-      const int pt = tid & 127;
-      const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
-      uint8_t* ga = smem + P_GRP + g * P_GS;
-      float* M = reinterpret_cast<float*>(ga + GA_AF);
-      float* Xs = reinterpret_cast<float*>(ga + GA_XS);
-      const int gbar = 1 + 3 * g;  // this group's named barriers: gbar (all), gbar+1, gbar+2
-      PrepIter it;
-      pi_start<kSeg>(it, p, sJ, iend, prank);
-      pi_align<kSeg>(it, p, sJ, iend, g);
-      while (it.ok) {
-        const int k = it.k, kg = k >> 1, t = k % 3, pb = kg & 1;
-        uint8_t* set = smem + t * P_SET;
-        const float* gt = reinterpret_cast<const float*>(ga + GA_GT + pb * PG_BYTES);
-        const uint32_t tm = tmem + PT_WG * g;
-        // gates written, P1 done (the group's Aqk buffer was copied into the
-        // set of its previous item k - 2 at that item's end)
-        const bool ready =
-            mbar_wait(&bars[PB_GATEF + 2 * g + pb], (kg >> 1) & 1, abort_flag, err, 4u, p.spin_limit) &&
-            mbar_wait(&bars[PB_P1F + 2 * g + pb], (kg >> 1) & 1, abort_flag, err, 4u, p.spin_limit);
-        if (!named_all(gbar, 128, ready)) break;
-        tc_fence_after();
-        // ---- P1 row pt: K K^T (pt < 64) or Q K^T (pt >= 64), times e^{G_r - G_s}
-        // (s <= r): two factors <= 1 for the blocks of s before r's 16-row
-        // block, a direct exponential inside it.
-        {
-          const int r = pt & 63, rb = r >> 4;
-          const float Gr = gt[PG_G + r];
-          const float e1 = gt[PG_E1 + r];
-          const float br = gt[PG_BET + r];
-          const float* e2 = gt + PG_E2 + 64 * rb;
-          float v[64];
-          tmem_ld32(tm + lane_off + 64u * pb, *reinterpret_cast<float(*)[32]>(v));
-          tmem_ld32(tm + lane_off + 64u * pb + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-          tmem_ld_wait();
-          tc_fence_before();
-          mbar_arrive(&bars[PB_P1FREE + 2 * g + pb]);
-#pragma unroll
-          for (int sb = 0; sb < 4; ++sb) {
-            float f[16];
-            if (sb < rb) {
-#pragma unroll
-              for (int jj = 0; jj < 16; jj += 4) {
-                const float4 e4 = *reinterpret_cast<const float4*>(e2 + 16 * sb + jj);
-                f[jj] = e1 * e4.x;
-                f[jj + 1] = e1 * e4.y;
-                f[jj + 2] = e1 * e4.z;
-                f[jj + 3] = e1 * e4.w;
-              }
-            } else if (sb == rb) {
-#pragma unroll
-              for (int jj = 0; jj < 16; jj += 4) {
-                const int s2 = 16 * sb + jj;
-                const float4 g4 = *reinterpret_cast<const float4*>(gt + PG_G + s2);
-                f[jj] = (s2 <= r) ? __expf(Gr - g4.x) : 0.f;
-                f[jj + 1] = (s2 + 1 <= r) ? __expf(Gr - g4.y) : 0.f;
-                f[jj + 2] = (s2 + 2 <= r) ? __expf(Gr - g4.z) : 0.f;
-                f[jj + 3] = (s2 + 3 <= r) ? __expf(Gr - g4.w) : 0.f;
-              }
-            } else {
-#pragma unroll
-              for (int jj = 0; jj < 16; ++jj) f[jj] = 0.f;
-            }
-            if (pt < 64) {  // A[r][s] = beta_r e^{G_r-G_s} k_r.k_s, s < r
-#pragma unroll
-              for (int jj = 0; jj < 16; jj += 4) {
-                const int s2 = 16 * sb + jj;
-                *reinterpret_cast<float4*>(M + r * kAS + s2) = make_float4(
-                    s2 + 0 < r ? br * f[jj] * v[s2] : 0.f,
-                    s2 + 1 < r ? br * f[jj + 1] * v[s2 + 1] : 0.f,
-                    s2 + 2 < r ? br * f[jj + 2] * v[s2 + 2] : 0.f,
-                    s2 + 3 < r ? br * f[jj + 3] * v[s2 + 3] : 0.f);
-              }
-            } else {  // Aqk[r][s] = scale e^{G_r-G_s} q_r.k_s, s <= r  (bf16, swizzled)
-              const float sc = p.scale;
-#pragma unroll
-              for (int hc = 0; hc < 2; ++hc) {
-                const int s2 = 16 * sb + 8 * hc, o = 8 * hc;
-                *reinterpret_cast<uint4*>(ga + GA_AQK + sw128_offset(r, (2 * sb + hc) * 16)) =
-                    make_uint4(pack_bf16x2(sc * f[o] * v[s2], sc * f[o + 1] * v[s2 + 1]),
-                               pack_bf16x2(sc * f[o + 2] * v[s2 + 2], sc * f[o + 3] * v[s2 + 3]),
-                               pack_bf16x2(sc * f[o + 4] * v[s2 + 4], sc * f[o + 5] * v[s2 + 5]),
-                               pack_bf16x2(sc * f[o + 6] * v[s2 + 6], sc * f[o + 7] * v[s2 + 7]));
-              }
-            }
-          }
-        }
-        named_sync(gbar, 128);
-        // ---- T = (I + A)^{-1}, in place
-        invert_unit_lower64(M, Xs, pt, gbar);
-        // ---- T1 = T diag(beta e^G) (rows pt < 64), T2 = T diag(beta) (rows pt >= 64),
-        // into the item's Q boxes (Q was last read by P1)
-        {
-          const int r = pt & 63;
-          const float* scv = gt + (pt < 64 ? PG_BEG : PG_BET);
-          uint8_t* tile = set + (pt < 64 ? P_T1B : P_T2B);
-#pragma unroll 1
-          for (int cc = 0; cc < 8; ++cc) {
-            const float4 ta = *reinterpret_cast<const float4*>(M + r * kAS + 8 * cc);
-            const float4 tb2 = *reinterpret_cast<const float4*>(M + r * kAS + 8 * cc + 4);
-            const float4 sa = *reinterpret_cast<const float4*>(scv + 8 * cc);
-            const float4 sb2 = *reinterpret_cast<const float4*>(scv + 8 * cc + 4);
-            const int s0 = 8 * cc;
-            *reinterpret_cast<uint4*>(tile + sw128_offset(r, cc * 16)) = make_uint4(
-                pack_bf16x2(s0 + 0 <= r ? ta.x * sa.x : 0.f, s0 + 1 <= r ? ta.y * sa.y : 0.f),
-                pack_bf16x2(s0 + 2 <= r ? ta.z * sa.z : 0.f, s0 + 3 <= r ? ta.w * sa.w : 0.f),
-                pack_bf16x2(s0 + 4 <= r ? tb2.x * sb2.x : 0.f, s0 + 5 <= r ? tb2.y * sb2.y : 0.f),
-                pack_bf16x2(s0 + 6 <= r ? tb2.z * sb2.z : 0.f, s0 + 7 <= r ? tb2.w * sb2.w : 0.f));
-          }
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&bars[PB_TREADY + g]);
-        // ---- W (row-major), U^T into [0, 32 KB) of the item's set
-        if (!named_all(gbar, 128, mbar_wait(&bars[PB_WUF + g], kg & 1, abort_flag, err, 4u, p.spin_limit))) break;
-        tc_fence_after();
-        {
-          uint8_t* wcol = set + G_W + uint32_t(pt >> 6) * 8192;
-          const uint32_t wbyte = uint32_t(pt & 63) * 2;
-#pragma unroll 1
-          for (int hf = 0; hf < 2; ++hf) {
-            float wv[32], uv[32];
-            tmem_ld32(tm + lane_off + PT_W + 32u * hf, wv);
-            tmem_ld32(tm + lane_off + PT_U + 32u * hf, uv);
-            tmem_ld_wait();
-#pragma unroll
-            for (int hc = 0; hc < 4; ++hc) {
-              const uint32_t off = sw128_offset(pt, (4 * hf + hc) * 16);
-              *reinterpret_cast<uint4*>(set + G_U + off) =
-                  make_uint4(pack_bf16x2(uv[8 * hc], uv[8 * hc + 1]),
-                             pack_bf16x2(uv[8 * hc + 2], uv[8 * hc + 3]),
-                             pack_bf16x2(uv[8 * hc + 4], uv[8 * hc + 5]),
-                             pack_bf16x2(uv[8 * hc + 6], uv[8 * hc + 7]));
-            }
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              *reinterpret_cast<uint16_t*>(wcol + sw128_offset(uint32_t(32 * hf + i), wbyte)) =
-                  __bfloat16_as_ushort(__float2bfloat16_rn(wv[i]));
-          }
-          // Aqk into the set's V boxes (free once the U MMA is done), so that
-          // the group's buffer is its own again for item k + 2
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t off = uint32_t(pt) * 64u + uint32_t(q) * 16u;
-            *reinterpret_cast<uint4*>(set + P_V + off) = *reinterpret_cast<const uint4*>(ga + GA_AQK + off);
-          }
-        }
-        tc_fence_before();
-        fence_proxy_async_smem();
-        named_sync(gbar, 128);
-        if (pt == 0) mbar_arrive(&bars[PB_STAGED + g]);
-        pi_next<kSeg>(it, p, sJ, iend);
-        pi_align<kSeg>(it, p, sJ, iend, g);
-      }
+      }  // warps 12 - 15: no prep role
     }
   }
 
@@ -1421,14 +1452,14 @@ cudaError_t launch_prefill_call(const PrefillCall& c, cudaStream_t s) {
     uint32_t box[3] = {64, 1, 64};
     if (!encode_tmap_bf16(&tv, c.v, 3, dims, strides, box, true)) return cudaErrorInvalidValue;
   }
-  // o [T, H_v, d_v]: the spines store 16 rows x d_v of one head at a time
+  // o [T, H_v, d_v]: the spines store 16 rows x 64 columns of one head at a time
   CUtensorMap to;
   memset(&to, 0, sizeof(to));
   if (c.o != nullptr) {
     uint64_t dims[3] = {uint64_t(D), uint64_t(c.H_v), uint64_t(c.total_tokens)};
     uint64_t strides[2] = {uint64_t(D) * 2, uint64_t(c.H_v) * uint64_t(D) * 2};
-    uint32_t box[3] = {uint32_t(D), 1, 16};
-    if (!encode_tmap_bf16(&to, c.o, 3, dims, strides, box, false)) return cudaErrorInvalidValue;
+    uint32_t box[3] = {64, 1, 16};  // 16 rows x 64 columns, 128-byte swizzle
+    if (!encode_tmap_bf16(&to, c.o, 3, dims, strides, box, true)) return cudaErrorInvalidValue;
   }
   // The plain form (whole sequences, h0 / hT arrays, real v) carries none of
   // the segment-pass branches.
