@@ -8,10 +8,12 @@
 //
 //   SPINES (the first S CTAs) each own (sequence, v-head) units u = s, s+S, ...
 //     and run their per-chunk critical chain on tcgen05 MMAs with TMEM
-//     accumulators (M = d_v = 128 lanes), keeping H^T in registers (f32):
+//     accumulators (M = d_v = 128 lanes), keeping H^T in registers (f32) and
+//     its bf16 copy in TMEM as the A operand of the first MMA:
 //       [Vn' | O1]^T = H^T [W; Q]^T,  Vn = U - Vn',
-//       H^T <- e^{G_C} H^T + (e^{G_C - G_r} Vn)^T K,
-//     and the outputs  o_r = e^{G_r} scale O1_r + (Aqk Vn)_r;
+//       H^T <- e^{G_C} H^T + (e^{G_C - G_r} Vn)^T K;
+//     a separate output warpgroup forms  o_r = e^{G_r} scale O1_r + (Aqk Vn)_r
+//     off that chain and stores it with TMA tensor stores;
 //   PREPS (all other CTAs) compute everything that does not depend on H, for
 //     chunk items of one spine each (prep p serves spine p % S and, with the
 //     other preps of that spine, takes every n-th of its chunks), two items
@@ -39,10 +41,15 @@
 // grid-wide abort word, and every CTA then returns instead of waiting.  Named
 // barriers are used only among threads that are all guaranteed to arrive.
 //
-// Progress: prep items are produced in increasing global index and consumed by
-// each spine in increasing chunk order; the oldest unfinished item never waits
-// on a younger one (its ring entry was freed by an older, already produced
-// item), so the pipeline cannot deadlock while all CTAs are resident.
+// Progress: a spine consumes its chunks in order; each of its preps produces
+// its share of them in order and only ever waits for that spine to free the
+// ring entry of an older chunk, so the oldest unfinished chunk of every spine
+// waits on nothing younger and the pipeline cannot deadlock while all CTAs
+// are resident.
+//
+// Registers: 16 warps at 128 registers each; warps 0-7 (state warps, prep
+// item groups) take 176 and warps 8-15 (single-thread roles, output warps)
+// keep 80, each warpgroup changing its allocation at the top of its role.
 #include <cuda.h>
 #include <string.h>
 #include <cuda_bf16.h>
