@@ -161,8 +161,10 @@ enum {
   PB_GATEF = 18,   // +2g+buf: gate block written (32, the loader warp)
   PB_STAGED = 22,  // +g: W | U^T staged (1)
   PB_DRAIN = 24,
-  PB_COUNT = 25
+  PB_GBFREE = 25,  // +2g+buf: gate block read by the bulk store (1, the store warp)
+  PB_COUNT = 29
 };
+static_assert(int(PB_COUNT) <= 32 && int(SB_COUNT) <= 32, "barrier area");
 
 // ---- TMEM columns
 // spine: [H^T W^T | O1^T] x2 (128 columns each), O2^T x2, dH^T (lane j = row j of H^T)
@@ -771,8 +773,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             agreed = false;
             break;
           }
-          if (leader) {
-            // the output warps are done with this parity's O1 / O2 (chunk c - 2)
+          if (leader && kLimbs == 1) {
+            // Vn' first, into the VO buffer's lower half (free: the output
+            // warps read only the upper half), so that the chain never waits
+            // for them; then O1 into the upper half once the output warps are
+            // done with chunk c - 2's O1 / O2 (OEMPTY)
+            tc_fence_after();
+            for (int kk = 0; kk < ksteps_d; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+              mma_bf16_ts(tmem + ST_VO + 128u * st, tmem + ST_VO + 128u * uint32_t(st ^ 1) + 8u * kk,
+                          make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_o2, kk > 0);
+            }
+            mma_commit(&bars[SB_VOFULL]);
+            if (c >= 2)
+              mbar_wait(&bars[SB_OEMPTY + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 16u, p.spin_limit);
+            tc_fence_after();
+            for (int kk = 0; kk < ksteps_d; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+              mma_bf16_ts(tmem + ST_VO + 128u * st + 64u,
+                          tmem + ST_VO + 128u * uint32_t(st ^ 1) + 8u * kk,
+                          make_sdesc_sw128(stg + STG_WQ + 8192 + off, 16, 1024), id_o2, kk > 0);
+            }
+            mma_commit(&bars[SB_AE + st]);
+          } else if (leader) {
+            // two limbs: the low limb sits in the Vn buffer, which the state
+            // warps overwrite right after VOFULL, so [W; Q] goes as one, after
+            // the output warps are done with chunk c - 2's O1 / O2 (OEMPTY)
             if (c >= 2)
               mbar_wait(&bars[SB_OEMPTY + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 16u, p.spin_limit);
             tc_fence_after();
@@ -1276,6 +1302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_store_commit();
           tma_store_wait_read<0>();
           mbar_arrive(&bars[PB_STORED + t]);
+          mbar_arrive(&bars[PB_GBFREE + 2 * g + (kg & 1)]);
           tma_store_wait_all<0>();
           fence_proxy_async_global();
           st_release_gpu(ready_flag(p, it.s, e), uint32_t(it.j + 1));
@@ -1289,14 +1316,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     } else if (warp == 11) {
       // ---------------- gate factors of item k (whole warp), into gate block
-      // kg & 1 of group k & 1 once item k - 3 is stored (so the block's last
-      // reader, the store of item k - 4, is done), beside the loader
+      // kg & 1 of group k & 1 once the store of item k - 4, the block's last
+      // reader, has read it (GBFREE), beside the loader
       PrepIter it;
       pi_start<kSeg>(it, p, sJ, iend, prank);
       bool ok = true;
       while (it.ok && ok) {
-        const int k = it.k, t = k % 3, g = k & 1, gb = (k >> 1) & 1;
-        ok = k < 3 || mbar_wait(&bars[PB_STORED + t], ((k / 3) & 1) ^ 1, abort_flag, err, 1u, p.spin_limit);
+        const int k = it.k, g = k & 1, gb = (k >> 1) & 1;
+        ok = k < 4 || mbar_wait(&bars[PB_GBFREE + 2 * g + gb], ((k >> 2) & 1) ^ 1, abort_flag, err, 1u,
+                                p.spin_limit);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
