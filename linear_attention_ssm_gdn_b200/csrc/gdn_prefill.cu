@@ -21,7 +21,7 @@
 //       P1 = [K;Q] K^T                                 (MMA)
 //       A[r][s]   = beta_r e^{G_r-G_s} k_r.k_s, s < r   (f32)
 //       Aqk[r][s] = scale e^{G_r-G_s} q_r.k_s, s <= r
-//       T = (I + A)^{-1}                               (blocked, f32, CUDA cores)
+//       T = (I + A)^{-1}                   (blocked, f32; larger products TF32 MMA)
 //       W^T = K^T (T diag(beta e^G))^T,  U^T = V^T (T diag(beta))^T   (MMAs)
 //     and bulk-store W (row-major), U^T, Aqk (bf16) and the gate factors into the
 //     owning spine's ring of kRing entries in the workspace (it stays in L2).
@@ -364,10 +364,36 @@ __device__ __forceinline__ void st_row64_bf16_lo(uint32_t tile, uint32_t row, co
 //      written over A_{2p+1,2p} once the pair has read it;
 //   3. X = A[32:64, 0:32] T[0:32, 0:32];
 //   4. T[32:64, 0:32] = -T[32:64, 32:64] X, written over A[32:64, 0:32].
-// The upper blocks stay the zeros of A.  Each thread of steps 2-4 owns a small
-// output tile.  bar_base: named barrier ids bar_base (128 threads),
-// bar_base+1+p (pairs).  X and the pair products use the 32x32 f32 scratch Xs.
+// Steps 3 and 4 (most of the arithmetic) run on the tensor cores as
+// warp-level m16n8k8 products with TF32 inputs and f32 accumulation, each
+// warp a 16x16 output tile: they read a quarter of the shared memory that
+// CUDA-core tiles would, and shared memory is what two item groups on one SM
+// compete for (a probe: 5371 -> 3781 cycles per inverse with both groups
+// busy).  TF32 keeps 10 mantissa bits, and T is rounded to bf16 (8 bits)
+// right after; on random inputs T differs from the f32 products by 7e-5
+// relative.  The upper blocks stay the zeros of A.  bar_base: named barrier
+// ids bar_base (128 threads), bar_base+1+p (pairs).  X and the pair products
+// use the 32x32 f32 scratch Xs.
 // ---------------------------------------------------------------------------
+// TF32 tensor-core products inside the blocked inverse: f32 -> tf32 (round
+// to nearest) and one warp-level m16n8k8 MMA with f32 accumulation.  The
+// fragments: A (16x8) a0 = (g, t), a1 = (g+8, t), a2 = (g, t+4), a3 = (g+8, t+4);
+// B (8x8) b0 = (t, g), b1 = (t+4, g); D (16x8) d0/d1 = (g, 2t / 2t+1), d2/d3 =
+// (g+8, 2t / 2t+1), with g = lane / 4 and t = lane % 4.
+__device__ __forceinline__ uint32_t f2tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ void invert_unit_lower64(float* M, float* Xs, int p, int bar_base) {
   const int w = p >> 5, ln = p & 31;
   // 1. diagonal blocks
@@ -437,61 +463,51 @@ __device__ __forceinline__ void invert_unit_lower64(float* M, float* Xs, int p, 
         make_float4(-z[0], -z[1], -z[2], -z[3]);
   }
   named_sync(bar_base, 128);
-  // 3. X = A[32:64, 0:32] T[0:32, 0:32]; thread p owns rows 2(p>>3)..+1, cols 4(p&7)..+3
-  const int r0 = 2 * (p >> 3), c0 = 4 * (p & 7);
+  // 3. X = A[32:64, 0:32] T[0:32, 0:32] and 4. T[32:64, 0:32] = -T[32:64, 32:64] X
+  //    on the tensor cores (m16n8k8, TF32 inputs, f32 accumulate): warp w
+  //    computes rows 16 (w >> 1) .., columns 16 (w & 1) .. of each product
+  const int wq = p >> 5, gq = (p & 31) >> 2, tq = p & 3;
+  const int mr = 16 * (wq >> 1), ncol = 16 * (wq & 1);
   {
-    float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* a0r = M + (32 + r0) * kAS;
-    const float* a1r = a0r + kAS;
-#pragma unroll 2
-    for (int k = 0; k < 32; k += 4) {
-      const float4 a0 = *reinterpret_cast<const float4*>(a0r + k);
-      const float4 a1 = *reinterpret_cast<const float4*>(a1r + k);
-      const float av0[4] = {a0.x, a0.y, a0.z, a0.w}, av1[4] = {a1.x, a1.y, a1.z, a1.w};
+    float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float4 tv = *reinterpret_cast<const float4*>(M + (k + m) * kAS + c0);
-        x0[0] = fmaf(av0[m], tv.x, x0[0]);
-        x0[1] = fmaf(av0[m], tv.y, x0[1]);
-        x0[2] = fmaf(av0[m], tv.z, x0[2]);
-        x0[3] = fmaf(av0[m], tv.w, x0[3]);
-        x1[0] = fmaf(av1[m], tv.x, x1[0]);
-        x1[1] = fmaf(av1[m], tv.y, x1[1]);
-        x1[2] = fmaf(av1[m], tv.z, x1[2]);
-        x1[3] = fmaf(av1[m], tv.w, x1[3]);
+    for (int k0 = 0; k0 < 32; k0 += 8) {
+      const float* ab = M + (32 + mr) * kAS + k0;
+      const uint32_t a0 = f2tf32(ab[gq * kAS + tq]), a1 = f2tf32(ab[(gq + 8) * kAS + tq]);
+      const uint32_t a2 = f2tf32(ab[gq * kAS + tq + 4]), a3 = f2tf32(ab[(gq + 8) * kAS + tq + 4]);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const float* bb = M + k0 * kAS + ncol + 8 * nt;
+        mma_tf32_16x8x8(d[nt], a0, a1, a2, a3, f2tf32(bb[tq * kAS + gq]), f2tf32(bb[(tq + 4) * kAS + gq]));
       }
     }
-    *reinterpret_cast<float4*>(Xs + r0 * 32 + c0) = make_float4(x0[0], x0[1], x0[2], x0[3]);
-    *reinterpret_cast<float4*>(Xs + (r0 + 1) * 32 + c0) = make_float4(x1[0], x1[1], x1[2], x1[3]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int cc = ncol + 8 * nt + 2 * tq;
+      *reinterpret_cast<float2*>(Xs + (mr + gq) * 32 + cc) = make_float2(d[nt][0], d[nt][1]);
+      *reinterpret_cast<float2*>(Xs + (mr + gq + 8) * 32 + cc) = make_float2(d[nt][2], d[nt][3]);
+    }
   }
   named_sync(bar_base, 128);  // A[32:64, 0:32] read, X complete
-  // 4. T[32:64, 0:32] = -T[32:64, 32:64] X  (T[32+r, 32+k] = 0 for k > r)
   {
-    float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* t0r = M + (32 + r0) * kAS + 32;
-    const float* t1r = t0r + kAS;
-#pragma unroll 2
-    for (int k = 0; k < 32; k += 4) {
-      const float4 a0 = *reinterpret_cast<const float4*>(t0r + k);
-      const float4 a1 = *reinterpret_cast<const float4*>(t1r + k);
-      const float av0[4] = {a0.x, a0.y, a0.z, a0.w}, av1[4] = {a1.x, a1.y, a1.z, a1.w};
+    float d[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float4 xv = *reinterpret_cast<const float4*>(Xs + (k + m) * 32 + c0);
-        z0[0] = fmaf(av0[m], xv.x, z0[0]);
-        z0[1] = fmaf(av0[m], xv.y, z0[1]);
-        z0[2] = fmaf(av0[m], xv.z, z0[2]);
-        z0[3] = fmaf(av0[m], xv.w, z0[3]);
-        z1[0] = fmaf(av1[m], xv.x, z1[0]);
-        z1[1] = fmaf(av1[m], xv.y, z1[1]);
-        z1[2] = fmaf(av1[m], xv.z, z1[2]);
-        z1[3] = fmaf(av1[m], xv.w, z1[3]);
+    for (int k0 = 0; k0 < 32; k0 += 8) {
+      const float* ab = M + (32 + mr) * kAS + 32 + k0;
+      const uint32_t a0 = f2tf32(ab[gq * kAS + tq]), a1 = f2tf32(ab[(gq + 8) * kAS + tq]);
+      const uint32_t a2 = f2tf32(ab[gq * kAS + tq + 4]), a3 = f2tf32(ab[(gq + 8) * kAS + tq + 4]);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const float* bb = Xs + k0 * 32 + ncol + 8 * nt;
+        mma_tf32_16x8x8(d[nt], a0, a1, a2, a3, f2tf32(bb[tq * 32 + gq]), f2tf32(bb[(tq + 4) * 32 + gq]));
       }
     }
-    *reinterpret_cast<float4*>(M + (32 + r0) * kAS + c0) =
-        make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
-    *reinterpret_cast<float4*>(M + (32 + r0 + 1) * kAS + c0) =
-        make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int cc = ncol + 8 * nt + 2 * tq;
+      *reinterpret_cast<float2*>(M + (32 + mr + gq) * kAS + cc) = make_float2(-d[nt][0], -d[nt][1]);
+      *reinterpret_cast<float2*>(M + (32 + mr + gq + 8) * kAS + cc) = make_float2(-d[nt][2], -d[nt][3]);
+    }
   }
   named_sync(bar_base, 128);
 }
