@@ -1152,13 +1152,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!named_all(gbar, 128, mbar_wait(&bars[PB_WUF + g], kg & 1, abort_flag, err, 4u, p.spin_limit))) break;
         tc_fence_after();
         {
-          uint8_t* wcol = set + G_W + uint32_t(pt >> 6) * 8192;
-          const uint32_t wbyte = uint32_t(pt & 63) * 2;
+          // U^T: TMEM lane pt is row pt of U^T, stored as it is.  W: TMEM lane
+          // pt is d_k column pt of W; 16 lanes x 16 chunk rows at a time in
+          // the 16x256b form, then transposing matrix stores write whole
+          // 16-byte row pieces of row-major W into its two 128B-swizzled boxes.
+          const int wq = warp & 3, sm = lane >> 3, sk = lane & 7;
+          const uint32_t wbase = smem_u32(set) + G_W;
 #pragma unroll 1
           for (int hf = 0; hf < 2; ++hf) {
-            float wv[32], uv[32];
-            tmem_ld32(tm + lane_off + PT_W + 32u * hf, wv);
+            float uv[32], wf[4][8];
             tmem_ld32(tm + lane_off + PT_U + 32u * hf, uv);
+#pragma unroll
+            for (int b4 = 0; b4 < 4; ++b4) {  // (lane half, 16-row block)
+              const uint32_t lb = uint32_t(32 * wq + 16 * (b4 & 1));
+              tmem_ld_16x256b_x2(tm + (lb << 16) + PT_W + 32u * hf + 16u * uint32_t(b4 >> 1), wf[b4]);
+            }
             tmem_ld_wait();
 #pragma unroll
             for (int hc = 0; hc < 4; ++hc) {
@@ -1170,9 +1178,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                              pack_bf16x2(uv[8 * hc + 6], uv[8 * hc + 7]));
             }
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              *reinterpret_cast<uint16_t*>(wcol + sw128_offset(uint32_t(32 * hf + i), wbyte)) =
-                  __bfloat16_as_ushort(__float2bfloat16_rn(wv[i]));
+            for (int b4 = 0; b4 < 4; ++b4) {
+              const float* x = wf[b4];
+              const int dk = 32 * wq + 16 * (b4 & 1) + 8 * (sm & 1);
+              const int row = 32 * hf + 16 * (b4 >> 1) + sk + 8 * (sm >> 1);
+              stmatrix_x4_trans(wbase + uint32_t(dk >> 6) * 8192u + uint32_t(row) * 128u +
+                                    (uint32_t(((dk & 63) >> 3) ^ (row & 7)) << 4),
+                                pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                                pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+            }
           }
           // Aqk into the set's V boxes (free once the U MMA is done), so that
           // the group's buffer is its own again for item k + 2
