@@ -1060,65 +1060,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         // ---- P1 row pt: K K^T (pt < 64) or Q K^T (pt >= 64), times e^{G_r - G_s}
         // (s <= r): two factors <= 1 for the blocks of s before r's 16-row
-        // block, a direct exponential inside it.
+        // block, a direct exponential inside it.  One 16-column block per
+        // pass of a loop kept rolled: the two 16-row halves of a warp take
+        // different branches, and unrolled code this size runs from a cold
+        // instruction cache.
         {
           const int r = pt & 63, rb = r >> 4;
           const float Gr = gt[PG_G + r];
           const float e1 = gt[PG_E1 + r];
-          const float br = gt[PG_BET + r];
+          const float rf = pt < 64 ? gt[PG_BET + r] : p.scale;
           const float* e2 = gt + PG_E2 + 64 * rb;
-          float v[64];
-          tmem_ld32(tm + lane_off + 64u * pb, *reinterpret_cast<float(*)[32]>(v));
-          tmem_ld32(tm + lane_off + 64u * pb + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-          tmem_ld_wait();
-          tc_fence_before();
-          mbar_arrive(&bars[PB_P1FREE + 2 * g + pb]);
-#pragma unroll
+#pragma unroll 1
           for (int sb = 0; sb < 4; ++sb) {
-            float f[16];
+            float v[16], f[16];
+            tmem_ld16(tm + lane_off + 64u * pb + 16u * uint32_t(sb), v);
+            tmem_ld_wait();
+            if (sb == 3) {
+              tc_fence_before();
+              mbar_arrive(&bars[PB_P1FREE + 2 * g + pb]);
+            }
+            const int s0 = 16 * sb;
+            // strict lower triangle for A, lower triangle with the diagonal for Aqk
+            const int lim = pt < 64 ? r - s0 - 1 : r - s0;
             if (sb < rb) {
 #pragma unroll
               for (int jj = 0; jj < 16; jj += 4) {
-                const float4 e4 = *reinterpret_cast<const float4*>(e2 + 16 * sb + jj);
-                f[jj] = e1 * e4.x;
-                f[jj + 1] = e1 * e4.y;
-                f[jj + 2] = e1 * e4.z;
-                f[jj + 3] = e1 * e4.w;
-              }
-            } else if (sb == rb) {
-#pragma unroll
-              for (int jj = 0; jj < 16; jj += 4) {
-                const int s2 = 16 * sb + jj;
-                const float4 g4 = *reinterpret_cast<const float4*>(gt + PG_G + s2);
-                f[jj] = (s2 <= r) ? __expf(Gr - g4.x) : 0.f;
-                f[jj + 1] = (s2 + 1 <= r) ? __expf(Gr - g4.y) : 0.f;
-                f[jj + 2] = (s2 + 2 <= r) ? __expf(Gr - g4.z) : 0.f;
-                f[jj + 3] = (s2 + 3 <= r) ? __expf(Gr - g4.w) : 0.f;
+                const float4 e4 = *reinterpret_cast<const float4*>(e2 + s0 + jj);
+                f[jj] = rf * e1 * e4.x;
+                f[jj + 1] = rf * e1 * e4.y;
+                f[jj + 2] = rf * e1 * e4.z;
+                f[jj + 3] = rf * e1 * e4.w;
               }
             } else {
 #pragma unroll
-              for (int jj = 0; jj < 16; ++jj) f[jj] = 0.f;
+              for (int jj = 0; jj < 16; jj += 4) {
+                const float4 g4 = *reinterpret_cast<const float4*>(gt + PG_G + s0 + jj);
+                f[jj] = jj <= lim ? rf * __expf(Gr - g4.x) : 0.f;
+                f[jj + 1] = jj + 1 <= lim ? rf * __expf(Gr - g4.y) : 0.f;
+                f[jj + 2] = jj + 2 <= lim ? rf * __expf(Gr - g4.z) : 0.f;
+                f[jj + 3] = jj + 3 <= lim ? rf * __expf(Gr - g4.w) : 0.f;
+              }
             }
             if (pt < 64) {  // A[r][s] = beta_r e^{G_r-G_s} k_r.k_s, s < r
 #pragma unroll
-              for (int jj = 0; jj < 16; jj += 4) {
-                const int s2 = 16 * sb + jj;
-                *reinterpret_cast<float4*>(M + r * kAS + s2) = make_float4(
-                    s2 + 0 < r ? br * f[jj] * v[s2] : 0.f,
-                    s2 + 1 < r ? br * f[jj + 1] * v[s2 + 1] : 0.f,
-                    s2 + 2 < r ? br * f[jj + 2] * v[s2 + 2] : 0.f,
-                    s2 + 3 < r ? br * f[jj + 3] * v[s2 + 3] : 0.f);
-              }
+              for (int jj = 0; jj < 16; jj += 4)
+                *reinterpret_cast<float4*>(M + r * kAS + s0 + jj) =
+                    make_float4(f[jj] * v[jj], f[jj + 1] * v[jj + 1], f[jj + 2] * v[jj + 2],
+                                f[jj + 3] * v[jj + 3]);
             } else {  // Aqk[r][s] = scale e^{G_r-G_s} q_r.k_s, s <= r  (bf16, swizzled)
-              const float sc = p.scale;
 #pragma unroll
               for (int hc = 0; hc < 2; ++hc) {
-                const int s2 = 16 * sb + 8 * hc, o = 8 * hc;
+                const int o = 8 * hc;
                 *reinterpret_cast<uint4*>(ga + GA_AQK + sw128_offset(r, (2 * sb + hc) * 16)) =
-                    make_uint4(pack_bf16x2(sc * f[o] * v[s2], sc * f[o + 1] * v[s2 + 1]),
-                               pack_bf16x2(sc * f[o + 2] * v[s2 + 2], sc * f[o + 3] * v[s2 + 3]),
-                               pack_bf16x2(sc * f[o + 4] * v[s2 + 4], sc * f[o + 5] * v[s2 + 5]),
-                               pack_bf16x2(sc * f[o + 6] * v[s2 + 6], sc * f[o + 7] * v[s2 + 7]));
+                    make_uint4(pack_bf16x2(f[o] * v[o], f[o + 1] * v[o + 1]),
+                               pack_bf16x2(f[o + 2] * v[o + 2], f[o + 3] * v[o + 3]),
+                               pack_bf16x2(f[o + 4] * v[o + 4], f[o + 5] * v[o + 5]),
+                               pack_bf16x2(f[o + 6] * v[o + 6], f[o + 7] * v[o + 7]));
               }
             }
           }
