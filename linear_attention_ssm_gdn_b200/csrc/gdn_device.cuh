@@ -234,8 +234,6 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
-// Arrive on `bar` once every previously issued tcgen05.mma of this thread has
-// completed (implicitly a tcgen05.fence::before_thread_sync).
 // Same, with A read from tensor memory: row m of A in lane m, two bf16
 // elements (k, k + 1) per 32-bit column, k along the columns from a_tmem.
 __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
@@ -248,6 +246,8 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// Arrive on `bar` once every previously issued tcgen05.mma of this thread has
+// completed (implicitly a tcgen05.fence::before_thread_sync).
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(

@@ -52,6 +52,7 @@
 // keep 80, each warpgroup changing its allocation at the top of its role.
 #include <cuda.h>
 #include <string.h>
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -97,12 +98,14 @@ constexpr uint32_t STG_WQ = 0, STG_K = 32768, STG_U = 49152, STG_AQK = 65536, ST
 constexpr uint32_t STG_BYTES = 74752;  // 73 KB
 constexpr uint32_t S_STG = 0;
 constexpr uint32_t S_OT = S_STG + 2 * STG_BYTES;  // outputs, 2 chunks x 64 rows x d_v bf16
-constexpr uint32_t S_VN = S_OT + 32768;           // Vn^T bf16 [128 x 128B]
-constexpr uint32_t S_VNS = S_VN + 16384;          // e^{G_C - G_r} Vn^T bf16
-constexpr uint32_t S_EG = S_VNS + 16384;          // 4 x 64 f32: scale e^{G_r} per chunk
+constexpr uint32_t S_VN = S_OT + 32768;           // two limbs: the low limb of H^T, bf16,
+constexpr uint32_t S_VNS = S_VN + 16384;          //   [128 x 128B] per 64 d_k (S_VN, S_VNS)
+constexpr uint32_t S_ID = S_VNS + 16384;          // the 64x64 identity, bf16 [64 x 128B]
+constexpr uint32_t S_EG = S_ID + 8192;            // 4 x 64 f32: -scale e^{G_r} per chunk
 constexpr uint32_t S_ECG = S_EG + 1024;           // 2 x 64 f32: e^{G_C - G_r} per chunk
 constexpr uint32_t S_BARS = S_ECG + 512;
-static_assert(S_OT % 1024 == 0 && STG_BYTES % 1024 == 0, "swizzled tiles are 1024-aligned");
+static_assert(S_OT % 1024 == 0 && STG_BYTES % 1024 == 0 && S_ID % 1024 == 0,
+              "swizzled tiles are 1024-aligned");
 static_assert(STG_GATE + G_GATE_BYTES <= STG_BYTES, "stage layout");
 // ---- prep shared memory: two 128-thread item groups (item k: group k & 1)
 // and three tile sets that rotate over the items (item k: set k % 3), so that
@@ -329,17 +332,9 @@ __device__ __forceinline__ void pi_align(PrepIter& it, const Params& p, const in
   while (it.ok && (it.k & 1) != w) pi_next<kSeg>(it, p, sJ, iend);
 }
 
-// Write 64 bf16 values as a 128-byte row of a 128B-swizzled tile (local smem).
-__device__ __forceinline__ void st_row64_bf16(uint32_t tile, uint32_t row, const float* x) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c)
-    st_shared_v4(tile + sw128_offset(row, c * 16), pack_bf16x2(x[8 * c + 0], x[8 * c + 1]),
-                 pack_bf16x2(x[8 * c + 2], x[8 * c + 3]), pack_bf16x2(x[8 * c + 4], x[8 * c + 5]),
-                 pack_bf16x2(x[8 * c + 6], x[8 * c + 7]));
-}
-
-// The low bf16 limb of 64 f32 values: x - bf16(x), rounded to bf16, as one
-// 128-byte row of a 128B-swizzled tile (the second limb of the state copy).
+// The low bf16 limb of 64 f32 values: x - bf16(x) (exact in f32), rounded to
+// bf16, as one 128-byte row of a 128B-swizzled tile (the second limb of the
+// state copy).
 __device__ __forceinline__ void st_row64_bf16_lo(uint32_t tile, uint32_t row, const float* x) {
   float r[8];
 #pragma unroll
@@ -518,8 +513,8 @@ using namespace pf;
 
 // kLimbs = 1: the state enters the H-dependent MMA as one bf16 copy; 2: as
 // two bf16 limbs hi + lo (page "ssm_gdn_tc_route.rs": the _tcfuse spine uses
-// one limb of S_c, the _tcfuse_x2 spine two), the low limb staged in the Vn
-// buffers, which that MMA does not read.
+// one limb of S_c, the _tcfuse_x2 spine two), the low limb staged in shared
+// memory.
 template <int kLimbs, bool kSeg>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -550,6 +545,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (uint32_t i = tid * 16; i < kSmemBytes; i += kThreads * 16)
     *reinterpret_cast<uint4*>(smem + i) = make_uint4(0, 0, 0, 0);
   __syncthreads();
+  if (spine && tid < C) {  // the identity's diagonal (bf16 1.0), for the tensor cores
+    *reinterpret_cast<uint16_t*>(smem + S_ID + sw128_offset(uint32_t(tid), uint32_t(2 * tid))) = 0x3F80u;
+    fence_proxy_async_smem();
+  }
   if (tid == 0) {
     if (spine) {
       for (int b = 0; b < SB_COUNT; ++b) mbar_init(&bars[b], 1u);
@@ -601,10 +600,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (row j of H^T) and half hh = w >> 2: columns d_k 64 hh .. 64 hh + 63 of
       // H^T (kept in registers, f32) and chunk rows 32 hh .. 32 hh + 31 of Vn^T
       // and of the outputs.  Per chunk c:
-      //   H <- e^{G_C} H + dH (dH of chunk c-1, from TMEM); bf16 copy -> TMEM;
-      //   [Vn' | O1]^T = H^T [W; Q]^T  (one N = 128 MMA);
-      //   Vn = U - Vn' -> Vn^T, e^{G_C - G_r} Vn^T (bf16);
-      //   dH = Vns^T K,  O2^T = Vn^T Aqk^T;
+      //   H <- e^{G_C} H + dH (dH of chunk c-1, from TMEM); H^T in bf16 -> TMEM;
+      //   Vn^T = U^T - H^T W^T: B negated, accumulated onto U^T I (issued
+      //   before the barrier, off this chain);
+      //   Vn^T, e^{G_C - G_r} Vn^T in bf16 -> TMEM, in place;
+      //   dH^T = Vns^T K,  O2^T = Vn^T Aqk^T  (A operands from TMEM), then
+      //   O1^T = H^T Q^T off the chain;
       // warp 9 issues the MMAs right after the two named barriers; the
       // outputs are the output warps' (12 - 15), off this chain.
       const int qd = warp & 3, hh = warp >> 2;
@@ -663,8 +664,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           else if (tid < 128) ecg_s[64 * st + tid - 64] = sg[tid];
           {
             // bf16 H^T row j, d_k 64 hh .. + 63, as the A operand of the [W; Q]
-            // MMA in tensor memory: the Vn' columns of the other VO buffer
-            // (read out in the previous chunk; its O1 half is left alone)
+            // MMAs in tensor memory: the Vn columns of the other VO buffer,
+            // where the previous chunk's bf16 Vn, Vns were read by its dH and
+            // O2 (DHFULL covers both); its O1 half is left alone
             uint32_t hp[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) hp[i] = pack_bf16x2(H[2 * i], H[2 * i + 1]);
@@ -672,64 +674,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_wait();
           }
           if constexpr (kLimbs == 2) {
-            // the previous chunk's O2 MMA reads the Vn buffers: done first
-            if (c > c_first)
-              ok = mbar_wait(&bars[SB_OFULL + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag, err,
-                             16u, p.spin_limit) && ok;
+            // the previous chunk's O1, issued after DHFULL, reads the low limb
+            if (c > 0)
+              ok = mbar_wait(&bars[SB_OFULL + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag, err, 16u,
+                             p.spin_limit) && ok;
             st_row64_bf16_lo(sbase + S_VN + uint32_t(hh) * 16384, uint32_t(j), H);
+            fence_proxy_async_smem();
           }
-          fence_proxy_async_smem();
           tc_fence_before();
           if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts [W; Q]
             agreed = false;
             break;
           }
-          // Vn = U - Vn'  ->  Vn^T and e^{G_C - G_r} Vn^T rows in bf16
+          // Vn^T (f32, chunk rows 32 hh .. + 31) -> bf16 Vn^T and
+          // e^{G_C - G_r} Vn^T in its own 32 columns: the A operands of O2 and
+          // dH, k-steps 2 hh and 2 hh + 1 (Vn at +0, +8; Vns at +16, +24)
           ok = mbar_wait(&bars[SB_VOFULL], c & 1, abort_flag, err, 16u, p.spin_limit) && ok;
-          ok = mbar_wait(&bars[SB_BF + st], (c >> 1) & 1, abort_flag, err, 16u, p.spin_limit) && ok;
           tc_fence_after();
           {
-            const uint8_t* urow = smem + S_STG + st * STG_BYTES + STG_U;
-            const float* ecp = ecg_s + 64 * st;
+            const float* ecp = ecg_s + 64 * st + 32 * hh;
+            const uint32_t vcol = tmem + lane_off + ST_VO + 128u * uint32_t(st) + 32u * uint32_t(hh);
             float vn[32];
-            tmem_ld32(tmem + lane_off + ST_VO + 128u * st + 32u * uint32_t(hh), vn);
+            uint32_t pk[32];
+            tmem_ld32(vcol, vn);
             tmem_ld_wait();
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              // two 8-column chunks: loads first, then the shared stores
-              uint4 uvs[2];
-              float4 eca[2], ecb[2];
-#pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                const int cc = 4 * hh + 2 * h2 + q;
-                uvs[q] = *reinterpret_cast<const uint4*>(urow + sw128_offset(j, cc * 16));
-                eca[q] = *reinterpret_cast<const float4*>(ecp + 8 * cc);
-                ecb[q] = *reinterpret_cast<const float4*>(ecp + 8 * cc + 4);
-              }
-#pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                const int hc = 2 * h2 + q, cc = 4 * hh + hc;
-                const float4 e0 = eca[q], e1 = ecb[q];
-                const float ec[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-                const uint32_t uw[4] = {uvs[q].x, uvs[q].y, uvs[q].z, uvs[q].w};
-                float x[8], y[8];
-#pragma unroll
-                for (int k2 = 0; k2 < 4; ++k2) {
-                  x[2 * k2] = __uint_as_float(uw[k2] << 16) - vn[8 * hc + 2 * k2];
-                  x[2 * k2 + 1] = __uint_as_float(uw[k2] & 0xFFFF0000u) - vn[8 * hc + 2 * k2 + 1];
-                }
-#pragma unroll
-                for (int m = 0; m < 8; ++m) y[m] = x[m] * ec[m];
-                st_shared_v4(sbase + S_VN + sw128_offset(j, cc * 16), pack_bf16x2(x[0], x[1]),
-                             pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                             pack_bf16x2(x[6], x[7]));
-                st_shared_v4(sbase + S_VNS + sw128_offset(j, cc * 16), pack_bf16x2(y[0], y[1]),
-                             pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                             pack_bf16x2(y[6], y[7]));
-              }
+            for (int i4 = 0; i4 < 8; ++i4) {
+              const float4 e = *reinterpret_cast<const float4*>(ecp + 4 * i4);
+              pk[2 * i4] = pack_bf16x2(vn[4 * i4], vn[4 * i4 + 1]);
+              pk[2 * i4 + 1] = pack_bf16x2(vn[4 * i4 + 2], vn[4 * i4 + 3]);
+              pk[16 + 2 * i4] = pack_bf16x2(e.x * vn[4 * i4], e.y * vn[4 * i4 + 1]);
+              pk[17 + 2 * i4] = pack_bf16x2(e.z * vn[4 * i4 + 2], e.w * vn[4 * i4 + 3]);
             }
+            tmem_st32u(vcol, pk);
+            tmem_st_wait();
           }
-          fence_proxy_async_smem();
           tc_fence_before();
           if (!named_all(1, kSpineSync, ok)) {  // the issuer warp starts dH, O2
             agreed = false;
@@ -771,91 +750,99 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (warp == 9) {
       // ---------------- issuer: joins the state warps' two barriers per chunk
       // (bar.red: every participant gets the same outcome) and issues
-      //   after the first:  [Vn' | O1]^T = H^T [W; Q]^T              (N = 128)
-      //   after the second: dH^T = Vns^T K (fresh), O2^T = Vn^T Aqk^T
-      const uint32_t id_vo = make_idesc_bf16(128, 128, 0, 0);
-      const uint32_t id_dh = make_idesc_bf16(128, 128, 0, 1);
-      const uint32_t id_o2 = make_idesc_bf16(128, 64, 0, 0);
+      //   before the first:  Vn^T := U^T I, once chunk c-1's O1 (the last MMA
+      //                      that read this buffer) is done
+      //   after the first:   Vn^T += H^T (-W)^T
+      //   after the second:  dH^T = Vns^T K (fresh), O2^T = Vn^T Aqk^T (DHFULL
+      //                      covers both), then O1^T = H^T Q^T off the chain
+      // One thread issues everything, so the stream is kept short: the
+      // shared-memory descriptors are built once and offset per k-step, and
+      // the k-step loops have compile-time trip counts.
       const bool leader = lane == 0;
-      int c = 0;
-      for (int u = s; u < units; u += p.S) {
-        int tb, te;
-        seq_range<kSeg>(p, u / p.H_v, tb, te);
-        bool agreed = true;
-        for (int t0 = tb; t0 < te; t0 += C, ++c) {
-          const int st = c & 1;
-          const uint32_t stg = sbase + S_STG + uint32_t(st) * STG_BYTES;
-          if (!named_all(1, kSpineSync, true)) {
-            agreed = false;
-            break;
-          }
-          if (leader && kLimbs == 1) {
-            // Vn' first, into the VO buffer's lower half (free: the output
-            // warps read only the upper half), so that the chain never waits
-            // for them; then O1 into the upper half once the output warps are
-            // done with chunk c - 2's O1 / O2 (OEMPTY)
-            tc_fence_after();
-            for (int kk = 0; kk < ksteps_d; ++kk) {
-              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_bf16_ts(tmem + ST_VO + 128u * st, tmem + ST_VO + 128u * uint32_t(st ^ 1) + 8u * kk,
-                          make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_o2, kk > 0);
-            }
-            mma_commit(&bars[SB_VOFULL]);
-            if (c >= 2)
-              mbar_wait(&bars[SB_OEMPTY + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 16u, p.spin_limit);
-            tc_fence_after();
-            for (int kk = 0; kk < ksteps_d; ++kk) {
-              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_bf16_ts(tmem + ST_VO + 128u * st + 64u,
-                          tmem + ST_VO + 128u * uint32_t(st ^ 1) + 8u * kk,
-                          make_sdesc_sw128(stg + STG_WQ + 8192 + off, 16, 1024), id_o2, kk > 0);
-            }
-            mma_commit(&bars[SB_AE + st]);
-          } else if (leader) {
-            // two limbs: the low limb sits in the Vn buffer, which the state
-            // warps overwrite right after VOFULL, so [W; Q] goes as one, after
-            // the output warps are done with chunk c - 2's O1 / O2 (OEMPTY)
-            if (c >= 2)
-              mbar_wait(&bars[SB_OEMPTY + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 16u, p.spin_limit);
-            tc_fence_after();
-            for (int kk = 0; kk < ksteps_d; ++kk) {
-              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_bf16_ts(tmem + ST_VO + 128u * st, tmem + ST_VO + 128u * uint32_t(st ^ 1) + 8u * kk,
-                          make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_vo, kk > 0);
-            }
-            if constexpr (kLimbs == 2) {
-              for (int kk = 0; kk < ksteps_d; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16_ss(tmem + ST_VO + 128u * st, make_sdesc_sw128(sbase + S_VN + off, 16, 1024),
-                            make_sdesc_sw128(stg + STG_WQ + off, 16, 1024), id_vo, 1u);
+      const uint64_t dsw = make_sdesc_sw128(0, 16, 1024);    // K-major operands
+      const uint64_t dswk = make_sdesc_sw128(0, 8192, 1024);  // K as the MN-major B of dH
+      auto walk = [&](auto ks_tag) {
+        constexpr int KS = decltype(ks_tag)::value;  // k-steps over d_k
+        constexpr uint32_t id_dh = make_idesc_bf16(128, 128, 0, 1);
+        constexpr uint32_t id_n64 = make_idesc_bf16(128, 64, 0, 0);
+        constexpr uint32_t id_vn = make_idesc_bf16(128, 64, 0, 0, 1);  // B negated
+        int c = 0;
+        for (int u = s; u < units; u += p.S) {
+          int tb, te;
+          seq_range<kSeg>(p, u / p.H_v, tb, te);
+          for (int t0 = tb; t0 < te; t0 += C, ++c) {
+            const int st = c & 1;
+            const uint32_t stg4 = (sbase + S_STG + uint32_t(st) * STG_BYTES) >> 4;
+            const uint32_t vo = tmem + ST_VO + 128u * uint32_t(st);       // Vn | O1 of this chunk
+            const uint32_t hs = tmem + ST_VO + 128u * uint32_t(st ^ 1);  // H^T (bf16) for it
+            bool okw = true;
+            if (leader) {
+              if (c > 0)
+                okw = mbar_wait(&bars[SB_OFULL + (st ^ 1)], ((c - 1) >> 1) & 1, abort_flag, err, 16u,
+                                p.spin_limit);
+              okw = okw && mbar_wait(&bars[SB_BF + st], (c >> 1) & 1, abort_flag, err, 16u, p.spin_limit);
+              if (okw) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_bf16_ss(vo, dsw + (stg4 + (STG_U >> 4) + 2 * kk),
+                              dsw + ((sbase + S_ID) >> 4) + 2 * kk, id_n64, kk > 0);
               }
             }
-            mma_commit(&bars[SB_VOFULL]);
-            mma_commit(&bars[SB_AE + st]);
+            okw = __shfl_sync(0xffffffffu, okw, 0);
+            if (!named_all(1, kSpineSync, okw)) return false;
+            if (leader) {
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < KS; ++kk) {
+                const uint32_t off4 = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+                mma_bf16_ts(vo, hs + 8u * kk, dsw + (stg4 + (STG_WQ >> 4) + off4), id_vn, 1u);
+                if constexpr (kLimbs == 2)
+                  mma_bf16_ss(vo, dsw + (((sbase + S_VN) >> 4) + off4), dsw + (stg4 + (STG_WQ >> 4) + off4),
+                              id_vn, 1u);
+              }
+              mma_commit(&bars[SB_VOFULL]);
+            }
+            __syncwarp();
+            if (!named_all(1, kSpineSync, true)) return false;
+            if (leader) {
+              // O2 rewrites chunk c - 2's O2, O1 its O1: read out by now
+              if (c >= 2)
+                mbar_wait(&bars[SB_OEMPTY + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 16u, p.spin_limit);
+              tc_fence_after();
+              // k-step kk: chunk rows 16 kk .. + 15, written by the state
+              // warps of half kk >> 1 at column 32 (kk >> 1) + 8 (kk & 1)
+              // (Vn), + 16 (Vns)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ts(tmem + ST_DH, vo + 32u * uint32_t(kk >> 1) + 16u + 8u * uint32_t(kk & 1),
+                            dswk + (stg4 + (STG_K >> 4) + 128 * kk), id_dh, kk > 0);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ts(tmem + ST_O2 + 64u * st, vo + 32u * uint32_t(kk >> 1) + 8u * uint32_t(kk & 1),
+                            dsw + (stg4 + (STG_AQK >> 4) + 2 * kk), id_n64, kk > 0);
+              mma_commit(&bars[SB_DHFULL]);
+              mma_commit(&bars[SB_BE + st]);
+#pragma unroll
+              for (int kk = 0; kk < KS; ++kk) {
+                const uint32_t off4 = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+                mma_bf16_ts(vo + 64u, hs + 8u * kk, dsw + (stg4 + ((STG_WQ + 8192) >> 4) + off4), id_n64,
+                            kk > 0);
+                if constexpr (kLimbs == 2)
+                  mma_bf16_ss(vo + 64u, dsw + (((sbase + S_VN) >> 4) + off4),
+                              dsw + (stg4 + ((STG_WQ + 8192) >> 4) + off4), id_n64, 1u);
+              }
+              mma_commit(&bars[SB_OFULL + st]);
+              mma_commit(&bars[SB_AE + st]);
+            }
+            __syncwarp();
           }
-          __syncwarp();
-          if (!named_all(1, kSpineSync, true)) {
-            agreed = false;
-            break;
-          }
-          if (leader) {
-            tc_fence_after();
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(tmem + ST_DH, make_sdesc_sw128(sbase + S_VNS + kk * 32, 16, 1024),
-                          make_sdesc_sw128(stg + STG_K + kk * 2048, 8192, 1024), id_dh, kk > 0);
-            mma_commit(&bars[SB_DHFULL]);
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(tmem + ST_O2 + 64u * st,
-                          make_sdesc_sw128(sbase + S_VN + kk * 32, 16, 1024),
-                          make_sdesc_sw128(stg + STG_AQK + kk * 32, 16, 1024), id_o2, kk > 0);
-            mma_commit(&bars[SB_OFULL + st]);
-            mma_commit(&bars[SB_BE + st]);
-          }
-          __syncwarp();
+          if (te > tb && !named_all(1, kSpineSync, true)) return false;  // the unit-end agreement
         }
-        if (!agreed) break;
-        if (te > tb && !named_all(1, kSpineSync, true)) break;  // the unit-end agreement
-      }
+        return true;
+      };
+      if (D == 128) walk(std::integral_constant<int, 8>{});
+      else walk(std::integral_constant<int, 4>{});
       if (leader) {  // every MMA this thread issued has completed
         mma_commit(&bars[SB_DRAIN]);
         mbar_wait(&bars[SB_DRAIN], 0, nullptr, err, 8u);
@@ -864,9 +851,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (warp == 8) {
       // ---------------- feeder: chunk c into stage c & 1, part by part.
       // Part A (Q by TMA; W and the gates from the ring entry) as soon as
-      // chunk c - 2's [W; Q] MMA is done; part B (K by TMA; U^T and Aqk) once
-      // chunk c - 2's dH and O2 are done, when its ring entry also goes back
-      // to the preps.
+      // chunk c - 2's [W; Q] MMAs are done; part B (K by TMA; U^T and Aqk)
+      // once chunk c - 2's dH and O2 are done, when its ring entry also goes
+      // back to the preps.
       if (lane == 0) {
         ChunkIter fd;
         it_start<kSeg>(fd, p, s);
@@ -889,7 +876,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int b = 0; b < nbox; ++b)
             tma_load_3d(stg + STG_WQ + b * 16384 + 8192, &tm_q, fa, b * 64, hk, fd.t0);
           issued_a = cc + 1;
-          ok = poll_geq(ready_flag(p, s, cc % kRing), uint32_t(cc + 1), gabort, err, 1u, p.spin_limit);
+          // chunk cc - 2 fully consumed (its dH and O2 done): its ring entry
+          // goes back to the preps before this chunk's is awaited
+          if (cc >= 2) {
+            ok = mbar_wait(&bars[SB_BE + st], ((cc >> 1) & 1) ^ 1, abort_flag, err, 1u, p.spin_limit);
+            if (ok) st_release_gpu(free_flag(p, s, (cc - 2) % kRing), uint32_t(cc - 1));
+          }
+          ok = ok && poll_geq(ready_flag(p, s, cc % kRing), uint32_t(cc + 1), gabort, err, 1u, p.spin_limit);
           if (!ok) {  // the phase still completes once the Q tiles landed
             mbar_arrive(fa);
             break;
@@ -899,13 +892,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_load_g2s(stg + STG_WQ, src + G_W, 8192, fa);
           bulk_load_g2s(stg + STG_WQ + 16384, src + G_W + 8192, 8192, fa);
           bulk_load_g2s(stg + STG_GATE, src + G_GATE, G_GATE_BYTES, fa);
-          // ---- part B
-          if (cc >= 2) {
-            ok = mbar_wait(&bars[SB_BE + st], ((cc >> 1) & 1) ^ 1, abort_flag, err, 1u, p.spin_limit);
-            if (!ok) break;
-            // chunk cc - 2 is fully consumed: its ring entry may be reused
-            st_release_gpu(free_flag(p, s, (cc - 2) % kRing), uint32_t(cc - 1));
-          }
+          // ---- part B (its buffers freed with BE above)
           uint64_t* fb = &bars[SB_BF + st];
           mbar_arrive_expect_tx(fb, uint32_t(nbox) * 8192 + 16384 + 8192);
           for (int b = 0; b < nbox; ++b)
