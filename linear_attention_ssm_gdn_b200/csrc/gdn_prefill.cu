@@ -149,7 +149,8 @@ enum {
   SB_DHFULL = 9,   // dH = Vns^T K done (commit)
   SB_OFULL = 10,   // +buf: O2 (and so O1) done (commit)
   SB_DRAIN = 12,
-  SB_OEMPTY = 13,  // +buf: the output warps have read O1 / O2 of the chunk (1)
+  SB_OEMPTY = 13,  // +buf: the output warps have read O1 / O2 of the chunk and zeroed
+                   // the O1 half (1; once more at start-up)
   SB_COUNT = 15
 };
 // ---- barriers (prep).  Item k: group g = k & 1, kg = k >> 1 its index in
@@ -601,11 +602,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // H^T (kept in registers, f32) and chunk rows 32 hh .. 32 hh + 31 of Vn^T
       // and of the outputs.  Per chunk c:
       //   H <- e^{G_C} H + dH (dH of chunk c-1, from TMEM); H^T in bf16 -> TMEM;
-      //   Vn^T = U^T - H^T W^T: B negated, accumulated onto U^T I (issued
-      //   before the barrier, off this chain);
+      //   [Vn | -O1]^T = [U^T I | 0] - H^T [W; Q]^T: one N = 128 MMA with B
+      //   negated, accumulated onto U^T I (issued before the barrier, off
+      //   this chain) and onto the zeros the output warps left;
       //   Vn^T, e^{G_C - G_r} Vn^T in bf16 -> TMEM, in place;
-      //   dH^T = Vns^T K,  O2^T = Vn^T Aqk^T  (A operands from TMEM), then
-      //   O1^T = H^T Q^T off the chain;
+      //   dH^T = Vns^T K,  O2^T = Vn^T Aqk^T  (A operands from TMEM);
       // warp 9 issues the MMAs right after the two named barriers; the
       // outputs are the output warps' (12 - 15), off this chain.
       const int qd = warp & 3, hh = warp >> 2;
@@ -660,11 +661,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float dec_cur = sg[128];
           // part A is released after the [W; Q] MMA: keep the gate factors
-          if (tid < 64) eg_s[64 * (c & 3) + tid] = sg[tid] * p.scale;
+          // (the output factor negated: the MMA forms -O1)
+          if (tid < 64) eg_s[64 * (c & 3) + tid] = -(sg[tid] * p.scale);
           else if (tid < 128) ecg_s[64 * st + tid - 64] = sg[tid];
           {
             // bf16 H^T row j, d_k 64 hh .. + 63, as the A operand of the [W; Q]
-            // MMAs in tensor memory: the Vn columns of the other VO buffer,
+            // MMA in tensor memory: the Vn columns of the other VO buffer,
             // where the previous chunk's bf16 Vn, Vns were read by its dH and
             // O2 (DHFULL covers both); its O1 half is left alone
             uint32_t hp[32];
@@ -674,10 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_wait();
           }
           if constexpr (kLimbs == 2) {
-            // the previous chunk's O1, issued after DHFULL, reads the low limb
-            if (c > 0)
-              ok = mbar_wait(&bars[SB_OFULL + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag, err, 16u,
-                             p.spin_limit) && ok;
+            // the previous chunk's [W; Q] MMA read the low limb before VOFULL
             st_row64_bf16_lo(sbase + S_VN + uint32_t(hh) * 16384, uint32_t(j), H);
             fence_proxy_async_smem();
           }
@@ -750,14 +749,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (warp == 9) {
       // ---------------- issuer: joins the state warps' two barriers per chunk
       // (bar.red: every participant gets the same outcome) and issues
-      //   before the first:  Vn^T := U^T I, once chunk c-1's O1 (the last MMA
-      //                      that read this buffer) is done
-      //   after the first:   Vn^T += H^T (-W)^T
+      //   before the first:  Vn^T := U^T I, once the output warps have read
+      //                      chunk c-2 out of this buffer and zeroed its O1
+      //                      half (OEMPTY) and chunk c-1's [W; Q] MMA has read
+      //                      the H^T copy that sat in its Vn half
+      //   after the first:   [Vn | -O1]^T += H^T (-[W; Q])^T  (N = 128)
       //   after the second:  dH^T = Vns^T K (fresh), O2^T = Vn^T Aqk^T (DHFULL
-      //                      covers both), then O1^T = H^T Q^T off the chain
-      // One thread issues everything, so the stream is kept short: the
-      // shared-memory descriptors are built once and offset per k-step, and
-      // the k-step loops have compile-time trip counts.
+      //                      and OFULL cover both)
+      // A tcgen05.mma costs about the same to issue at N = 64 as at N = 128,
+      // and one thread issues everything, so the stream has few and wide
+      // MMAs; the shared-memory descriptors are built once and offset per
+      // k-step, and the k-step loops have compile-time trip counts.
       const bool leader = lane == 0;
       const uint64_t dsw = make_sdesc_sw128(0, 16, 1024);    // K-major operands
       const uint64_t dswk = make_sdesc_sw128(0, 8192, 1024);  // K as the MN-major B of dH
@@ -765,7 +767,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int KS = decltype(ks_tag)::value;  // k-steps over d_k
         constexpr uint32_t id_dh = make_idesc_bf16(128, 128, 0, 1);
         constexpr uint32_t id_n64 = make_idesc_bf16(128, 64, 0, 0);
-        constexpr uint32_t id_vn = make_idesc_bf16(128, 64, 0, 0, 1);  // B negated
+        constexpr uint32_t id_wq = make_idesc_bf16(128, 128, 0, 0, 1);  // B negated
         int c = 0;
         for (int u = s; u < units; u += p.S) {
           int tb, te;
@@ -777,9 +779,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t hs = tmem + ST_VO + 128u * uint32_t(st ^ 1);  // H^T (bf16) for it
             bool okw = true;
             if (leader) {
+              okw = mbar_wait(&bars[SB_OEMPTY + st], (c >> 1) & 1, abort_flag, err, 16u, p.spin_limit);
               if (c > 0)
-                okw = mbar_wait(&bars[SB_OFULL + (st ^ 1)], ((c - 1) >> 1) & 1, abort_flag, err, 16u,
-                                p.spin_limit);
+                okw = okw && mbar_wait(&bars[SB_VOFULL], (c - 1) & 1, abort_flag, err, 16u, p.spin_limit);
               okw = okw && mbar_wait(&bars[SB_BF + st], (c >> 1) & 1, abort_flag, err, 16u, p.spin_limit);
               if (okw) {
                 tc_fence_after();
@@ -796,19 +798,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int kk = 0; kk < KS; ++kk) {
                 const uint32_t off4 = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-                mma_bf16_ts(vo, hs + 8u * kk, dsw + (stg4 + (STG_WQ >> 4) + off4), id_vn, 1u);
+                mma_bf16_ts(vo, hs + 8u * kk, dsw + (stg4 + (STG_WQ >> 4) + off4), id_wq, 1u);
                 if constexpr (kLimbs == 2)
                   mma_bf16_ss(vo, dsw + (((sbase + S_VN) >> 4) + off4), dsw + (stg4 + (STG_WQ >> 4) + off4),
-                              id_vn, 1u);
+                              id_wq, 1u);
               }
               mma_commit(&bars[SB_VOFULL]);
+              mma_commit(&bars[SB_AE + st]);
             }
             __syncwarp();
             if (!named_all(1, kSpineSync, true)) return false;
             if (leader) {
-              // O2 rewrites chunk c - 2's O2, O1 its O1: read out by now
-              if (c >= 2)
-                mbar_wait(&bars[SB_OEMPTY + st], ((c >> 1) & 1) ^ 1, abort_flag, err, 16u, p.spin_limit);
               tc_fence_after();
               // k-step kk: chunk rows 16 kk .. + 15, written by the state
               // warps of half kk >> 1 at column 32 (kk >> 1) + 8 (kk & 1)
@@ -822,18 +822,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_bf16_ts(tmem + ST_O2 + 64u * st, vo + 32u * uint32_t(kk >> 1) + 8u * uint32_t(kk & 1),
                             dsw + (stg4 + (STG_AQK >> 4) + 2 * kk), id_n64, kk > 0);
               mma_commit(&bars[SB_DHFULL]);
-              mma_commit(&bars[SB_BE + st]);
-#pragma unroll
-              for (int kk = 0; kk < KS; ++kk) {
-                const uint32_t off4 = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-                mma_bf16_ts(vo + 64u, hs + 8u * kk, dsw + (stg4 + ((STG_WQ + 8192) >> 4) + off4), id_n64,
-                            kk > 0);
-                if constexpr (kLimbs == 2)
-                  mma_bf16_ss(vo + 64u, dsw + (((sbase + S_VN) >> 4) + off4),
-                              dsw + (stg4 + ((STG_WQ + 8192) >> 4) + off4), id_n64, 1u);
-              }
               mma_commit(&bars[SB_OFULL + st]);
-              mma_commit(&bars[SB_AE + st]);
+              mma_commit(&bars[SB_BE + st]);
             }
             __syncwarp();
           }
@@ -916,13 +906,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (warp >= 12) {
         // ---------------- output warps, off the chain: for every chunk c of
         // this spine, once OFULL(c), warp 12 + q reads TMEM lane quadrant q
-        // (d_v 32 q .. 32 q + 31) of O1^T (upper half of the VO buffer) and
+        // (d_v 32 q .. 32 q + 31) of -O1^T (upper half of the VO buffer) and
         // O2^T, 16 lanes x 16 chunk rows at a time in the 16x256b form, forms
         // o_r = scale e^{G_r} O1[r] + O2[r] in bf16 and writes it with
         // transposing matrix stores into the output tile of the chunk's
         // parity: two 64-column halves of [64 rows][128 B], 16-byte chunks
         // swizzled by row (the tensor stores' 128-byte swizzle).  Then it
-        // hands the TMEM buffers back to the issuer (OEMPTY), and one thread
+        // zeroes the O1 half (the next [W; Q] MMA into this buffer
+        // accumulates onto it), hands the TMEM buffers back to the issuer
+        // (OEMPTY; both buffers once at start-up, zeroed), and one thread
         // stores the full 16-row blocks with TMA tensor stores; the rows of a
         // ragged block go out with plain stores.  A tile is rewritten two
         // chunks later, and the storing thread sees every earlier store
@@ -933,6 +925,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float* eg_s = reinterpret_cast<const float*>(smem + S_EG);
         const bool elect = warp == 12 && lane == 0;
         const int halves = D / 64;
+        const uint32_t zeros[32] = {};
+        const uint32_t o1q = tmem + (uint32_t(32 * qd) << 16) + ST_VO + 64u;  // + 128 ob: O1 half
+        for (int ob = 0; ob < 2; ++ob) {
+          tmem_st32u(o1q + 128u * uint32_t(ob), zeros);
+          tmem_st32u(o1q + 128u * uint32_t(ob) + 32u, zeros);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        named_sync(2, 128);
+        if (elect) {
+          mbar_arrive(&bars[SB_OEMPTY]);
+          mbar_arrive(&bars[SB_OEMPTY + 1]);
+        }
         int c = 0;
         bool ok = true;
         for (int u = s; u < units && ok; u += p.S) {
@@ -981,6 +986,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (okc) stmatrix_x4_trans(addr, m0, m1, m2, m3);
               }
             }
+            tmem_st32u(o1q + 128u * uint32_t(ob), zeros);
+            tmem_st32u(o1q + 128u * uint32_t(ob) + 32u, zeros);
+            tmem_st_wait();
             tc_fence_before();
             fence_proxy_async_smem();  // the tile, before the tensor stores read it
             if (elect) tma_store_wait_read<0>();  // the other tile's stores (chunk c - 1)
