@@ -1086,7 +1086,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 f[jj + 2] = rf * e1 * e4.z;
                 f[jj + 3] = rf * e1 * e4.w;
               }
-            } else {
+            } else if (sb == rb) {  // the row's own block: one exponential each
 #pragma unroll
               for (int jj = 0; jj < 16; jj += 4) {
                 const float4 g4 = *reinterpret_cast<const float4*>(gt + PG_G + s0 + jj);
@@ -1095,6 +1095,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 f[jj + 2] = jj + 2 <= lim ? rf * __expf(Gr - g4.z) : 0.f;
                 f[jj + 3] = jj + 3 <= lim ? rf * __expf(Gr - g4.w) : 0.f;
               }
+            } else {  // above the diagonal block: zeros, no exponentials
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj) f[jj] = 0.f;
             }
             if (pt < 64) {  // A[r][s] = beta_r e^{G_r-G_s} k_r.k_s, s < r
 #pragma unroll
