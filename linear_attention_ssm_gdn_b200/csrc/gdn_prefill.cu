@@ -360,14 +360,14 @@ __device__ __forceinline__ void st_row64_bf16_lo(uint32_t tile, uint32_t row, co
 //      written over A_{2p+1,2p} once the pair has read it;
 //   3. X = A[32:64, 0:32] T[0:32, 0:32];
 //   4. T[32:64, 0:32] = -T[32:64, 32:64] X, written over A[32:64, 0:32].
-// Steps 3 and 4 (most of the arithmetic) run on the tensor cores as
-// warp-level m16n8k8 products with TF32 inputs and f32 accumulation, each
-// warp a 16x16 output tile: they read a quarter of the shared memory that
-// CUDA-core tiles would, and shared memory is what two item groups on one SM
-// compete for (a probe: 5371 -> 3781 cycles per inverse with both groups
-// busy).  TF32 keeps 10 mantissa bits, and T is rounded to bf16 (8 bits)
-// right after; on random inputs T differs from the f32 products by 7e-5
-// relative.  The upper blocks stay the zeros of A.  bar_base: named barrier
+// Steps 2, 3 and 4 (most of the arithmetic) run on the tensor cores as
+// warp-level m16n8k8 products with TF32 inputs and f32 accumulation (steps 3
+// and 4: each warp a 16x16 output tile; step 2: each warp 16 rows x 8
+// columns): they read a quarter of the shared memory that CUDA-core tiles
+// would, and shared memory is what two item groups on one SM compete for (a
+// probe: 5371 -> 3781 cycles per inverse with both groups busy, steps 3 and
+// 4).  TF32 keeps 10 mantissa bits, and T is rounded to bf16 (8 bits) right
+// after; on random inputs T differs from the f32 products by 7e-5 relative.  The upper blocks stay the zeros of A.  bar_base: named barrier
 // ids bar_base (128 threads), bar_base+1+p (pairs).  X and the pair products
 // use the 32x32 f32 scratch Xs.
 // ---------------------------------------------------------------------------
@@ -415,48 +415,40 @@ __device__ __forceinline__ void invert_unit_lower64(float* M, float* Xs, int p, 
       for (int i = 0; i < 16; ++i) Tb[i * kAS] = x[i];
     }
   }
-  // 2. first sub-diagonal blocks, one per warp pair: thread t of the pair owns
-  //    row t>>2, columns 4(t&3)..+3
+  // 2. first sub-diagonal blocks, one per warp pair (blocks 2p, 2p+1), on
+  //    the tensor cores like steps 3 and 4: warp 2p + h computes columns
+  //    8 h .. 8 h + 7 of Y = A_{2p+1,2p} D_{2p} (into the pair's scratch),
+  //    then of -D_{2p+1} Y over A_{2p+1,2p} once the pair has read it
   {
-    const int pr = w >> 1, t = p & 63;
+    const int pr = w >> 1, h = w & 1;
     const int bi = 2 * pr + 1, bj = 2 * pr;
-    const int i = t >> 2, c4 = 4 * (t & 3);
-    float* Y = Xs + pr * 256;
+    const int gq = ln >> 2, tq = ln & 3;
+    float* Y = Xs + pr * 256;  // 16 x 16, row stride 16
     named_sync(bar_base + 1 + pr, 64);
-    float y[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* ar = M + (16 * bi + i) * kAS + 16 * bj;
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int l = 0; l < 16; l += 4) {
-      const float4 a = *reinterpret_cast<const float4*>(ar + l);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float4 d = *reinterpret_cast<const float4*>(M + (16 * bj + l + m) * kAS + 16 * bj + c4);
-        y[0] = fmaf(av[m], d.x, y[0]);
-        y[1] = fmaf(av[m], d.y, y[1]);
-        y[2] = fmaf(av[m], d.z, y[2]);
-        y[3] = fmaf(av[m], d.w, y[3]);
-      }
+    for (int k0 = 0; k0 < 16; k0 += 8) {
+      const float* ab = M + (16 * bi) * kAS + 16 * bj + k0;
+      const float* bb = M + (16 * bj + k0) * kAS + 16 * bj + 8 * h;
+      mma_tf32_16x8x8(d, f2tf32(ab[gq * kAS + tq]), f2tf32(ab[(gq + 8) * kAS + tq]),
+                      f2tf32(ab[gq * kAS + tq + 4]), f2tf32(ab[(gq + 8) * kAS + tq + 4]),
+                      f2tf32(bb[tq * kAS + gq]), f2tf32(bb[(tq + 4) * kAS + gq]));
     }
-    *reinterpret_cast<float4*>(Y + i * 16 + c4) = make_float4(y[0], y[1], y[2], y[3]);
-    named_sync(bar_base + 1 + pr, 64);  // A_{2p+1,2p} read by the pair
+    *reinterpret_cast<float2*>(Y + gq * 16 + 8 * h + 2 * tq) = make_float2(d[0], d[1]);
+    *reinterpret_cast<float2*>(Y + (gq + 8) * 16 + 8 * h + 2 * tq) = make_float2(d[2], d[3]);
+    named_sync(bar_base + 1 + pr, 64);  // Y complete, A_{2p+1,2p} read by the pair
     float z[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* dr = M + (16 * bi + i) * kAS + 16 * bi;
 #pragma unroll
-    for (int l = 0; l < 16; l += 4) {
-      const float4 a = *reinterpret_cast<const float4*>(dr + l);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float4 yv = *reinterpret_cast<const float4*>(Y + (l + m) * 16 + c4);
-        z[0] = fmaf(av[m], yv.x, z[0]);
-        z[1] = fmaf(av[m], yv.y, z[1]);
-        z[2] = fmaf(av[m], yv.z, z[2]);
-        z[3] = fmaf(av[m], yv.w, z[3]);
-      }
+    for (int k0 = 0; k0 < 16; k0 += 8) {
+      const float* ab = M + (16 * bi) * kAS + 16 * bi + k0;
+      const float* yb = Y + k0 * 16 + 8 * h;
+      mma_tf32_16x8x8(z, f2tf32(ab[gq * kAS + tq]), f2tf32(ab[(gq + 8) * kAS + tq]),
+                      f2tf32(ab[gq * kAS + tq + 4]), f2tf32(ab[(gq + 8) * kAS + tq + 4]),
+                      f2tf32(yb[tq * 16 + gq]), f2tf32(yb[(tq + 4) * 16 + gq]));
     }
-    *reinterpret_cast<float4*>(M + (16 * bi + i) * kAS + 16 * bj + c4) =
-        make_float4(-z[0], -z[1], -z[2], -z[3]);
+    float* tb = M + (16 * bi) * kAS + 16 * bj + 8 * h + 2 * tq;
+    *reinterpret_cast<float2*>(tb + gq * kAS) = make_float2(-z[0], -z[1]);
+    *reinterpret_cast<float2*>(tb + (gq + 8) * kAS) = make_float2(-z[2], -z[3]);
   }
   named_sync(bar_base, 128);
   // 3. X = A[32:64, 0:32] T[0:32, 0:32] and 4. T[32:64, 0:32] = -T[32:64, 32:64] X
