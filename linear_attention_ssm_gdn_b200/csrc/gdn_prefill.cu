@@ -10,8 +10,8 @@
 //     and run their per-chunk critical chain on tcgen05 MMAs with TMEM
 //     accumulators (M = d_v = 128 lanes), keeping H^T in registers (f32) and
 //     its bf16 copy in TMEM as the A operand of the first MMA:
-//       [Vn' | O1]^T = H^T [W; Q]^T,  Vn = U - Vn',
-//       H^T <- e^{G_C} H^T + (e^{G_C - G_r} Vn)^T K;
+//       [Vn | -O1]^T = [U^T | 0] - H^T [W; Q]^T   (U^T preloaded by U^T I),
+//       H^T <- e^{G_C} H^T + (e^{G_C - G_r} Vn)^T K   (Vn in bf16, from TMEM);
 //     a separate output warpgroup forms  o_r = e^{G_r} scale O1_r + (Aqk Vn)_r
 //     off that chain and stores it with TMA tensor stores;
 //   PREPS (all other CTAs) compute everything that does not depend on H, for
@@ -171,7 +171,9 @@ enum {
 static_assert(int(PB_COUNT) <= 32 && int(SB_COUNT) <= 32, "barrier area");
 
 // ---- TMEM columns
-// spine: [H^T W^T | O1^T] x2 (128 columns each), O2^T x2, dH^T (lane j = row j of H^T)
+// spine: [Vn^T | -O1^T] x2 (128 columns each; the Vn half also holds the bf16
+// copy of H^T for the next chunk, then bf16 Vn, Vns), O2^T x2, dH^T (lane j =
+// d_v row j)
 constexpr uint32_t ST_VO = 0, ST_O2 = 256, ST_DH = 384;
 constexpr uint32_t PT_W = 128, PT_U = 192, PT_WG = 256;  // prep, per group: P1 x2 at 0, 64
 
@@ -833,9 +835,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (warp == 8) {
       // ---------------- feeder: chunk c into stage c & 1, part by part.
       // Part A (Q by TMA; W and the gates from the ring entry) as soon as
-      // chunk c - 2's [W; Q] MMAs are done; part B (K by TMA; U^T and Aqk)
+      // chunk c - 2's [W; Q] MMA is done; part B (K by TMA; U^T and Aqk)
       // once chunk c - 2's dH and O2 are done, when its ring entry also goes
-      // back to the preps.
+      // back to the preps (before this chunk's entry is awaited).
       if (lane == 0) {
         ChunkIter fd;
         it_start<kSeg>(fd, p, s);
