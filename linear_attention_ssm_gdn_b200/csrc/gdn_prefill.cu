@@ -71,7 +71,7 @@ constexpr uint32_t kRegsWide = 176, kRegsNarrow = 80;  // warps 0-7 / warps 8-15
 static_assert(2 * 128 * kRegsWide + 2 * 128 * kRegsNarrow == 128 * kThreads,
               "the re-allocated registers add up to the launch's allocation");
 constexpr int kAS = 68;        // f32 row stride of the A / T scratch (16-byte rows)
-constexpr int kRing = 4;       // ring entries per spine
+constexpr int kRing = 8;       // ring entries per spine
 constexpr int kMaxSpines = 256;
 constexpr int kSpineSync = 288;  // the spine's per-chunk barriers: 8 state warps + the issuer warp
 // Largest rise of the cumulative gate within a chunk (G_r - G_s, s <= r) that
