@@ -171,10 +171,9 @@ enum {
 static_assert(int(PB_COUNT) <= 32 && int(SB_COUNT) <= 32, "barrier area");
 
 // ---- TMEM columns
-// spine: [Vn^T | -O1^T] x2 (128 columns each; the Vn half also holds the bf16
-// copy of H^T for the next chunk, then bf16 Vn, Vns), O2^T x2, dH^T (lane j =
-// d_v row j)
-constexpr uint32_t ST_VO = 0, ST_O2 = 256, ST_DH = 384;
+// spine: [Vn^T | -O1^T] x2 (128 columns each; the Vn half ends as bf16 Vn,
+// Vns), O2^T (64), the bf16 copy of H^T (64), dH^T (lane j = d_v row j)
+constexpr uint32_t ST_VO = 0, ST_O2 = 256, ST_HT = 320, ST_DH = 384;
 constexpr uint32_t PT_W = 128, PT_U = 192, PT_WG = 256;  // prep, per group: P1 x2 at 0, 64
 
 struct Params {
@@ -600,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       //   negated, accumulated onto U^T I (issued before the barrier, off
       //   this chain) and onto the zeros the output warps left;
       //   Vn^T, e^{G_C - G_r} Vn^T in bf16 -> TMEM, in place;
-      //   dH^T = Vns^T K,  O2^T = Vn^T Aqk^T  (A operands from TMEM);
+      //   dH^T = Vns^T K (A from TMEM); then, off this chain, O2^T = Vn^T Aqk^T;
       // warp 9 issues the MMAs right after the two named barriers; the
       // outputs are the output warps' (12 - 15), off this chain.
       const int qd = warp & 3, hh = warp >> 2;
@@ -660,13 +659,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           else if (tid < 128) ecg_s[64 * st + tid - 64] = sg[tid];
           {
             // bf16 H^T row j, d_k 64 hh .. + 63, as the A operand of the [W; Q]
-            // MMA in tensor memory: the Vn columns of the other VO buffer,
-            // where the previous chunk's bf16 Vn, Vns were read by its dH and
-            // O2 (DHFULL covers both); its O1 half is left alone
+            // MMA in tensor memory (the previous chunk's [W; Q] MMA, done
+            // before VOFULL, was the last reader)
             uint32_t hp[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) hp[i] = pack_bf16x2(H[2 * i], H[2 * i + 1]);
-            tmem_st32u(tmem + lane_off + ST_VO + 128u * uint32_t(st ^ 1) + 32u * uint32_t(hh), hp);
+            tmem_st32u(tmem + lane_off + ST_HT + 32u * uint32_t(hh), hp);
             tmem_st_wait();
           }
           if constexpr (kLimbs == 2) {
@@ -745,11 +743,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (bar.red: every participant gets the same outcome) and issues
       //   before the first:  Vn^T := U^T I, once the output warps have read
       //                      chunk c-2 out of this buffer and zeroed its O1
-      //                      half (OEMPTY) and chunk c-1's [W; Q] MMA has read
-      //                      the H^T copy that sat in its Vn half
+      //                      half (OEMPTY: its dH and O2 are done with the Vn
+      //                      half too)
       //   after the first:   [Vn | -O1]^T += H^T (-[W; Q])^T  (N = 128)
-      //   after the second:  dH^T = Vns^T K (fresh), O2^T = Vn^T Aqk^T (DHFULL
-      //                      and OFULL cover both)
+      //   after the second:  dH^T = Vns^T K (fresh), committed on its own
+      //                      (DHFULL: the chain goes on), then O2^T = Vn^T
+      //                      Aqk^T into the one O2 buffer once the output
+      //                      warps have read chunk c-1's (OEMPTY); OFULL
+      //                      covers both
       // A tcgen05.mma costs about the same to issue at N = 64 as at N = 128,
       // and one thread issues everything, so the stream has few and wide
       // MMAs; the shared-memory descriptors are built once and offset per
@@ -770,12 +771,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int st = c & 1;
             const uint32_t stg4 = (sbase + S_STG + uint32_t(st) * STG_BYTES) >> 4;
             const uint32_t vo = tmem + ST_VO + 128u * uint32_t(st);       // Vn | O1 of this chunk
-            const uint32_t hs = tmem + ST_VO + 128u * uint32_t(st ^ 1);  // H^T (bf16) for it
             bool okw = true;
             if (leader) {
               okw = mbar_wait(&bars[SB_OEMPTY + st], (c >> 1) & 1, abort_flag, err, 16u, p.spin_limit);
-              if (c > 0)
-                okw = okw && mbar_wait(&bars[SB_VOFULL], (c - 1) & 1, abort_flag, err, 16u, p.spin_limit);
               okw = okw && mbar_wait(&bars[SB_BF + st], (c >> 1) & 1, abort_flag, err, 16u, p.spin_limit);
               if (okw) {
                 tc_fence_after();
@@ -792,7 +790,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int kk = 0; kk < KS; ++kk) {
                 const uint32_t off4 = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-                mma_bf16_ts(vo, hs + 8u * kk, dsw + (stg4 + (STG_WQ >> 4) + off4), id_wq, 1u);
+                mma_bf16_ts(vo, tmem + ST_HT + 8u * kk, dsw + (stg4 + (STG_WQ >> 4) + off4), id_wq, 1u);
                 if constexpr (kLimbs == 2)
                   mma_bf16_ss(vo, dsw + (((sbase + S_VN) >> 4) + off4), dsw + (stg4 + (STG_WQ >> 4) + off4),
                               id_wq, 1u);
@@ -811,11 +809,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ts(tmem + ST_DH, vo + 32u * uint32_t(kk >> 1) + 16u + 8u * uint32_t(kk & 1),
                             dswk + (stg4 + (STG_K >> 4) + 128 * kk), id_dh, kk > 0);
+              mma_commit(&bars[SB_DHFULL]);
+              if (c > 0)  // chunk c-1's O2 read out
+                mbar_wait(&bars[SB_OEMPTY + (st ^ 1)], (((c - 1) >> 1) + 1) & 1, abort_flag, err, 16u,
+                          p.spin_limit);
+              tc_fence_after();
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ts(tmem + ST_O2 + 64u * st, vo + 32u * uint32_t(kk >> 1) + 8u * uint32_t(kk & 1),
+                mma_bf16_ts(tmem + ST_O2, vo + 32u * uint32_t(kk >> 1) + 8u * uint32_t(kk & 1),
                             dsw + (stg4 + (STG_AQK >> 4) + 2 * kk), id_n64, kk > 0);
-              mma_commit(&bars[SB_DHFULL]);
               mma_commit(&bars[SB_OFULL + st]);
               mma_commit(&bars[SB_BE + st]);
             }
@@ -954,7 +956,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t lb = uint32_t(32 * qd + 16 * hf);  // TMEM lane base (d_v)
                 if (int(lb) < D) {  // warp-uniform (d = 64: quadrants 2, 3 empty)
                   tmem_ld_16x256b_x2(tmem + (lb << 16) + ST_VO + 128u * uint32_t(ob) + 64u + uint32_t(r0), a1[hf]);
-                  tmem_ld_16x256b_x2(tmem + (lb << 16) + ST_O2 + 64u * uint32_t(ob) + uint32_t(r0), a2[hf]);
+                  tmem_ld_16x256b_x2(tmem + (lb << 16) + ST_O2 + uint32_t(r0), a2[hf]);
                 }
               }
               tmem_ld_wait();
